@@ -1,0 +1,430 @@
+/*
+ * oracle.c -- plain, slow fp64 CPU statement of one decode step of LLaMA-style
+ * attention against a paged KV cache.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product library links, loads or
+ * calls this file; only the tests, the smoke check and the CPU-baseline leg of
+ * the benchmark do.  It shares no code, header, table or constant with the
+ * CUDA path.
+ *
+ * Sources (three web pages on writing an LLM inference engine):
+ *   [ENGINE]  "为什么要自己动手写一个LLM推理引擎" (wzjinhao.cn/news/61427), chapter 1:
+ *             s3.4  KV-cache size formula, fixed 16/32-token pages from a free list,
+ *                   attention finds the cached block through the page index;
+ *             s4.2  RoPE puts the position into q and k through a rotation;
+ *             s4.3  forward with a KV cache: q/k/v views with n_heads / n_kv_heads,
+ *                   apply_rotary_emb(q, k, start_pos), append to the cache,
+ *                   scores q.k^T / sqrt(head_dim) + causal mask, softmax, times v;
+ *             s5.2  check a cache by disabling it and recomputing the whole sequence.
+ *   [FLOW]    "大模型推理全流程解析" (stapisi.com/news/4049481), s2.2.2: one query
+ *             against all cached keys, scaled, softmax, weighted sum of values.
+ *   [WEIGHTS] dpshk.com/news/4990443, s3.2: fp16 q.k products can overflow before the
+ *             softmax (so accumulate wide); s5.1: GQA gives k_proj n_kv_heads*head_dim.
+ *
+ * Storage values are IEEE binary16 or bfloat16 bit patterns (uint16); every
+ * function decodes them to double, computes in double, and (where the method
+ * stores a result) rounds once, to nearest-even, straight from double.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORA_F16 0
+#define ORA_BF16 1
+
+/* ------------------------------------------------------------------------- */
+/* storage formats                                                            */
+/* ------------------------------------------------------------------------- */
+
+/* IEEE 754 binary16: 1 sign, 5 exponent (bias 15), 10 fraction bits. */
+double ora_half_to_double(uint16_t h)
+{
+    int sign = (h >> 15) & 1;
+    int e = (h >> 10) & 0x1f;
+    int f = h & 0x3ff;
+    double v;
+    if (e == 0)
+        v = ldexp((double)f, -24);               /* subnormal: f * 2^-24 */
+    else if (e == 31)
+        v = f ? NAN : INFINITY;
+    else
+        v = ldexp((double)(1024 + f), e - 25);   /* 1.f * 2^(e-15) */
+    return sign ? -v : v;
+}
+
+/* bfloat16: the top 16 bits of an IEEE binary32 (8 exponent bits, bias 127). */
+double ora_bf16_to_double(uint16_t h)
+{
+    int sign = (h >> 15) & 1;
+    int e = (h >> 7) & 0xff;
+    int f = h & 0x7f;
+    double v;
+    if (e == 0)
+        v = ldexp((double)f, -133);              /* subnormal: f * 2^-133 */
+    else if (e == 255)
+        v = f ? NAN : INFINITY;
+    else
+        v = ldexp((double)(128 + f), e - 134);   /* 1.f * 2^(e-127) */
+    return sign ? -v : v;
+}
+
+/*
+ * Round a double to a binary format with `mbits` fraction bits and exponent
+ * bias `bias`, to nearest with ties to even, in one step.  Scaling by a power
+ * of two is exact, and rint() rounds to nearest-even in the default mode.
+ */
+static uint16_t round_to_format(double x, int mbits, int bias, int ebits)
+{
+    uint16_t sign = signbit(x) ? (uint16_t)(1u << 15) : 0;
+    int emax_field = (1 << ebits) - 1;
+    if (isnan(x))
+        return (uint16_t)(sign | (emax_field << mbits) | (1u << (mbits - 1)));
+    double a = fabs(x);
+    if (isinf(a))
+        return (uint16_t)(sign | (emax_field << mbits));
+    if (a == 0.0)
+        return sign;
+    int e2;
+    frexp(a, &e2);                   /* a = m * 2^e2, m in [0.5, 1) */
+    int E = e2 - 1;                  /* a = 1.x * 2^E */
+    int emin = 1 - bias;
+    double units;
+    long long bits;
+    if (E < emin) {
+        /* subnormal range: count units of 2^(emin - mbits) */
+        units = rint(ldexp(a, mbits - emin));
+        bits = (long long)units;     /* a carry into 2^mbits lands on the min normal */
+    } else {
+        units = rint(ldexp(a, mbits - E));          /* in [2^mbits, 2^(mbits+1)] */
+        bits = ((long long)(E + bias) << mbits) + (long long)units - (1ll << mbits);
+    }
+    if (bits >= ((long long)emax_field << mbits))
+        bits = (long long)emax_field << mbits;     /* overflow to infinity */
+    return (uint16_t)(sign | (uint16_t)bits);
+}
+
+uint16_t ora_double_to_half(double x) { return round_to_format(x, 10, 15, 5); }
+uint16_t ora_double_to_bf16(double x) { return round_to_format(x, 7, 127, 8); }
+
+static double dec(uint16_t h, int dtype)
+{
+    return dtype == ORA_BF16 ? ora_bf16_to_double(h) : ora_half_to_double(h);
+}
+
+static uint16_t enc(double x, int dtype)
+{
+    return dtype == ORA_BF16 ? ora_double_to_bf16(x) : ora_double_to_half(x);
+}
+
+void ora_decode_array(const uint16_t* src, double* dst, int64_t n, int dtype)
+{
+    for (int64_t i = 0; i < n; ++i) dst[i] = dec(src[i], dtype);
+}
+
+void ora_encode_array(const double* src, uint16_t* dst, int64_t n, int dtype)
+{
+    for (int64_t i = 0; i < n; ++i) dst[i] = enc(src[i], dtype);
+}
+
+/* ------------------------------------------------------------------------- */
+/* RoPE  [ENGINE] s4.2, s4.3                                                   */
+/* ------------------------------------------------------------------------- */
+
+/*
+ * Rotary position embedding of one token's heads, in double.
+ * x, y: [n_tokens][heads][head_dim].  Pair i of a head is (x[2i], x[2i+1]);
+ * it is turned by the angle pos * theta^(-2i/head_dim):
+ *   y[2i]   = x[2i] cos a - x[2i+1] sin a
+ *   y[2i+1] = x[2i] sin a + x[2i+1] cos a
+ * (the pages name a rotation applied at start_pos; the pairing and the
+ * frequency ladder are the ones the name apply_rotary_emb refers to).
+ */
+void ora_rope_f64(const double* x, double* y, const int32_t* positions,
+                  int n_tokens, int heads, int head_dim, double theta)
+{
+    for (int t = 0; t < n_tokens; ++t) {
+        for (int h = 0; h < heads; ++h) {
+            const double* xs = x + ((int64_t)t * heads + h) * head_dim;
+            double* ys = y + ((int64_t)t * heads + h) * head_dim;
+            for (int i = 0; i < head_dim / 2; ++i) {
+                double freq = pow(theta, -2.0 * i / head_dim);
+                double angle = (double)positions[t] * freq;
+                double c = cos(angle), s = sin(angle);
+                double x0 = xs[2 * i], x1 = xs[2 * i + 1];
+                ys[2 * i] = x0 * c - x1 * s;
+                ys[2 * i + 1] = x0 * s + x1 * c;
+            }
+        }
+    }
+}
+
+/* RoPE on storage values: decode, rotate in double, round once to the dtype.
+ * exact_out (optional) receives the unrounded doubles. */
+void ora_rope(const uint16_t* x, uint16_t* y, double* exact_out, const int32_t* positions,
+              int n_tokens, int heads, int head_dim, double theta, int dtype)
+{
+    int64_t n = (int64_t)n_tokens * heads * head_dim;
+    double* xd = (double*)malloc(sizeof(double) * (size_t)(n ? n : 1));
+    double* yd = (double*)malloc(sizeof(double) * (size_t)(n ? n : 1));
+    ora_decode_array(x, xd, n, dtype);
+    ora_rope_f64(xd, yd, positions, n_tokens, heads, head_dim, theta);
+    ora_encode_array(yd, y, n, dtype);
+    if (exact_out) memcpy(exact_out, yd, sizeof(double) * (size_t)n);
+    free(xd);
+    free(yd);
+}
+
+/* ------------------------------------------------------------------------- */
+/* page table  [ENGINE] s3.4                                                   */
+/* ------------------------------------------------------------------------- */
+
+/*
+ * Flat slot of the token at `position` of sequence b: the page that the page
+ * table names for logical page position/P, and the row position%P inside it.
+ * A negative position (a padded batch row) gives slot -1.
+ */
+void ora_slot_mapping(const int32_t* block_tables, int max_pages_per_seq,
+                      const int32_t* positions, int n, int page_size, int64_t* slots)
+{
+    for (int b = 0; b < n; ++b) {
+        int pos = positions[b];
+        if (pos < 0) {
+            slots[b] = -1;
+            continue;
+        }
+        int logical_page = pos / page_size;
+        int row = pos % page_size;
+        int64_t physical = block_tables[(int64_t)b * max_pages_per_seq + logical_page];
+        slots[b] = physical * page_size + row;
+    }
+}
+
+/*
+ * Cache update of one decode step for one layer ([ENGINE] s4.3 appends the new
+ * k and v behind the cached ones; s5.3 asks for a preallocated pool in place of
+ * concatenation).  pool: [num_pages][kv_heads][page_size][head_dim];
+ * k, v: [n][kv_heads][head_dim]; the token of row b goes to position positions[b]
+ * of sequence b.  Values are copied bit for bit.
+ */
+void ora_kv_append(uint16_t* k_pool, uint16_t* v_pool, const uint16_t* k, const uint16_t* v,
+                   const int32_t* block_tables, int max_pages_per_seq, const int32_t* positions,
+                   int n, int kv_heads, int page_size, int head_dim)
+{
+    for (int b = 0; b < n; ++b) {
+        int pos = positions[b];
+        if (pos < 0) continue;
+        int64_t page = block_tables[(int64_t)b * max_pages_per_seq + pos / page_size];
+        int row = pos % page_size;
+        for (int h = 0; h < kv_heads; ++h) {
+            for (int i = 0; i < head_dim; ++i) {
+                int64_t dst = ((page * kv_heads + h) * page_size + row) * head_dim + i;
+                int64_t src = ((int64_t)b * kv_heads + h) * head_dim + i;
+                k_pool[dst] = k[src];
+                v_pool[dst] = v[src];
+            }
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------- */
+/* attention                                                                   */
+/* ------------------------------------------------------------------------- */
+
+/*
+ * Copy the first `len` cached tokens of sequence b out of the pages into a
+ * contiguous [len][kv_heads][head_dim] array of doubles, in logical order: token
+ * t lives in page block_tables[b][t / P], row t % P ([ENGINE] s3.4).
+ */
+static void gather_sequence(const uint16_t* pool, const int32_t* block_tables, int max_pages_per_seq,
+                            int b, int len, int kv_heads, int page_size, int head_dim, int dtype,
+                            double* dst)
+{
+    for (int t = 0; t < len; ++t) {
+        int64_t page = block_tables[(int64_t)b * max_pages_per_seq + t / page_size];
+        int row = t % page_size;
+        for (int h = 0; h < kv_heads; ++h) {
+            const uint16_t* src = pool + ((page * kv_heads + h) * page_size + row) * head_dim;
+            for (int i = 0; i < head_dim; ++i)
+                dst[((int64_t)t * kv_heads + h) * head_dim + i] = dec(src[i], dtype);
+        }
+    }
+}
+
+/*
+ * Decode attention of one query token per sequence over its paged cache.
+ *   q:   [batch][q_heads][head_dim] (storage), already rotated;
+ *   pools: [num_pages][kv_heads][page_size][head_dim] (storage);
+ *   context_lens[b]: tokens in the cache, the new one included (0 = padded row);
+ *   out: [batch][q_heads][head_dim] double, before any rounding;
+ *   weights (optional): [batch][q_heads][max_len] softmax weights, 0 past len.
+ * For q head h the key/value head is h / (q_heads / kv_heads) (groups of
+ * consecutive query heads share one kv head, [ENGINE] s4.3 n_kv_heads).
+ * The single query sits at the last position, so the causal mask keeps every
+ * cached token.  Softmax is taken with the maximum subtracted.
+ */
+void ora_decode_attention(const uint16_t* q, const uint16_t* k_pool, const uint16_t* v_pool,
+                          const int32_t* block_tables, int max_pages_per_seq,
+                          const int32_t* context_lens, int batch, int q_heads, int kv_heads,
+                          int head_dim, int page_size, double scale, int dtype,
+                          double* out, double* weights, int max_len)
+{
+    int group = q_heads / kv_heads;
+    for (int b = 0; b < batch; ++b) {
+        int len = context_lens[b];
+        if (len <= 0) {
+            for (int h = 0; h < q_heads; ++h)
+                for (int i = 0; i < head_dim; ++i)
+                    out[((int64_t)b * q_heads + h) * head_dim + i] = 0.0;
+            if (weights)
+                for (int h = 0; h < q_heads; ++h)
+                    for (int t = 0; t < max_len; ++t)
+                        weights[((int64_t)b * q_heads + h) * max_len + t] = 0.0;
+            continue;
+        }
+        size_t n = (size_t)len * kv_heads * head_dim;
+        double* K = (double*)malloc(sizeof(double) * n);
+        double* V = (double*)malloc(sizeof(double) * n);
+        double* s = (double*)malloc(sizeof(double) * (size_t)len);
+        gather_sequence(k_pool, block_tables, max_pages_per_seq, b, len, kv_heads, page_size,
+                        head_dim, dtype, K);
+        gather_sequence(v_pool, block_tables, max_pages_per_seq, b, len, kv_heads, page_size,
+                        head_dim, dtype, V);
+        for (int h = 0; h < q_heads; ++h) {
+            int g = h / group;
+            const uint16_t* qh = q + ((int64_t)b * q_heads + h) * head_dim;
+            double mx = -INFINITY;
+            for (int t = 0; t < len; ++t) {
+                double dot = 0.0;
+                for (int i = 0; i < head_dim; ++i)
+                    dot += dec(qh[i], dtype) * K[((int64_t)t * kv_heads + g) * head_dim + i];
+                s[t] = scale * dot;
+                if (s[t] > mx) mx = s[t];
+            }
+            double z = 0.0;
+            for (int t = 0; t < len; ++t) {
+                s[t] = exp(s[t] - mx);
+                z += s[t];
+            }
+            double* o = out + ((int64_t)b * q_heads + h) * head_dim;
+            for (int i = 0; i < head_dim; ++i) {
+                double acc = 0.0;
+                for (int t = 0; t < len; ++t)
+                    acc += s[t] * V[((int64_t)t * kv_heads + g) * head_dim + i];
+                o[i] = acc / z;
+            }
+            if (weights) {
+                double* w = weights + ((int64_t)b * q_heads + h) * max_len;
+                for (int t = 0; t < max_len; ++t) w[t] = t < len ? s[t] / z : 0.0;
+            }
+        }
+        free(K);
+        free(V);
+        free(s);
+    }
+}
+
+/*
+ * Decode attention restricted to a list of (b, q head) pairs -- the same
+ * arithmetic as ora_decode_attention, for spot checks at sizes where the full
+ * batch would take too long.  out: [n_pairs][head_dim].
+ */
+void ora_decode_attention_pairs(const uint16_t* q, const uint16_t* k_pool, const uint16_t* v_pool,
+                                const int32_t* block_tables, int max_pages_per_seq,
+                                const int32_t* context_lens, int q_heads, int kv_heads,
+                                int head_dim, int page_size, double scale, int dtype,
+                                const int32_t* pair_b, const int32_t* pair_h, int n_pairs,
+                                double* out)
+{
+    int group = q_heads / kv_heads;
+    for (int p = 0; p < n_pairs; ++p) {
+        int b = pair_b[p], h = pair_h[p], g = h / group;
+        int len = context_lens[b];
+        double* o = out + (int64_t)p * head_dim;
+        if (len <= 0) {
+            for (int i = 0; i < head_dim; ++i) o[i] = 0.0;
+            continue;
+        }
+        const uint16_t* qh = q + ((int64_t)b * q_heads + h) * head_dim;
+        double* s = (double*)malloc(sizeof(double) * (size_t)len);
+        double mx = -INFINITY;
+        for (int t = 0; t < len; ++t) {
+            int64_t page = block_tables[(int64_t)b * max_pages_per_seq + t / page_size];
+            const uint16_t* kr = k_pool + ((page * kv_heads + g) * page_size + t % page_size) * head_dim;
+            double dot = 0.0;
+            for (int i = 0; i < head_dim; ++i) dot += dec(qh[i], dtype) * dec(kr[i], dtype);
+            s[t] = scale * dot;
+            if (s[t] > mx) mx = s[t];
+        }
+        double z = 0.0;
+        for (int t = 0; t < len; ++t) {
+            s[t] = exp(s[t] - mx);
+            z += s[t];
+        }
+        for (int i = 0; i < head_dim; ++i) o[i] = 0.0;
+        for (int t = 0; t < len; ++t) {
+            int64_t page = block_tables[(int64_t)b * max_pages_per_seq + t / page_size];
+            const uint16_t* vr = v_pool + ((page * kv_heads + g) * page_size + t % page_size) * head_dim;
+            for (int i = 0; i < head_dim; ++i) o[i] += s[t] * dec(vr[i], dtype);
+        }
+        for (int i = 0; i < head_dim; ++i) o[i] /= z;
+        free(s);
+    }
+}
+
+/*
+ * Full causal attention over a whole contiguous sequence, every position a
+ * query -- the "no cache, recompute everything" form of [ENGINE] s4.3 / s5.2:
+ * S = Q K^T * scale + M with M[i][j] = -inf for j > i, row softmax, times V.
+ *   q: [T][q_heads][head_dim], k, v: [T][kv_heads][head_dim] (doubles);
+ *   out: [T][q_heads][head_dim].
+ * Written with the explicit T x T score matrix and mask, independently of the
+ * paged decode routine, so that the last row checks it.
+ */
+void ora_causal_attention_full(const double* q, const double* k, const double* v, int T,
+                               int q_heads, int kv_heads, int head_dim, double scale, double* out)
+{
+    int group = q_heads / kv_heads;
+    double* S = (double*)malloc(sizeof(double) * (size_t)T * (size_t)T);
+    for (int h = 0; h < q_heads; ++h) {
+        int g = h / group;
+        for (int i = 0; i < T; ++i) {
+            for (int j = 0; j < T; ++j) {
+                double dot = 0.0;
+                for (int e = 0; e < head_dim; ++e)
+                    dot += q[((int64_t)i * q_heads + h) * head_dim + e] *
+                           k[((int64_t)j * kv_heads + g) * head_dim + e];
+                double mask = j > i ? -INFINITY : 0.0;
+                S[(int64_t)i * T + j] = dot * scale + mask;
+            }
+        }
+        for (int i = 0; i < T; ++i) {
+            double* row = S + (int64_t)i * T;
+            double mx = -INFINITY;
+            for (int j = 0; j < T; ++j)
+                if (row[j] > mx) mx = row[j];
+            double z = 0.0;
+            for (int j = 0; j < T; ++j) {
+                row[j] = exp(row[j] - mx);
+                z += row[j];
+            }
+            for (int j = 0; j < T; ++j) row[j] /= z;
+            for (int e = 0; e < head_dim; ++e) {
+                double acc = 0.0;
+                for (int j = 0; j < T; ++j) acc += row[j] * v[((int64_t)j * kv_heads + g) * head_dim + e];
+                out[((int64_t)i * q_heads + h) * head_dim + e] = acc;
+            }
+        }
+    }
+    free(S);
+}
+
+/* ------------------------------------------------------------------------- */
+/* KV-cache size  [ENGINE] s3.4                                                */
+/* ------------------------------------------------------------------------- */
+
+/* layers x 2 (K and V) x heads x head_dim x tokens x bytes per element */
+int64_t ora_kv_cache_bytes(int layers, int heads, int head_dim, int64_t tokens, int elt_bytes)
+{
+    return (int64_t)layers * 2 * heads * head_dim * tokens * elt_bytes;
+}
