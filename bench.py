@@ -1,0 +1,417 @@
+"""Benchmark of one decode step of attention against a paged KV cache on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload batch10] [--layers L] [--splits S]
+
+A step is one pass of the whole hot path over one batch: for every layer, RoPE on
+the new token's q and k, the KV append through the slot mapping, and paged decode
+attention (streaming pass + merge).  The default workload is the batch-10,
+32-layer, 32-head, head_dim-128, fp16 decode step with context lengths uniform in
+[128, 2048] and 16-token pages interleaved across the requests.
+
+Prints one JSON line.  `value` is KV-read throughput (algorithmic K+V bytes the
+attention must read, per second) of whole steps timed with CUDA events, inputs
+resident in HBM; `e2e` is the same metric with each step's inputs copied from
+pinned host memory and its outputs read back inside the timed region; `roofline`
+is the attention call alone, timed per launch, against the measured HBM copy
+bandwidth.  With --impl reference the fp64 CPU oracle is timed instead, on a
+bounded sample of the same workload.
+"""
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0
+METRIC = "paged decode-attention KV-read GB/s (% of HBM peak); us per layer-step"
+UNIT = "GB/s"
+INPUT_SETS = 16          # distinct per-step q/k/v sets cycled through the timed steps
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", choices=synth.WORKLOADS, default="batch10")
+    ap.add_argument("--layers", type=int, default=None, help="override the workload's layer count")
+    ap.add_argument("--splits", type=int, default=0, help="attention work partitions (0 = auto)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the CPU-baseline sample")
+    return ap.parse_args(argv)
+
+
+# ------------------------------------------------------------------ helpers
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_digest():
+    h = hashlib.sha256()
+    for name in ("decode_attention.cuh", "pkv_device.cuh"):
+        with open(os.path.join(ROOT, "paged_kv_cache_460_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload):
+    """DRAM bytes per attention launch from the committed ncu summary, if it was taken
+    on the kernel source as it is now (else None)."""
+    path = os.path.join(ROOT, "profiles", "decode_attention_%s.md" % workload)
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line and line.strip().startswith("- "):
+                k, v = line.strip()[2:].split(":", 1)
+                vals[k.strip()] = v.strip().strip("`")
+    if vals.get("kernel_source_digest") != kernel_source_digest():
+        return None
+    try:
+        return int(float(vals["dram_bytes_per_attention_call"]))
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples while the timed regions run."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.device_index = device_index
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.device_index), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(mx)), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world and world > 1:
+        raise SystemExit("--gpus %d but WORLD_SIZE %d" % (args.gpus, world))
+    return world, rank, local
+
+
+def max_over_ranks(value, world, device=None):
+    """Max of a per-rank float across the process group (the identity with one rank)."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ CPU oracle timing
+def time_oracle_sample(s, seconds, seed=0, max_pairs=None):
+    """Time the fp64 oracle (single thread) on (b, kv head) pairs of the workload, each
+    pair a standalone mini pool, until ~`seconds` have passed.  Returns
+    (GB/s of algorithmic KV bytes, description)."""
+    import oracle
+    r = np.random.Generator(np.random.PCG64(seed))
+    G = s.q_heads // s.kv_heads
+    live = np.nonzero(s.context_lens > 0)[0]
+    scale = 1.0 / math.sqrt(s.head_dim)
+    total_bytes, total_t, n = 0, 0.0, 0
+    while total_t < seconds and (max_pairs is None or n < max_pairs):
+        b = int(r.choice(live))
+        g = int(r.integers(0, s.kv_heads))
+        kmini, vmini = synth.mini_pool_numpy(s, b, g, seed=int(r.integers(1 << 30)))
+        q = synth.round_f32(r.standard_normal((1, G, s.head_dim), dtype=np.float32), s.dtype)
+        table = np.arange(kmini.shape[0], dtype=np.int32)[None, :]
+        cl = np.array([s.context_lens[b]], np.int32)
+        pairs = [(0, h) for h in range(G)]
+        t0 = time.perf_counter()
+        oracle.decode_attention_pairs(q, kmini, vmini, table, cl, scale, s.dtype, pairs)
+        total_t += time.perf_counter() - t0
+        total_bytes += int(cl[0]) * 2 * s.head_dim * s.elt_bytes
+        n += 1
+    gbs = total_bytes / total_t / 1e9
+    return gbs, "%d random (sequence, kv head) pairs of one %s layer (%d query heads each), %.1f s" % (
+        n, s.name, G, total_t)
+
+
+def run_reference(args):
+    world, rank, _ = dist_setup(args)
+    if rank != 0:
+        return 0
+    s = synth.spec(args.workload, num_layers=args.layers)
+    per_step = max(0.02, min(2.0, 150.0 / max(1, args.steps + args.warmup)))
+    for i in range(args.warmup):
+        time_oracle_sample(s, per_step, seed=i)
+    vals, t_all = [], 0.0
+    import oracle  # noqa: F401
+    for i in range(args.steps):
+        t0 = time.perf_counter()
+        g, _ = time_oracle_sample(s, per_step, seed=1000 + i)
+        t_all += time.perf_counter() - t0
+        vals.append(g)
+    value = float(np.mean(vals))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * t_all / max(1, args.steps),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(s, args),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": "each step: ~%.2f s of single-thread fp64 oracle on random (sequence, kv head) "
+                                   "pairs of the workload" % per_step},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(s, args):
+    return {"workload": "%s: batch %d, %d layers, %d q / %d kv heads, head_dim %d, page %d, %s, context %d..%d"
+                        % (s.name, s.batch, s.num_layers, s.q_heads, s.kv_heads, s.head_dim, s.page_size, s.dtype,
+                           int(s.context_lens.min()), int(s.context_lens.max())),
+            "batch": s.batch, "layers": s.num_layers, "q_heads": s.q_heads, "kv_heads": s.kv_heads,
+            "head_dim": s.head_dim, "page_size": s.page_size,
+            "kv_bytes_per_layer": s.kv_bytes_read(), "kv_bytes_per_step": s.kv_bytes_read() * s.num_layers,
+            "parallelism": "replicas" if args.gpus > 1 else "single",
+            "l2": "inputs larger than L2: each step streams %d layer caches (%.2f GB of K+V)"
+                  % (s.num_layers, s.kv_bytes_read() * s.num_layers / 1e9)
+                  if s.kv_bytes_read() * s.num_layers > 2 * 126e6 else "L2 flushed between steps"}
+
+
+# ------------------------------------------------------------------ GPU run
+def run_ours(args):
+    import torch
+    import paged_kv_cache_460_b200 as pkv
+
+    world, rank, local = dist_setup(args)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", device_id=dev, timeout=timedelta(seconds=120))
+
+    s = synth.spec(args.workload, num_layers=args.layers)
+    L = s.num_layers
+    tdt = torch.float16 if s.dtype == "f16" else torch.bfloat16
+    kp, vp = synth.pool_values_torch(s, dev)
+    pool = pkv.KVPool(kp, vp)
+    qs, ks, vs = synth.step_values_torch(s, INPUT_SETS, dev)
+    bt = torch.from_numpy(s.block_tables).to(dev)
+    cl = torch.from_numpy(s.context_lens).to(dev)
+    pos = torch.from_numpy(s.positions).to(dev)
+    slots = torch.from_numpy(pkv.pkv_slot_mapping(s.block_tables, s.positions, s.page_size)).to(dev)
+    ws = pkv.DecodeWorkspace(s.batch, s.q_heads, s.kv_heads, s.head_dim, s.page_size, tdt, args.splits, device=dev)
+    out = torch.empty((L, s.batch, s.q_heads, s.head_dim), dtype=tdt, device=dev)
+    scale = 1.0 / math.sqrt(s.head_dim)
+    stream = torch.cuda.current_stream()
+    small = s.kv_bytes_read() * L < 2 * 126e6
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev) if small else None
+
+    def step(i, events=None):
+        j = i % INPUT_SETS
+        for layer in range(L):
+            q, k, v = qs[j, layer], ks[j, layer], vs[j, layer]
+            pkv.rope_apply(q, k, pos, s.theta, stream)
+            pkv.paged_kv_append(pool, layer, k, v, slots, stream)
+            if events is not None:
+                events[layer][0].record(stream)
+            pkv.paged_decode_attention(pool, layer, out[layer], q, bt, cl, scale, num_splits=ws.num_splits,
+                                       workspace=ws, stream=stream)
+            if events is not None:
+                events[layer][1].record(stream)
+
+    def sync_all():
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+
+    for i in range(args.warmup):
+        step(i)
+    sync_all()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    # ---- phase A: whole steps (headline value)
+    sync_all()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        if flush is not None:
+            flush.zero_()
+        step(i)
+    e1.record(stream)
+    sync_all()
+    ms_total = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    # ---- phase B: the attention call timed per launch (roofline)
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(L)]
+          for _ in range(args.steps)]
+    sync_all()
+    for i in range(args.steps):
+        if flush is not None:
+            flush.zero_()
+        step(i, ev[i])
+    sync_all()
+    attn_ms = [ev[i][l][0].elapsed_time(ev[i][l][1]) for i in range(args.steps) for l in range(L)]
+    attn_ms_mean = max_over_ranks(float(np.mean(attn_ms)), world, dev)
+    clk = clocks.stop()
+
+    # ---- e2e through the public API, host buffers in and out
+    e2e = None
+    if not args.no_e2e:
+        hq = torch.empty(qs.shape[1:], dtype=tdt).pin_memory()
+        hk = torch.empty(ks.shape[1:], dtype=tdt).pin_memory()
+        hv = torch.empty(vs.shape[1:], dtype=tdt).pin_memory()
+        hq.copy_(qs[0])
+        hk.copy_(ks[0])
+        hv.copy_(vs[0])
+        h_meta = [torch.from_numpy(x).pin_memory() for x in
+                  (s.block_tables, s.context_lens, s.positions, pkv.pkv_slot_mapping(s.block_tables, s.positions,
+                                                                                     s.page_size))]
+        hout = torch.empty(out.shape, dtype=tdt).pin_memory()
+        dq, dk, dv = torch.empty_like(qs[0]), torch.empty_like(ks[0]), torch.empty_like(vs[0])
+        dmeta = [torch.empty_like(x, device=dev) for x in h_meta]
+        h2d = sum(t.numel() * t.element_size() for t in [hq, hk, hv] + h_meta)
+        d2h = hout.numel() * hout.element_size()
+
+        def e2e_step():
+            for dst, src in zip([dq, dk, dv] + dmeta, [hq, hk, hv] + h_meta):
+                dst.copy_(src, non_blocking=True)
+            dbt, dcl, dpos, dslot = dmeta
+            for layer in range(L):
+                pkv.rope_apply(dq[layer], dk[layer], dpos, s.theta, stream)
+                pkv.paged_kv_append(pool, layer, dk[layer], dv[layer], dslot, stream)
+                pkv.paged_decode_attention(pool, layer, out[layer], dq[layer], dbt, dcl, scale,
+                                           num_splits=ws.num_splits, workspace=ws, stream=stream)
+            hout.copy_(out, non_blocking=True)
+
+        for _ in range(max(1, args.warmup)):
+            e2e_step()
+        sync_all()
+        n_e2e = max(1, args.steps // 2)
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(n_e2e):
+            if flush is not None:
+                flush.zero_()
+            e2e_step()
+        a1.record(stream)
+        sync_all()
+        ms_e2e = max_over_ranks(a0.elapsed_time(a1), world, dev)
+        e2e = {"value": world * s.kv_bytes_read() * L * n_e2e / (ms_e2e * 1e-3) / 1e9, "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": ms_e2e / n_e2e}
+
+    err = pkv.kv_get_device_error()
+    if err:
+        raise SystemExit("device error word 0x%x after the benchmark" % err)
+
+    if rank == 0:
+        per_step_ms = ms_total / args.steps
+        value = world * s.kv_bytes_read() * L * args.steps / (ms_total * 1e-3) / 1e9
+        peak, peak_kind = measured_peaks()
+        achieved = s.kv_bytes_read() / (attn_ms_mean * 1e-3) / 1e9
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            gbs, desc = time_oracle_sample(s, args.cpu_seconds)
+            cpu = {"value": gbs, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc}
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": per_step_ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": s.dtype, "data": "synthetic", "config": workload_config(s, args),
+            "us_per_layer_step": 1000.0 * per_step_ms / L,
+            "attention_us_per_layer": 1000.0 * attn_ms_mean,
+            "pct_of_8tbs": 100.0 * value / NOMINAL_HBM_GBS,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": profiled_traffic(args.workload),
+                         "peak_source": "%s copy bandwidth" % peak_kind,
+                         "kernel": "paged_decode_attention (streaming pass + merge), per call",
+                         "frac_of_8tbs": achieved / NOMINAL_HBM_GBS},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": args.steps * L * 4 * world,
+            "num_splits": ws.num_splits,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

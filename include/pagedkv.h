@@ -1,0 +1,213 @@
+/*
+ * pagedkv.h -- C ABI of libpagedkv.so: one autoregressive decode step of
+ * LLaMA-style attention against a paged KV cache, on NVIDIA B200 (sm_100a).
+ *
+ * Sources, cited by page title and section:
+ *   [ENGINE] "为什么要自己动手写一个LLM推理引擎" (wzjinhao.cn/news/61427), chapter 1
+ *            s3.4  KV-cache management: size formula; the cache cut into fixed pages of
+ *                  16 or 32 tokens, allocated from a free list and given back when a
+ *                  request ends; attention locates a token's block through a page index.
+ *            s4.2  RoPE: position enters q and k through a rotation.
+ *            s4.3  forward with a cache: n_heads / n_kv_heads views,
+ *                  apply_rotary_emb(q, k, start_pos), cache update, q k^T / sqrt(head_dim)
+ *                  plus causal mask, softmax, times v.
+ *            s5.3  replace concatenation with a preallocated cache pool; fused attention.
+ *   [FLOW]   "大模型推理全流程解析" (stapisi.com/news/4049481) s2.2.2: decode attention of
+ *            the new token against every cached K/V; KV read bandwidth is the bottleneck.
+ *
+ * Conventions for every entry point
+ *   - Return value: PKV_OK (0) or one of the PKV_ERR_* codes below;
+ *     pkv_status_string() names it.  Arguments are validated on the host before any
+ *     launch; a call that returns an error has launched nothing.
+ *   - Memory: every device pointer is owned by the caller (allocated by any CUDA
+ *     allocator, e.g. PyTorch).  The library allocates no device memory on any path;
+ *     scratch comes from a caller-provided workspace.
+ *   - Streams: device work is enqueued asynchronously on the caller's stream (a
+ *     cudaStream_t; NULL = legacy default stream); no entry point synchronises the
+ *     host except kv_get_device_error().  Consecutive kernels of the library use
+ *     programmatic dependent launch, so a kernel's prologue may overlap the tail of the
+ *     library kernel before it on the same stream.
+ *   - Layouts are row-major, innermost index last.  Element type: PKV_F16 (IEEE
+ *     binary16) or PKV_BF16 (bfloat16), the same for q, k, v, the pool and the output.
+ *   - Device-side index checks: an out-of-range page id or slot is never dereferenced;
+ *     the access is skipped and a bit is set in a device error word that
+ *     kv_get_device_error() returns.  Bounded waits inside the kernels set a bit there
+ *     too instead of spinning forever.
+ */
+#ifndef PAGEDKV_H_
+#define PAGEDKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* status codes */
+#define PKV_OK 0
+#define PKV_ERR_INVALID_ARG 1   /* null pointer, negative or inconsistent size */
+#define PKV_ERR_UNSUPPORTED 2   /* a shape/dtype combination with no compiled kernel */
+#define PKV_ERR_CUDA 3          /* a CUDA runtime call or launch failed */
+#define PKV_ERR_NO_SPACE 4      /* free list too short, or workspace too small */
+
+/* element types */
+#define PKV_F16 0
+#define PKV_BF16 1
+
+/* device error word bits (kv_get_device_error) */
+#define PKV_DEVERR_BAD_PAGE 0x1u     /* block-table entry outside [0, num_pages) */
+#define PKV_DEVERR_BAD_SLOT 0x2u     /* slot_mapping entry >= num_pages * page_size */
+#define PKV_DEVERR_TIMEOUT 0x4u      /* a bounded wait on a shared-memory barrier gave up */
+
+typedef struct CUstream_st* pkv_stream_t; /* identical to cudaStream_t */
+typedef struct pkv_pool pkv_pool;         /* opaque host-side pool descriptor */
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* pkv_status_string(int status);
+
+/* ------------------------------------------------------------------------
+ * KV pool  ([ENGINE] s3.4, s5.3)
+ * ---------------------------------------------------------------------- */
+
+/*
+ * Describe a preallocated paged KV pool and create its host free list.
+ *   k_base, v_base: device arrays of [num_layers][num_pages][kv_heads][page_size][head_dim]
+ *                   elements of `dtype`; one (page, head) is page_size*head_dim contiguous
+ *                   elements.  Both must be 16-byte aligned.  The caller keeps ownership and
+ *                   must keep them alive while the pool is used; nothing is read or written
+ *                   here.
+ *   page_size: 16 or 32 tokens; head_dim: 64 or 128; dtype: PKV_F16 or PKV_BF16.
+ * The free list starts with every page id 0..num_pages-1, handed out in increasing order.
+ * Errors: INVALID_ARG for null/non-positive/misaligned arguments, UNSUPPORTED for other
+ * page sizes, head dims or dtypes.
+ */
+int kv_pool_create(int num_layers, int num_pages, int page_size, int kv_heads, int head_dim,
+                   int dtype, void* k_base, void* v_base, pkv_pool** out);
+
+/* Free the host descriptor (not the caller's device arrays).  NULL is ignored. */
+void kv_pool_destroy(pkv_pool* pool);
+
+/*
+ * Take n page ids from the free list into page_ids_out[0..n) (host array).  All or
+ * nothing: NO_SPACE, with nothing taken, when fewer than n pages are free.
+ */
+int kv_pool_alloc(pkv_pool* pool, int n, int32_t* page_ids_out);
+
+/*
+ * Give n page ids back (host array).  INVALID_ARG, with nothing returned, if any id is out of
+ * range, not currently allocated, or repeated in the list.  Freed pages are handed out again
+ * before never-used ones, most recently freed first.
+ */
+int kv_pool_free(pkv_pool* pool, int n, const int32_t* page_ids);
+
+/* Number of free pages, or -1 for a NULL pool. */
+int kv_pool_free_count(const pkv_pool* pool);
+
+/* Shape of the pool: writes any of the non-NULL outputs; INVALID_ARG for a NULL pool. */
+int kv_pool_info(const pkv_pool* pool, int* num_layers, int* num_pages, int* page_size,
+                 int* kv_heads, int* head_dim, int* dtype);
+
+/*
+ * KV-cache bytes for `tokens` tokens ([ENGINE] s3.4):
+ * layers x 2 (K and V) x kv_heads x head_dim x tokens x element bytes.  -1 on bad input.
+ */
+int64_t pkv_kv_cache_bytes(int num_layers, int kv_heads, int head_dim, int64_t tokens, int dtype);
+
+/*
+ * Slot of each new token (host arrays; [ENGINE] s3.4 page index):
+ *   slots_out[i] = block_tables[i][positions[i] / page_size] * page_size + positions[i] % page_size
+ * block_tables: [n][max_pages_per_seq] int32; positions[i] < 0 marks a padded row and
+ * gives slot -1.  INVALID_ARG if a position's page lies beyond max_pages_per_seq or its
+ * table entry is negative.
+ */
+int pkv_slot_mapping(const int32_t* block_tables, int max_pages_per_seq, const int32_t* positions,
+                     int n, int page_size, int64_t* slots_out);
+
+/* ------------------------------------------------------------------------
+ * Decode step kernels
+ * ---------------------------------------------------------------------- */
+
+/*
+ * RoPE on the new token's q and k, in place ([ENGINE] s4.2, s4.3 apply_rotary_emb(q, k,
+ * start_pos)).
+ *   q: device [n_tokens][q_heads][head_dim]; k: device [n_tokens][kv_heads][head_dim];
+ *   positions: device [n_tokens] int32, the position of each token; rows with a negative
+ *   position are left untouched.
+ * Pair i = (x[2i], x[2i+1]) of every head turns by pos * theta^(-2i/head_dim).  The angle,
+ * its cosine and sine and the rotation are evaluated in fp64 and rounded once to the
+ * element type.  head_dim: 64 or 128.  Either q or k may be NULL (with its head count 0).
+ */
+int rope_apply(void* q, void* k, const int32_t* positions, int n_tokens, int q_heads,
+               int kv_heads, int head_dim, double theta, int dtype, pkv_stream_t stream);
+
+/*
+ * Cache update of one layer ([ENGINE] s4.3 append to the cache, s5.3 preallocated pool):
+ * for each token i with slot s = slot_mapping[i] >= 0, copies k[i][h][:] and v[i][h][:]
+ * bit for bit into page s / page_size, row s % page_size of kv head h of `layer`.
+ *   k, v: device [n_tokens][kv_heads][head_dim] (pool's dtype), 16-byte aligned;
+ *   slot_mapping: device [n_tokens] int64 (negative = skip the row).
+ * A slot >= num_pages * page_size is skipped and sets PKV_DEVERR_BAD_SLOT.
+ */
+int paged_kv_append(const pkv_pool* pool, int layer, const void* k, const void* v,
+                    const int64_t* slot_mapping, int n_tokens, pkv_stream_t stream);
+
+/*
+ * Number of work partitions paged_decode_attention uses when called with num_splits = 0 on
+ * the current device (SM count x resident CTAs per SM for this shape).  Needs a CUDA
+ * device; PKV_ERR_CUDA without one.
+ */
+int pkv_decode_default_splits(int q_heads, int kv_heads, int head_dim, int page_size, int dtype,
+                              int* num_splits_out);
+
+/*
+ * Workspace bytes paged_decode_attention needs for `num_splits` (>= 1) partitions and a
+ * batch of `batch` rows: per partition two fp32 partial results (running max, sum and the
+ * unnormalised output of every query head of a kv-head group) plus the batch's page
+ * prefix sums.  0 on bad input.
+ */
+size_t pkv_decode_workspace_size(int batch, int q_heads, int kv_heads, int head_dim,
+                                 int num_splits);
+
+/*
+ * Decode attention of one new query token per sequence over its paged cache
+ * ([ENGINE] s4.3, [FLOW] s2.2.2):
+ *   out[b][h][:] = sum_t softmax_t(scale * <q[b][h], K_b[t][g]>) * V_b[t][g],
+ *   g = h / (q_heads / kv_heads), t over the context_lens[b] cached tokens, token t of
+ *   sequence b read from page block_tables[b][t / page_size], row t % page_size.
+ * The query sits at the last position, so the causal mask keeps every cached token.
+ *   out, q: device [batch][q_heads][head_dim] (pool's dtype), 16-byte aligned; out is
+ *           written once, rounded to nearest-even from fp32; rows with context_lens[b] <= 0
+ *           get zeros.
+ *   block_tables: device [batch][max_pages_per_seq] int32; entries past a row's
+ *           ceil(context_lens[b] / page_size) pages are not read.
+ *   context_lens: device [batch] int32, the new token included.
+ *   kv_heads must equal the pool's; q_heads a multiple of it with q_heads / kv_heads in
+ *   {1, 2, 4, 8}.
+ *   num_splits: number of work partitions (0 = pkv_decode_default_splits).  The batch's
+ *           pages x kv heads are laid end to end and cut into num_splits equal ranges, one
+ *           per CTA; a (sequence, kv head) cut by a range boundary is finished by a second
+ *           merge kernel that rescales the partial softmax sums (log-sum-exp).
+ *   workspace: device scratch of >= pkv_decode_workspace_size(batch, q_heads, kv_heads,
+ *           head_dim, num_splits) bytes, 256-byte aligned; no initial contents needed;
+ *           calls that share a workspace must be ordered on one stream.
+ * Errors: INVALID_ARG (bad pointer/shape/layer), UNSUPPORTED (group/head_dim/page/dtype
+ * combination), NO_SPACE (workspace too small), CUDA (launch failure).
+ */
+int paged_decode_attention(const pkv_pool* pool, int layer, void* out, const void* q,
+                           const int32_t* block_tables, int max_pages_per_seq,
+                           const int32_t* context_lens, int batch, int q_heads, int kv_heads,
+                           float scale, int num_splits, void* workspace, size_t workspace_bytes,
+                           pkv_stream_t stream);
+
+/*
+ * Read and clear the device error word (PKV_DEVERR_* bits) of the current device.
+ * Synchronises the device.  PKV_ERR_CUDA if the read fails.
+ */
+int kv_get_device_error(uint32_t* err_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDKV_H_ */

@@ -1,0 +1,216 @@
+"""Paged KV cache decode step on B200 (sm_100a): thin Python binding of libpagedkv.
+
+One autoregressive decode step of LLaMA-style attention against a paged KV cache
+("为什么要自己动手写一个LLM推理引擎", wzjinhao.cn/news/61427, s3.4 paging, s4.2 RoPE,
+s4.3 forward with a cache):
+
+    rope_apply              RoPE on the new token's q and k (in place)
+    pkv_slot_mapping        slot of each new token from the page table (host)
+    paged_kv_append         write the new k, v into their slots
+    paged_decode_attention  softmax(scale q.K^T) V over each sequence's pages
+
+Every function here only marshals arguments (torch tensors -> raw pointers, the
+current CUDA stream) and calls the C ABI of libpagedkv.so; all arithmetic of the
+step runs in the library's CUDA kernels.  PyTorch provides device memory and
+streams only.  Errors raise PagedKVError.
+"""
+import ctypes
+
+import numpy as np
+
+from . import _lib
+from ._lib import (PKV_BF16, PKV_DEVERR_BAD_PAGE, PKV_DEVERR_BAD_SLOT, PKV_DEVERR_TIMEOUT, PKV_F16,
+                   PagedKVError, lib)
+
+__all__ = [
+    "KVPool", "rope_apply", "paged_kv_append", "paged_decode_attention", "pkv_slot_mapping",
+    "pkv_kv_cache_bytes", "pkv_decode_workspace_size", "pkv_decode_default_splits",
+    "kv_get_device_error", "DecodeWorkspace", "PagedKVError", "PKV_F16", "PKV_BF16",
+    "PKV_DEVERR_BAD_PAGE", "PKV_DEVERR_BAD_SLOT", "PKV_DEVERR_TIMEOUT",
+]
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def dtype_code(dt):
+    torch = _torch()
+    if dt == torch.float16:
+        return PKV_F16
+    if dt == torch.bfloat16:
+        return PKV_BF16
+    raise PagedKVError("dtype", _lib.PKV_ERR_UNSUPPORTED)
+
+
+def _stream(stream):
+    torch = _torch()
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _need(t, name, dtype=None, cuda=True):
+    if t is None:
+        return
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if cuda and not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError("%s must be %s, got %s" % (name, dtype, t.dtype))
+
+
+# ------------------------------------------------------------------ pool
+class KVPool:
+    """A paged KV pool over caller-owned device tensors.
+
+    k_cache, v_cache: [num_layers, num_pages, kv_heads, page_size, head_dim], fp16 or bf16.
+    The host free list hands page ids out with ``alloc`` and takes them back with ``free``.
+    """
+
+    def __init__(self, k_cache, v_cache):
+        torch = _torch()
+        if k_cache.shape != v_cache.shape or k_cache.dtype != v_cache.dtype or k_cache.dim() != 5:
+            raise ValueError("k_cache and v_cache must both be [layers, pages, kv_heads, page, head_dim]")
+        _need(k_cache, "k_cache", cuda=False)
+        _need(v_cache, "v_cache", cuda=False)
+        self.k_cache, self.v_cache = k_cache, v_cache
+        L, N, H, P, D = k_cache.shape
+        self.num_layers, self.num_pages, self.kv_heads, self.page_size, self.head_dim = L, N, H, P, D
+        self.dtype = k_cache.dtype
+        h = ctypes.c_void_p()
+        st = lib().kv_pool_create(L, N, P, H, D, dtype_code(k_cache.dtype), _ptr(k_cache), _ptr(v_cache),
+                                  ctypes.byref(h))
+        _lib.check("kv_pool_create", st)
+        self.handle = h
+        del torch
+
+    def close(self):
+        if getattr(self, "handle", None) is not None and self.handle.value:
+            lib().kv_pool_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def alloc(self, n):
+        out = np.empty(n, np.int32)
+        _lib.check("kv_pool_alloc", lib().kv_pool_alloc(self.handle, n, out.ctypes.data_as(ctypes.c_void_p)))
+        return out
+
+    def free(self, ids):
+        ids = np.ascontiguousarray(ids, np.int32)
+        _lib.check("kv_pool_free", lib().kv_pool_free(self.handle, ids.size, ids.ctypes.data_as(ctypes.c_void_p)))
+
+    @property
+    def free_count(self):
+        return lib().kv_pool_free_count(self.handle)
+
+    def info(self):
+        vals = [ctypes.c_int() for _ in range(6)]
+        _lib.check("kv_pool_info", lib().kv_pool_info(self.handle, *[ctypes.byref(v) for v in vals]))
+        return tuple(v.value for v in vals)
+
+
+# ------------------------------------------------------------------ host helpers
+def pkv_kv_cache_bytes(num_layers, kv_heads, head_dim, tokens, dtype=PKV_F16):
+    return int(lib().pkv_kv_cache_bytes(num_layers, kv_heads, head_dim, tokens, dtype))
+
+
+def pkv_slot_mapping(block_tables, positions, page_size):
+    """Host: int32 [n, max_pages] table and int32 [n] positions -> int64 [n] slots."""
+    bt = np.ascontiguousarray(block_tables, np.int32)
+    pos = np.ascontiguousarray(positions, np.int32)
+    out = np.empty(pos.shape[0], np.int64)
+    st = lib().pkv_slot_mapping(bt.ctypes.data_as(ctypes.c_void_p), bt.shape[1], pos.ctypes.data_as(ctypes.c_void_p),
+                                pos.shape[0], page_size, out.ctypes.data_as(ctypes.c_void_p))
+    _lib.check("pkv_slot_mapping", st)
+    return out
+
+
+def pkv_decode_default_splits(q_heads, kv_heads, head_dim, page_size, dtype=PKV_F16):
+    n = ctypes.c_int()
+    _lib.check("pkv_decode_default_splits",
+               lib().pkv_decode_default_splits(q_heads, kv_heads, head_dim, page_size, dtype, ctypes.byref(n)))
+    return n.value
+
+
+def pkv_decode_workspace_size(batch, q_heads, kv_heads, head_dim, num_splits):
+    return int(lib().pkv_decode_workspace_size(batch, q_heads, kv_heads, head_dim, num_splits))
+
+
+def kv_get_device_error():
+    v = ctypes.c_uint32()
+    _lib.check("kv_get_device_error", lib().kv_get_device_error(ctypes.byref(v)))
+    return v.value
+
+
+# ------------------------------------------------------------------ kernels
+def rope_apply(q, k, positions, theta=10000.0, stream=None):
+    """In-place RoPE of q [n, q_heads, d] and k [n, kv_heads, d] at positions (int32 [n])."""
+    torch = _torch()
+    ref = q if q is not None else k
+    _need(q, "q", ref.dtype)
+    _need(k, "k", ref.dtype)
+    _need(positions, "positions", torch.int32)
+    n = ref.shape[0]
+    qh = q.shape[1] if q is not None else 0
+    kh = k.shape[1] if k is not None else 0
+    st = lib().rope_apply(_ptr(q), _ptr(k), _ptr(positions), n, qh, kh, ref.shape[2], float(theta),
+                          dtype_code(ref.dtype), _stream(stream))
+    _lib.check("rope_apply", st)
+
+
+def paged_kv_append(pool, layer, k, v, slot_mapping, stream=None):
+    """Write k, v [n, kv_heads, d] into the pool's slots (int64 [n], negative = skip)."""
+    torch = _torch()
+    _need(k, "k", pool.dtype)
+    _need(v, "v", pool.dtype)
+    _need(slot_mapping, "slot_mapping", torch.int64)
+    st = lib().paged_kv_append(pool.handle, layer, _ptr(k), _ptr(v), _ptr(slot_mapping), k.shape[0],
+                               _stream(stream))
+    _lib.check("paged_kv_append", st)
+
+
+class DecodeWorkspace:
+    """Device scratch for paged_decode_attention, sized for a batch and a split count."""
+
+    def __init__(self, batch, q_heads, kv_heads, head_dim, page_size, dtype, num_splits=0, device=None):
+        torch = _torch()
+        if num_splits == 0:
+            num_splits = pkv_decode_default_splits(q_heads, kv_heads, head_dim, page_size, dtype_code(dtype))
+        self.num_splits = num_splits
+        self.nbytes = pkv_decode_workspace_size(batch, q_heads, kv_heads, head_dim, num_splits)
+        self.buffer = torch.empty(self.nbytes, dtype=torch.uint8, device=device or "cuda")
+
+
+def paged_decode_attention(pool, layer, out, q, block_tables, context_lens, scale, kv_heads=None,
+                           num_splits=0, workspace=None, stream=None):
+    """out[b, h] = softmax(scale * q[b, h] . K_b^T) V_b over context_lens[b] paged tokens."""
+    torch = _torch()
+    _need(out, "out", pool.dtype)
+    _need(q, "q", pool.dtype)
+    _need(block_tables, "block_tables", torch.int32)
+    _need(context_lens, "context_lens", torch.int32)
+    B, Hq, _ = q.shape
+    if kv_heads is None:
+        kv_heads = pool.kv_heads
+    if workspace is None:
+        workspace = DecodeWorkspace(B, Hq, kv_heads, pool.head_dim, pool.page_size, pool.dtype, num_splits,
+                                    device=q.device)
+    if num_splits == 0:
+        num_splits = workspace.num_splits
+    st = lib().paged_decode_attention(pool.handle, layer, _ptr(out), _ptr(q), _ptr(block_tables),
+                                      block_tables.shape[1], _ptr(context_lens), B, Hq, kv_heads, float(scale),
+                                      num_splits, _ptr(workspace.buffer), workspace.nbytes, _stream(stream))
+    _lib.check("paged_decode_attention", st)
+    return out

@@ -1,0 +1,256 @@
+// libpagedkv: C-ABI entry points that launch the decode-step kernels on sm_100a.
+//
+// Every entry point validates its arguments on the host, launches asynchronously on
+// the caller's stream and returns a PKV_* status.  Kernels are launched with
+// programmatic stream serialization (programmatic dependent launch), so the next
+// library kernel on the stream can start its prologue while the previous one drains;
+// each kernel waits (griddepcontrol.wait) before touching data the previous kernel
+// may write.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+
+#include "decode_attention.cuh"
+#include "pagedkv.h"
+#include "pkv_internal.h"
+#include "rope_append.cuh"
+
+namespace pkv {
+namespace {
+
+template <typename Kernel, typename... Args>
+cudaError_t launch_pdl(Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream, Args... args)
+{
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+int status_of(cudaError_t e) { return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA; }
+
+constexpr int kMaxDevices = 64;
+
+// Raise a kernel's dynamic shared-memory limit once per device (and size).
+template <typename Kernel>
+cudaError_t ensure_smem(Kernel kernel, int bytes, int* configured)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    if (configured[dev] >= bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) configured[dev] = bytes;
+    return e;
+}
+
+constexpr int kMaxSmemPerCta = 227 * 1024;
+
+struct DecodeOps {
+    int (*launch)(const DecodeParams&, cudaStream_t);
+    int (*splits)(int*);
+    int group;
+};
+
+template <int D, int P, int G, typename T>
+struct DecodeImpl {
+    using S = DecodeShape<D, P, G>;
+    static int configured[kMaxDevices];
+
+    static int launch(const DecodeParams& prm, cudaStream_t st)
+    {
+        const int smem = S::smem_bytes(prm.batch);
+        if (smem > kMaxSmemPerCta) return PKV_ERR_UNSUPPORTED;
+        cudaError_t e = ensure_smem(decode_pass1_kernel<D, P, G, T>, smem, configured);
+        if (e != cudaSuccess) return PKV_ERR_CUDA;
+        e = launch_pdl(decode_pass1_kernel<D, P, G, T>, dim3(prm.num_splits), dim3(kDecodeThreads), smem, st, prm);
+        if (e != cudaSuccess) return PKV_ERR_CUDA;
+        e = launch_pdl(decode_merge_kernel<D, G, T>, dim3(prm.batch * prm.kv_heads), dim3(128), 0, st, prm);
+        return status_of(e);
+    }
+
+    // SMs x resident CTAs per SM at the shared-memory size of a 64-row batch.
+    static int splits(int* out)
+    {
+        int dev = 0, sms = 0, per_sm = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess) return PKV_ERR_CUDA;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return PKV_ERR_CUDA;
+        const int smem = S::smem_bytes(64);
+        if (ensure_smem(decode_pass1_kernel<D, P, G, T>, smem, configured) != cudaSuccess) return PKV_ERR_CUDA;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_pass1_kernel<D, P, G, T>, kDecodeThreads,
+                                                          smem) != cudaSuccess)
+            return PKV_ERR_CUDA;
+        *out = sms * (per_sm > 0 ? per_sm : 1);
+        return PKV_OK;
+    }
+};
+
+template <int D, int P, int G, typename T>
+int DecodeImpl<D, P, G, T>::configured[kMaxDevices] = {0};
+
+template <int D, int P, typename T>
+bool pick_group(int group, DecodeOps& ops)
+{
+    switch (group) {
+    case 1: ops = {DecodeImpl<D, P, 1, T>::launch, DecodeImpl<D, P, 1, T>::splits, 1}; return true;
+    case 2: ops = {DecodeImpl<D, P, 2, T>::launch, DecodeImpl<D, P, 2, T>::splits, 2}; return true;
+    case 4: ops = {DecodeImpl<D, P, 4, T>::launch, DecodeImpl<D, P, 4, T>::splits, 4}; return true;
+    case 8: ops = {DecodeImpl<D, P, 8, T>::launch, DecodeImpl<D, P, 8, T>::splits, 8}; return true;
+    default: return false;
+    }
+}
+
+template <typename T>
+bool pick_shape(int head_dim, int page_size, int group, DecodeOps& ops)
+{
+    if (head_dim == 128 && page_size == 16) return pick_group<128, 16, T>(group, ops);
+    if (head_dim == 128 && page_size == 32) return pick_group<128, 32, T>(group, ops);
+    if (head_dim == 64 && page_size == 16) return pick_group<64, 16, T>(group, ops);
+    if (head_dim == 64 && page_size == 32) return pick_group<64, 32, T>(group, ops);
+    return false;
+}
+
+bool pick_decode(int head_dim, int page_size, int group, int dtype, DecodeOps& ops)
+{
+    if (dtype == PKV_F16) return pick_shape<__half>(head_dim, page_size, group, ops);
+    if (dtype == PKV_BF16) return pick_shape<__nv_bfloat16>(head_dim, page_size, group, ops);
+    return false;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct WorkspaceLayout {
+    size_t meta, part_o, part_ml, total;
+};
+
+WorkspaceLayout workspace_layout(int batch, int group, int head_dim, int num_splits)
+{
+    WorkspaceLayout w;
+    w.meta = 0;
+    w.part_o = align256(kMetaHeaderBytes + sizeof(int) * ((size_t)batch + 1));
+    w.part_ml = w.part_o + align256(sizeof(float) * 2 * (size_t)num_splits * group * head_dim);
+    w.total = w.part_ml + align256(sizeof(float) * 2 * (size_t)num_splits * group * 2);
+    return w;
+}
+
+}  // namespace
+}  // namespace pkv
+
+using namespace pkv;
+
+extern "C" int rope_apply(void* q, void* k, const int32_t* positions, int n_tokens, int q_heads, int kv_heads,
+                          int head_dim, double theta, int dtype, pkv_stream_t stream)
+{
+    if (n_tokens < 0 || q_heads < 0 || kv_heads < 0 || !(theta > 0.0)) return PKV_ERR_INVALID_ARG;
+    if ((q_heads > 0 && !q) || (kv_heads > 0 && !k)) return PKV_ERR_INVALID_ARG;
+    if (head_dim != 64 && head_dim != 128) return PKV_ERR_UNSUPPORTED;
+    if (dtype != PKV_F16 && dtype != PKV_BF16) return PKV_ERR_UNSUPPORTED;
+    if (n_tokens == 0 || q_heads + kv_heads == 0) return PKV_OK;
+    if (!positions) return PKV_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if (dtype == PKV_F16)
+        e = launch_pdl(rope_kernel<__half>, dim3(n_tokens), dim3(256), 0, st, static_cast<__half*>(q),
+                       static_cast<__half*>(k), positions, q_heads, kv_heads, head_dim, theta);
+    else
+        e = launch_pdl(rope_kernel<__nv_bfloat16>, dim3(n_tokens), dim3(256), 0, st, static_cast<__nv_bfloat16*>(q),
+                       static_cast<__nv_bfloat16*>(k), positions, q_heads, kv_heads, head_dim, theta);
+    return status_of(e);
+}
+
+extern "C" int paged_kv_append(const pkv_pool* pool, int layer, const void* k, const void* v,
+                               const int64_t* slot_mapping, int n_tokens, pkv_stream_t stream)
+{
+    if (!pool || layer < 0 || layer >= pool->num_layers || n_tokens < 0) return PKV_ERR_INVALID_ARG;
+    if (n_tokens == 0) return PKV_OK;
+    if (!k || !v || !slot_mapping) return PKV_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v)) & 15u) return PKV_ERR_INVALID_ARG;
+    const size_t elt = 2;
+    uint4* kl = reinterpret_cast<uint4*>(static_cast<char*>(pool->k_base) + (size_t)layer * pool->layer_elems * elt);
+    uint4* vl = reinterpret_cast<uint4*>(static_cast<char*>(pool->v_base) + (size_t)layer * pool->layer_elems * elt);
+    const int64_t num_slots = (int64_t)pool->num_pages * pool->page_size;
+    cudaError_t e = launch_pdl(append_kernel, dim3(n_tokens), dim3(128), 0, reinterpret_cast<cudaStream_t>(stream), kl,
+                               vl, static_cast<const uint4*>(k), static_cast<const uint4*>(v), slot_mapping,
+                               pool->kv_heads, pool->head_dim, pool->page_size, num_slots);
+    return status_of(e);
+}
+
+extern "C" int pkv_decode_default_splits(int q_heads, int kv_heads, int head_dim, int page_size, int dtype,
+                                         int* num_splits_out)
+{
+    if (!num_splits_out || q_heads <= 0 || kv_heads <= 0 || q_heads % kv_heads) return PKV_ERR_INVALID_ARG;
+    DecodeOps ops;
+    if (!pick_decode(head_dim, page_size, q_heads / kv_heads, dtype, ops)) return PKV_ERR_UNSUPPORTED;
+    return ops.splits(num_splits_out);
+}
+
+extern "C" size_t pkv_decode_workspace_size(int batch, int q_heads, int kv_heads, int head_dim, int num_splits)
+{
+    if (batch < 0 || q_heads <= 0 || kv_heads <= 0 || q_heads % kv_heads || head_dim <= 0 || num_splits <= 0)
+        return 0;
+    return workspace_layout(batch, q_heads / kv_heads, head_dim, num_splits).total;
+}
+
+extern "C" int paged_decode_attention(const pkv_pool* pool, int layer, void* out, const void* q,
+                                      const int32_t* block_tables, int max_pages_per_seq,
+                                      const int32_t* context_lens, int batch, int q_heads, int kv_heads, float scale,
+                                      int num_splits, void* workspace, size_t workspace_bytes, pkv_stream_t stream)
+{
+    if (!pool || layer < 0 || layer >= pool->num_layers) return PKV_ERR_INVALID_ARG;
+    if (batch < 0 || q_heads <= 0 || kv_heads != pool->kv_heads || q_heads % kv_heads) return PKV_ERR_INVALID_ARG;
+    if (num_splits < 0 || max_pages_per_seq <= 0 || !(scale == scale)) return PKV_ERR_INVALID_ARG;
+    if (batch == 0) return PKV_OK;
+    if (!out || !q || !block_tables || !context_lens || !workspace) return PKV_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(out) | reinterpret_cast<uintptr_t>(q)) & 15u) return PKV_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return PKV_ERR_INVALID_ARG;
+    DecodeOps ops;
+    if (!pick_decode(pool->head_dim, pool->page_size, q_heads / kv_heads, pool->dtype, ops))
+        return PKV_ERR_UNSUPPORTED;
+    if (num_splits == 0) {
+        const int st = ops.splits(&num_splits);
+        if (st != PKV_OK) return st;
+    }
+    const WorkspaceLayout wl = workspace_layout(batch, ops.group, pool->head_dim, num_splits);
+    if (workspace_bytes < wl.total) return PKV_ERR_NO_SPACE;
+    DecodeParams prm;
+    const size_t elt = 2;
+    prm.k = static_cast<const char*>(pool->k_base) + (size_t)layer * pool->layer_elems * elt;
+    prm.v = static_cast<const char*>(pool->v_base) + (size_t)layer * pool->layer_elems * elt;
+    prm.q = q;
+    prm.out = out;
+    prm.block_tables = block_tables;
+    prm.context_lens = context_lens;
+    unsigned char* ws = static_cast<unsigned char*>(workspace);
+    prm.meta = ws + wl.meta;
+    prm.part_o = reinterpret_cast<float*>(ws + wl.part_o);
+    prm.part_ml = reinterpret_cast<float*>(ws + wl.part_ml);
+    prm.batch = batch;
+    prm.max_pages = max_pages_per_seq;
+    prm.q_heads = q_heads;
+    prm.kv_heads = kv_heads;
+    prm.num_pages = pool->num_pages;
+    prm.num_splits = num_splits;
+    prm.scale_log2 = scale * 1.4426950408889634f;
+    return ops.launch(prm, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int kv_get_device_error(uint32_t* err_out)
+{
+    if (!err_out) return PKV_ERR_INVALID_ARG;
+    if (cudaDeviceSynchronize() != cudaSuccess) return PKV_ERR_CUDA;
+    unsigned int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_error_word, sizeof(v)) != cudaSuccess) return PKV_ERR_CUDA;
+    if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return PKV_ERR_CUDA;
+    *err_out = v;
+    return PKV_OK;
+}

@@ -1,0 +1,170 @@
+// Device-side building blocks for sm_100a: shared-memory barriers with bounded
+// waits, 1-D bulk (TMA) copies, programmatic dependent launch, element types.
+#ifndef PKV_DEVICE_CUH_
+#define PKV_DEVICE_CUH_
+
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "pagedkv.h"
+
+namespace pkv {
+
+// One device error word per device (PKV_DEVERR_* bits), read by kv_get_device_error().
+// The library's device code is a single translation unit (pagedkv.cu), which defines it.
+__device__ unsigned int g_error_word = 0;
+
+// A bounded wait gives up after this many SM clock cycles (about one second at the
+// B200's clocks); a healthy wait ends within microseconds.
+constexpr long long kWaitLimitCycles = 2000000000LL;
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+// Make barrier initialisation visible to the async (TMA) proxy.
+__device__ __forceinline__ void fence_barrier_init()
+{
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar)
+{
+    asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity)
+{
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+// Wait until the phase with the given parity has completed.  Gives up (returns
+// false) when *abort is set by another warp, or after kWaitLimitCycles, in which
+// case it sets *abort and PKV_DEVERR_TIMEOUT.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    for (uint32_t n = 1;; ++n) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((n & 31u) == 0) {
+            if (*abort) return false;
+            if (clock64() - t0 > kWaitLimitCycles) {
+                *abort = 1;
+                atomicOr(&g_error_word, PKV_DEVERR_TIMEOUT);
+                return false;
+            }
+        }
+    }
+}
+
+// 1-D bulk copy global -> shared through the TMA unit; completion is counted in
+// bytes on `bar`.  Addresses 16-byte aligned, size a multiple of 16.  The KV
+// stream is read exactly once, so it is marked evict-first in L2.
+__device__ __forceinline__ void bulk_load_evict_first(void* dst, const void* src, uint32_t bytes,
+                                                      uint64_t* bar, uint64_t policy)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+            smem_addr(dst)),
+        "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar)
+{
+    asm volatile("cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_addr(dst)),
+                 "l"(src), "r"(bytes), "r"(smem_addr(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ uint64_t l2_policy_evict_first()
+{
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+// Programmatic dependent launch: wait for the preceding kernel of the stream to
+// finish (and its writes to be visible); allow the next kernel to start its prologue.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Named barrier for a subset of warps (id 0 is __syncthreads).
+__device__ __forceinline__ void named_barrier(int id, int threads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+__device__ __forceinline__ float fast_exp2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// ---- element types -------------------------------------------------------
+template <typename T> struct Elt;
+
+template <> struct Elt<__half> {
+    static __device__ __forceinline__ float2 to_float2(uint32_t w)
+    {
+        __half2 h = *reinterpret_cast<const __half2*>(&w);
+        return __half22float2(h);
+    }
+    static __device__ __forceinline__ __half from_float(float x) { return __float2half_rn(x); }
+    static __device__ __forceinline__ __half from_double(double x) { return __double2half(x); }
+    static __device__ __forceinline__ double to_double(__half x) { return (double)__half2float(x); }
+};
+
+template <> struct Elt<__nv_bfloat16> {
+    static __device__ __forceinline__ float2 to_float2(uint32_t w)
+    {
+        // bfloat16 is the high half of an fp32: widening is a shift / mask.
+        return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+    }
+    static __device__ __forceinline__ __nv_bfloat16 from_float(float x) { return __float2bfloat16_rn(x); }
+    static __device__ __forceinline__ __nv_bfloat16 from_double(double x) { return __double2bfloat16(x); }
+    static __device__ __forceinline__ double to_double(__nv_bfloat16 x) { return (double)__bfloat162float(x); }
+};
+
+template <typename T>
+__device__ __forceinline__ void unpack8(const uint4& u, float (&f)[8])
+{
+    float2 a = Elt<T>::to_float2(u.x), b = Elt<T>::to_float2(u.y);
+    float2 c = Elt<T>::to_float2(u.z), d = Elt<T>::to_float2(u.w);
+    f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
+    f[4] = c.x; f[5] = c.y; f[6] = d.x; f[7] = d.y;
+}
+
+}  // namespace pkv
+
+#endif  // PKV_DEVICE_CUH_

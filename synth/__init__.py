@@ -269,3 +269,29 @@ def pool_values_torch(s, device, seed=None):
                 sel = kp[layer][pages, :, prow, :].float() * 8.0
                 kp[layer][pages, :, prow, :] = sel.to(tdt)
     return kp, vp
+
+
+def step_values_torch(s, n_sets, device, seed=None):
+    """n_sets independent (q, k, v) inputs for every layer, generated on `device`
+    by torch's seeded generator: tensors [n_sets, layers, B, H, d] of the storage type."""
+    import torch
+    tdt = torch.float16 if s.dtype == "f16" else torch.bfloat16
+    g = torch.Generator(device=device)
+    g.manual_seed((value_seed(s) if seed is None else seed) + 3_000_000)
+    out = []
+    for heads in (s.q_heads, s.kv_heads, s.kv_heads):
+        x = torch.randn((n_sets, s.num_layers, s.batch, heads, s.head_dim), generator=g, device=device,
+                        dtype=torch.float32)
+        out.append(x.to(tdt))
+    return tuple(out)
+
+
+def mini_pool_numpy(s, b, g, seed):
+    """K and V pages of one (sequence, kv head) as a standalone pool
+    [pages(b), 1, P, d] with an identity page table, numpy PCG64 (host-only runs)."""
+    rng = _rng(seed)
+    np_b = (int(s.context_lens[b]) + s.page_size - 1) // s.page_size
+    shape = (np_b, 1, s.page_size, s.head_dim)
+    k = round_f32(rng.standard_normal(shape, dtype=np.float32), s.dtype)
+    v = round_f32(rng.standard_normal(shape, dtype=np.float32), s.dtype)
+    return k, v
