@@ -21,7 +21,8 @@
  *     launch; a call that returns an error has launched nothing.
  *   - Memory: every device pointer is owned by the caller (allocated by any CUDA
  *     allocator, e.g. PyTorch).  The library allocates no device memory on any path;
- *     scratch comes from a caller-provided workspace.
+ *     scratch comes from a caller-provided workspace (paged_decode_attention_noalloc
+ *     instead uses a fixed array compiled into the library).
  *   - Streams: device work is enqueued asynchronously on the caller's stream (a
  *     cudaStream_t; NULL = legacy default stream); no entry point synchronises the
  *     host except kv_get_device_error().  Consecutive kernels of the library use
@@ -199,6 +200,32 @@ int paged_decode_attention(const pkv_pool* pool, int layer, void* out, const voi
                            const int32_t* context_lens, int batch, int q_heads, int kv_heads,
                            float scale, int num_splits, void* workspace, size_t workspace_bytes,
                            pkv_stream_t stream);
+
+/*
+ * paged_decode_attention for callers that cannot allocate device memory.  The pages have
+ * no counterpart: this is a library convenience, not part of the method.
+ * Who needs it: a plugin whose host application owns all device memory and gives the
+ * plugin no allocator, a runtime whose caching allocator has already reserved the whole
+ * GPU, or a serving loop that may not call cudaMalloc (it synchronises the device).
+ * Arguments, results and errors are those of paged_decode_attention, without the
+ * workspace: the scratch is a fixed 4 MiB array inside the library, in device memory
+ * that every GPU which loads the library holds until the process exits.
+ *   - A call whose scratch would exceed 4 MiB (2 x num_splits x (q_heads / kv_heads) x
+ *     (head_dim + 2) fp32 values plus the batch's page prefix sums) is rejected with
+ *     PKV_ERR_NO_SPACE and launches nothing.  On B200 the automatic split count
+ *     (num_splits = 0) fits for every shape and batch size the kernels accept.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call before any
+ *     stream capture begins.
+ *   - All calls on a device share the one array, which keeps the previous call's
+ *     contents; nothing in it needs clearing.  Calls that overlap on the GPU (different
+ *     streams, or several host threads) race on it: order them on one stream.
+ *   - No cudaMalloc, cudaFree or allocating library routine is called.
+ */
+int paged_decode_attention_noalloc(const pkv_pool* pool, int layer, void* out, const void* q,
+                                   const int32_t* block_tables, int max_pages_per_seq,
+                                   const int32_t* context_lens, int batch, int q_heads, int kv_heads,
+                                   float scale, int num_splits, pkv_stream_t stream);
 
 /*
  * Read and clear the device error word (PKV_DEVERR_* bits) of the current device.

@@ -10,6 +10,7 @@
 
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "decode_attention.cuh"
 #include "pagedkv.h"
@@ -253,4 +254,63 @@ extern "C" int kv_get_device_error(uint32_t* err_out)
     if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return PKV_ERR_CUDA;
     *err_out = v;
     return PKV_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Decode attention with library-owned scratch, for callers that cannot allocate.
+//
+// Some callers have no way to obtain device memory of their own: a plugin whose host
+// application owns every device allocation and hands the plugin none, a runtime whose
+// caching allocator has already reserved the whole device, or a latency-critical
+// serving loop that forbids cudaMalloc because it synchronises the device.  This entry
+// point serves them: its scratch is one fixed array in the library's device memory.
+namespace pkv {
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t(4) << 20;   // 4 MiB per device
+
+// Held by every GPU that loads the library, until the process exits.  In host code
+// this name is only a stand-in for the symbol; its device address comes from
+// cudaGetSymbolAddress below.
+__device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+std::mutex g_static_scratch_mutex;
+void* g_static_scratch_addr[kMaxDevices] = {};
+
+// Device address of g_static_scratch on the current device, looked up once per device.
+int static_scratch_address(void** out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return PKV_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return PKV_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_static_scratch_mutex);
+    if (!g_static_scratch_addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return PKV_ERR_CUDA;
+        g_static_scratch_addr[dev] = p;
+    }
+    *out = g_static_scratch_addr[dev];
+    return PKV_OK;
+}
+
+}  // namespace
+}  // namespace pkv
+
+extern "C" int paged_decode_attention_noalloc(const pkv_pool* pool, int layer, void* out, const void* q,
+                                              const int32_t* block_tables, int max_pages_per_seq,
+                                              const int32_t* context_lens, int batch, int q_heads, int kv_heads,
+                                              float scale, int num_splits, pkv_stream_t stream)
+{
+    if (!pool || batch < 0 || q_heads <= 0 || kv_heads <= 0 || q_heads % kv_heads || num_splits < 0)
+        return PKV_ERR_INVALID_ARG;
+    if (num_splits > 0 && workspace_layout(batch, q_heads / kv_heads, pool->head_dim, num_splits).total >
+                              kStaticScratchBytes)
+        return PKV_ERR_NO_SPACE;
+    void* scratch = nullptr;
+    const int st = static_scratch_address(&scratch);
+    if (st != PKV_OK) return st;
+    // Nothing in the scratch has to start at zero: every value a call reads was written
+    // earlier in the same call, so the previous call's contents do no harm.
+    return paged_decode_attention(pool, layer, out, q, block_tables, max_pages_per_seq, context_lens, batch,
+                                  q_heads, kv_heads, scale, num_splits, scratch, kStaticScratchBytes, stream);
 }
