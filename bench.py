@@ -38,7 +38,7 @@ FALLBACK_HBM_GBS = 6650.0
 NOMINAL_HBM_GBS = 8000.0
 METRIC = "paged decode-attention KV-read GB/s (% of HBM peak); us per layer-step"
 UNIT = "GB/s"
-INPUT_SETS = 16          # distinct per-step q/k/v sets cycled through the timed steps
+INPUT_SETS = 4           # distinct per-step q/k/v sets (one captured step each) cycled through
 
 
 def parse_args(argv=None):
@@ -248,6 +248,7 @@ def workload_config(s, args):
 def run_ours(args):
     import torch
     import paged_kv_cache_460_b200 as pkv
+    from paged_kv_cache_460_b200.step import DecodeStep
 
     world, rank, local = dist_setup(args)
     torch.cuda.set_device(local)
@@ -259,33 +260,20 @@ def run_ours(args):
 
     s = synth.spec(args.workload, num_layers=args.layers)
     L = s.num_layers
-    tdt = torch.float16 if s.dtype == "f16" else torch.bfloat16
     kp, vp = synth.pool_values_torch(s, dev)
     pool = pkv.KVPool(kp, vp)
     qs, ks, vs = synth.step_values_torch(s, INPUT_SETS, dev)
-    bt = torch.from_numpy(s.block_tables).to(dev)
-    cl = torch.from_numpy(s.context_lens).to(dev)
-    pos = torch.from_numpy(s.positions).to(dev)
-    slots = torch.from_numpy(pkv.pkv_slot_mapping(s.block_tables, s.positions, s.page_size)).to(dev)
-    ws = pkv.DecodeWorkspace(s.batch, s.q_heads, s.kv_heads, s.head_dim, s.page_size, tdt, args.splits, device=dev)
-    out = torch.empty((L, s.batch, s.q_heads, s.head_dim), dtype=tdt, device=dev)
-    scale = 1.0 / math.sqrt(s.head_dim)
-    stream = torch.cuda.current_stream()
+    steps = []
+    for j in range(INPUT_SETS):
+        st = DecodeStep(pool, s.batch, s.q_heads, s.max_pages, theta=s.theta, num_splits=args.splits, device=dev)
+        st.set_metadata(s.block_tables, s.context_lens, s.positions, non_blocking=False)
+        st.q.copy_(qs[j])
+        st.k.copy_(ks[j])
+        st.v.copy_(vs[j])
+        steps.append(st)
+    del qs, ks, vs
     small = s.kv_bytes_read() * L < 2 * 126e6
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev) if small else None
-
-    def step(i, events=None):
-        j = i % INPUT_SETS
-        for layer in range(L):
-            q, k, v = qs[j, layer], ks[j, layer], vs[j, layer]
-            pkv.rope_apply(q, k, pos, s.theta, stream)
-            pkv.paged_kv_append(pool, layer, k, v, slots, stream)
-            if events is not None:
-                events[layer][0].record(stream)
-            pkv.paged_decode_attention(pool, layer, out[layer], q, bt, cl, scale, num_splits=ws.num_splits,
-                                       workspace=ws, stream=stream)
-            if events is not None:
-                events[layer][1].record(stream)
 
     def sync_all():
         torch.cuda.synchronize()
@@ -293,67 +281,73 @@ def run_ours(args):
             torch.distributed.barrier()
         torch.cuda.synchronize()
 
+    # warm-up: eager steps (sets kernel attributes), then graph capture and replays
     for i in range(args.warmup):
-        step(i)
+        steps[i % INPUT_SETS].eager()
+    for st in steps:
+        st.capture()
+    attn = torch.cuda.CUDAGraph()                 # the 32 attention calls of one step alone
+    cs = torch.cuda.Stream()
+    cs.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(cs), torch.cuda.graph(attn, stream=cs):
+        st0 = steps[0]
+        for layer in range(L):
+            pkv.paged_decode_attention(pool, layer, st0.out[layer], st0.q[layer], st0.block_tables,
+                                       st0.context_lens, st0.scale, num_splits=st0.workspace.num_splits,
+                                       workspace=st0.workspace)
+    torch.cuda.current_stream().wait_stream(cs)
+    for i in range(args.warmup):
+        steps[i % INPUT_SETS].replay()
+        attn.replay()
     sync_all()
+
+    stream = torch.cuda.current_stream()
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.3)
-    # ---- phase A: whole steps (headline value)
+    # ---- phase A: whole steps (headline value), one graph launch per step
     sync_all()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for i in range(args.steps):
         if flush is not None:
             flush.zero_()
-        step(i)
+        steps[i % INPUT_SETS].replay()
     e1.record(stream)
     sync_all()
     ms_total = max_over_ranks(e0.elapsed_time(e1), world, dev)
-    # ---- phase B: the attention call timed per launch (roofline)
-    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(L)]
-          for _ in range(args.steps)]
-    sync_all()
+    # ---- phase B: the attention calls alone (roofline of the dominant kernel)
+    b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    b0.record(stream)
     for i in range(args.steps):
         if flush is not None:
             flush.zero_()
-        step(i, ev[i])
+        attn.replay()
+    b1.record(stream)
     sync_all()
-    attn_ms = [ev[i][l][0].elapsed_time(ev[i][l][1]) for i in range(args.steps) for l in range(L)]
-    attn_ms_mean = max_over_ranks(float(np.mean(attn_ms)), world, dev)
+    attn_ms_mean = max_over_ranks(b0.elapsed_time(b1), world, dev) / (args.steps * L)
     clk = clocks.stop()
 
-    # ---- e2e through the public API, host buffers in and out
+    # ---- e2e through the public API: host buffers in and out, one DecodeStep per step
     e2e = None
     if not args.no_e2e:
-        hq = torch.empty(qs.shape[1:], dtype=tdt).pin_memory()
-        hk = torch.empty(ks.shape[1:], dtype=tdt).pin_memory()
-        hv = torch.empty(vs.shape[1:], dtype=tdt).pin_memory()
-        hq.copy_(qs[0])
-        hk.copy_(ks[0])
-        hv.copy_(vs[0])
-        h_meta = [torch.from_numpy(x).pin_memory() for x in
-                  (s.block_tables, s.context_lens, s.positions, pkv.pkv_slot_mapping(s.block_tables, s.positions,
-                                                                                     s.page_size))]
-        hout = torch.empty(out.shape, dtype=tdt).pin_memory()
-        dq, dk, dv = torch.empty_like(qs[0]), torch.empty_like(ks[0]), torch.empty_like(vs[0])
-        dmeta = [torch.empty_like(x, device=dev) for x in h_meta]
-        h2d = sum(t.numel() * t.element_size() for t in [hq, hk, hv] + h_meta)
+        st = steps[0]
+        tdt = st.q.dtype
+        hq = torch.empty(st.q.shape, dtype=tdt).pin_memory()
+        hk = torch.empty(st.k.shape, dtype=tdt).pin_memory()
+        hv = torch.empty(st.v.shape, dtype=tdt).pin_memory()
+        hq.copy_(st.q)
+        hk.copy_(st.k)
+        hv.copy_(st.v)
+        hout = torch.empty(st.out.shape, dtype=tdt).pin_memory()
+        hbt = torch.from_numpy(s.block_tables).pin_memory()
+        hcl = torch.from_numpy(s.context_lens).pin_memory()
+        hpos = torch.from_numpy(s.positions).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hbt, hcl, hpos)) + 8 * s.batch
         d2h = hout.numel() * hout.element_size()
-
-        def e2e_step():
-            for dst, src in zip([dq, dk, dv] + dmeta, [hq, hk, hv] + h_meta):
-                dst.copy_(src, non_blocking=True)
-            dbt, dcl, dpos, dslot = dmeta
-            for layer in range(L):
-                pkv.rope_apply(dq[layer], dk[layer], dpos, s.theta, stream)
-                pkv.paged_kv_append(pool, layer, dk[layer], dv[layer], dslot, stream)
-                pkv.paged_decode_attention(pool, layer, out[layer], dq[layer], dbt, dcl, scale,
-                                           num_splits=ws.num_splits, workspace=ws, stream=stream)
-            hout.copy_(out, non_blocking=True)
-
         for _ in range(max(1, args.warmup)):
-            e2e_step()
+            st.set_metadata(hbt, hcl, hpos)
+            st.run(hq, hk, hv, hout)
         sync_all()
         n_e2e = max(1, args.steps // 2)
         a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -361,13 +355,13 @@ def run_ours(args):
         for _ in range(n_e2e):
             if flush is not None:
                 flush.zero_()
-            e2e_step()
+            st.set_metadata(hbt, hcl, hpos)
+            st.run(hq, hk, hv, hout)
         a1.record(stream)
         sync_all()
         ms_e2e = max_over_ranks(a0.elapsed_time(a1), world, dev)
         e2e = {"value": world * s.kv_bytes_read() * L * n_e2e / (ms_e2e * 1e-3) / 1e9, "unit": UNIT,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "ms_per_step": ms_e2e / n_e2e}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e / n_e2e}
 
     err = pkv.kv_get_device_error()
     if err:
@@ -396,11 +390,15 @@ def run_ours(args):
                          "frac_of_8tbs": achieved / NOMINAL_HBM_GBS},
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": args.steps * L * 4 * world,
-            "num_splits": ws.num_splits,
+            "gpu_launches": args.steps * steps[0].kernels_per_step * world,
+            "num_splits": steps[0].workspace.num_splits,
+            "launch": "one CUDA graph per step (%d kernels)" % steps[0].kernels_per_step,
             "clocks": clk,
         }
         print(json.dumps(line), flush=True)
+    for st in steps:
+        st.graph = None
+    attn = None
     if world > 1:
         torch.distributed.destroy_process_group()
     return 0

@@ -137,7 +137,8 @@ int pkv_slot_mapping(const int32_t* block_tables, int max_pages_per_seq, const i
  *   position are left untouched.
  * Pair i = (x[2i], x[2i+1]) of every head turns by pos * theta^(-2i/head_dim).  The angle,
  * its cosine and sine and the rotation are evaluated in fp64 and rounded once to the
- * element type.  head_dim: 64 or 128.  Either q or k may be NULL (with its head count 0).
+ * element type.  head_dim: 64 or 128.  Either q or k may be NULL (with its head count 0);
+ * q and k 16-byte aligned.
  */
 int rope_apply(void* q, void* k, const int32_t* positions, int n_tokens, int q_heads,
                int kv_heads, int head_dim, double theta, int dtype, pkv_stream_t stream);
@@ -152,6 +153,19 @@ int rope_apply(void* q, void* k, const int32_t* positions, int n_tokens, int q_h
  */
 int paged_kv_append(const pkv_pool* pool, int layer, const void* k, const void* v,
                     const int64_t* slot_mapping, int n_tokens, pkv_stream_t stream);
+
+/*
+ * rope_apply followed by paged_kv_append in one launch ([ENGINE] s4.3 rotate then append;
+ * s5.3 fuse small kernels and cut launch overhead): q [n_tokens][q_heads][head_dim] and
+ * k [n_tokens][kv_heads][head_dim] are rotated in place at positions[i] (fp64, one rounding),
+ * and the rotated k and v [n_tokens][kv_heads][head_dim] are copied bit for bit into the
+ * pool slots slot_mapping[i] of `layer` (negative = skip; past the pool = skip and set
+ * PKV_DEVERR_BAD_SLOT).  kv_heads, head_dim and the element type are the pool's.  Results
+ * are identical to the two separate calls.  q, k, v 16-byte aligned.
+ */
+int rope_append(const pkv_pool* pool, int layer, void* q, void* k, const void* v,
+                const int32_t* positions, const int64_t* slot_mapping, int n_tokens, int q_heads,
+                double theta, pkv_stream_t stream);
 
 /*
  * Number of work partitions paged_decode_attention uses when called with num_splits = 0 on

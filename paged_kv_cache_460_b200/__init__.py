@@ -23,7 +23,7 @@ from ._lib import (PKV_BF16, PKV_DEVERR_BAD_PAGE, PKV_DEVERR_BAD_SLOT, PKV_DEVER
                    PagedKVError, lib)
 
 __all__ = [
-    "KVPool", "rope_apply", "paged_kv_append", "paged_decode_attention", "pkv_slot_mapping",
+    "KVPool", "rope_apply", "paged_kv_append", "rope_append", "paged_decode_attention", "pkv_slot_mapping",
     "pkv_kv_cache_bytes", "pkv_decode_workspace_size", "pkv_decode_default_splits",
     "kv_get_device_error", "DecodeWorkspace", "PagedKVError", "PKV_F16", "PKV_BF16",
     "PKV_DEVERR_BAD_PAGE", "PKV_DEVERR_BAD_SLOT", "PKV_DEVERR_TIMEOUT",
@@ -179,6 +179,20 @@ def paged_kv_append(pool, layer, k, v, slot_mapping, stream=None):
     st = lib().paged_kv_append(pool.handle, layer, _ptr(k), _ptr(v), _ptr(slot_mapping), k.shape[0],
                                _stream(stream))
     _lib.check("paged_kv_append", st)
+
+
+def rope_append(pool, layer, q, k, v, positions, slot_mapping, theta=10000.0, stream=None):
+    """RoPE on q [n, q_heads, d] and k [n, kv_heads, d] (in place), then append k and v
+    into the pool's slots -- one launch, same results as rope_apply + paged_kv_append."""
+    torch = _torch()
+    _need(q, "q", pool.dtype)
+    _need(k, "k", pool.dtype)
+    _need(v, "v", pool.dtype)
+    _need(positions, "positions", torch.int32)
+    _need(slot_mapping, "slot_mapping", torch.int64)
+    st = lib().rope_append(pool.handle, layer, _ptr(q), _ptr(k), _ptr(v), _ptr(positions), _ptr(slot_mapping),
+                           k.shape[0], q.shape[1], float(theta), _stream(stream))
+    _lib.check("rope_append", st)
 
 
 class DecodeWorkspace:

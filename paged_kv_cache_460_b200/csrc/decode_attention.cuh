@@ -13,19 +13,23 @@
 // W = kv_heads * sum_b pages(b) "page-head" units in (sequence, kv head, page) order and
 // cut it into num_splits equal contiguous ranges, one per CTA.  Every CTA therefore
 // streams the same number of bytes whatever the length mix, and a (sequence, kv head)
-// pair is cut at most at range boundaries.  Inside a CTA:
-//   - a producer warp walks its range, reads the page table, and for each page issues
-//     two 1-D bulk (TMA) copies -- the page's K and V chunks of page_size*head_dim
-//     contiguous elements -- into a ring of shared-memory slots, plus the group's q
-//     rows when a (sequence, kv head) segment begins;
-//   - NW consumer warps all work on each page, warp w on its page_size/NW token rows:
-//     q.k dot products with 16-byte shared loads and shuffle reductions, an online
-//     softmax (running max m, running sum l, unnormalised output o), all in fp32 in
-//     the log2 domain;
-//   - at the end of a segment the warps' (m, l, o) are combined through shared memory;
-//     a segment wholly inside the range is normalised and written as the output, a cut
-//     one is written to one of the CTA's two partial slots (2c: the segment began before
-//     the range, 2c+1: it continues after it) for the merge kernel.
+// pair is cut at most at range boundaries.  Inside a CTA, warp w takes units
+// w, w + NW, w + 2 NW, ... of the range: a whole page-head per warp, so each per-page
+// reduction covers P tokens.  Every warp streams its own pages through a private ring
+// of DEPTH shared-memory slots with 16-byte cp.async copies (K chunk, V chunk and, when
+// the warp enters a new (sequence, kv head), the group's q rows), DEPTH pages ahead of
+// the one it computes; the page ids come from a 32-entry window of the page table that
+// the lanes fetch together.  Many independent warp streams keep enough bytes in flight
+// to saturate HBM; a single TMA-issuing thread per CTA could not (one bulk copy per
+// thread-instruction issue slot capped it near 4 TB/s on this access pattern).
+// Per page the warp computes q.k over its lanes' 16-byte column slices, reduces the
+// partial dots with a transposed shuffle reduction (each lane ends with one row's
+// score), updates an fp32 online softmax (running max m, sum l, unnormalised o) in
+// the log2 domain, and accumulates p.V with packed fp32 FMAs.  At the end of a segment
+// the warps' (m, l, o) are combined through shared memory: a segment wholly inside the
+// range is normalised and written as the output; a cut one is written to one of the
+// CTA's two partial slots (2c: it began before the range, 2c+1: it continues after it)
+// for the merge kernel.
 #ifndef PKV_DECODE_ATTENTION_CUH_
 #define PKV_DECODE_ATTENTION_CUH_
 
@@ -33,9 +37,9 @@
 
 namespace pkv {
 
-constexpr int kConsumerWarps = 4;
-constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;
-constexpr int kRingBudgetBytes = 96 * 1024;
+constexpr int kDecodeWarps = 4;
+constexpr int kDecodeThreads = kDecodeWarps * 32;
+constexpr int kRingBudgetBytes = 68 * 1024;    // three CTAs per SM at page 16, head_dim 128
 constexpr int kMetaHeaderBytes = 16;   // int64 chunk, int64 total units
 
 struct DecodeParams {
@@ -64,14 +68,13 @@ struct DecodeShape {
     static constexpr int kChunk = P * D * 2;                 // bytes of one (page, head)
     static constexpr int kQBytes = G * D * 2;
     static constexpr int kSlot = 2 * kChunk + kQBytes;
-    static constexpr int kStagesRaw = kRingBudgetBytes / kSlot;
-    static constexpr int kStages = kStagesRaw < 2 ? 2 : (kStagesRaw > 16 ? 16 : kStagesRaw);
-    static constexpr int kRingBytes = kStages * kSlot;
-    static constexpr int kBarOffset = kRingBytes;
-    static constexpr int kFlagOffset = kBarOffset + 2 * kStages * 8;
-    static constexpr int kCmbOffset = align_up(kFlagOffset + 16 + 8 * 4, 16);
-    static constexpr int kCmbFloats = kConsumerWarps * G * (D + 2);
-    static constexpr int kScanOffset = kCmbOffset + 2 * kCmbFloats * 4;
+    static constexpr int kDepthRaw = kRingBudgetBytes / (kDecodeWarps * kSlot);
+    static constexpr int kDepth = kDepthRaw < 2 ? 2 : (kDepthRaw > 8 ? 8 : kDepthRaw);
+    static constexpr int kRingBytes = kDecodeWarps * kDepth * kSlot;
+    static constexpr int kCmbOffset = kRingBytes;
+    static constexpr int kCmbFloats = kDecodeWarps * G * (D + 2);
+    static constexpr int kWarpTotOffset = kCmbOffset + 2 * kCmbFloats * 4;
+    static constexpr int kScanOffset = kWarpTotOffset + 64;
     // prefix[batch+1] and lens[batch] follow
     static int smem_bytes(int batch) { return kScanOffset + 4 * (2 * batch + 1); }
 };
@@ -142,40 +145,45 @@ template <int D, int P, int G, typename T>
 __global__ void __launch_bounds__(kDecodeThreads) decode_pass1_kernel(const DecodeParams p)
 {
     using S = DecodeShape<D, P, G>;
-    constexpr int NST = S::kStages;
-    constexpr int NW = kConsumerWarps;
+    constexpr int NW = kDecodeWarps;
+    constexpr int DEPTH = S::kDepth;
+    constexpr int LPR = D / 8;            // lanes per K/V row (16 bytes each)
+    constexpr int RPI = 32 / LPR;         // rows covered by one warp-wide 16-byte access
+    constexpr int NIT = P / RPI;          // accesses per page chunk
+    constexpr int QV = S::kQBytes / 16;   // 16-byte pieces of the group's q rows
+    static_assert(NIT <= LPR, "a page's rows must fit the transposed reduction");
     extern __shared__ __align__(128) unsigned char smem[];
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::kBarOffset);
-    uint64_t* empty = full + NST;
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S::kFlagOffset);
-    int* issued = reinterpret_cast<int*>(smem + S::kFlagOffset + 4);
-    volatile int* drain_abort = reinterpret_cast<volatile int*>(smem + S::kFlagOffset + 8);
-    int* warp_tot = reinterpret_cast<int*>(smem + S::kFlagOffset + 16);
     float* cmb = reinterpret_cast<float*>(smem + S::kCmbOffset);
+    int* warp_tot = reinterpret_cast<int*>(smem + S::kWarpTotOffset);
     int* prefix = reinterpret_cast<int*>(smem + S::kScanOffset);
     int* lens = prefix + p.batch + 1;
-
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    if (tid == 0) {
-        for (int s = 0; s < NST; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], NW);
-        }
-        *abort_flag = 0;
-        *issued = 0;
-        *drain_abort = 0;
-        fence_barrier_init();
-    }
-    // The prologue reads only the caller's lengths; the pool and the workspace are
-    // touched after pdl_wait, once the previous kernel on the stream has finished.
+
+    // Prologue: reads only the caller's lengths and page table, which the previous
+    // kernel on the stream does not write; pool, q and workspace wait for pdl_wait.
     block_page_prefix<P>(p.context_lens, p.batch, prefix, lens, warp_tot);
     __syncthreads();
-
     const int Hkv = p.kv_heads;
     const long long W = (long long)Hkv * prefix[p.batch];
     const long long chunk = W > 0 ? (W + p.num_splits - 1) / p.num_splits : 1;
     const long long r0 = (long long)blockIdx.x * chunk;
     const long long r1 = min(W, r0 + chunk);
+    const long long n_mine = r1 - r0 > warp ? (r1 - r0 - warp + NW - 1) / NW : 0;   // this warp's pages
+
+    // lane l holds the page id of this warp's page win0 + l (-1: outside the table)
+    auto load_window = [&](long long win0) {
+        const long long k = win0 + lane;
+        int id = 0;
+        if (k < n_mine) {
+            int bb, gg, jj;
+            locate_unit(r0 + warp + k * NW, prefix, p.batch, Hkv, bb, gg, jj);
+            id = jj < p.max_pages ? p.block_tables[(long long)bb * p.max_pages + jj] : -1;
+        }
+        return id;
+    };
+    long long win0 = 0;
+    int win = load_window(0);
+
     pdl_wait();
     pdl_launch_dependents();
     if (blockIdx.x == 0) {
@@ -189,196 +197,248 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_pass1_kernel(const Deco
     }
     if (r0 >= r1) return;
 
-    if (warp == NW) {
-        // ------------------------------------------------------------ producer
-        const uint64_t policy = l2_policy_evict_first();
-        int b, g, j;
-        locate_unit(r0, prefix, p.batch, Hkv, b, g, j);
-        int np = prefix[b + 1] - prefix[b];
-        int win_b = -1, win_j0 = 0, bt = 0;
-        int it = 0;
-        for (long long u = r0; u < r1; ++u, ++it) {
-            const int slot = it % NST;
-            if (it >= NST && !mbar_wait_bounded(&empty[slot], ((it / NST) - 1) & 1, abort_flag)) break;
-            if (b != win_b || j < win_j0 || j >= win_j0 + 32) {
-                win_b = b;
-                win_j0 = j & ~31;
-                const int jj = win_j0 + lane;
-                // a length beyond the table's width yields -1: flagged, never dereferenced
-                bt = jj < np ? (jj < p.max_pages ? p.block_tables[(long long)b * p.max_pages + jj] : -1) : 0;
-            }
-            const int page = __shfl_sync(0xffffffffu, bt, j - win_j0);
-            if (lane == 0) {
-                unsigned char* s = smem + slot * S::kSlot;
-                const bool ok = (unsigned)page < (unsigned)p.num_pages;
-                const bool seg_start = (j == 0) || (it == 0);
-                const uint32_t bytes = (ok ? 2u * S::kChunk : 0u) + (seg_start ? (uint32_t)S::kQBytes : 0u);
-                if (!ok) atomicOr(&g_error_word, PKV_DEVERR_BAD_PAGE);
-                fence_proxy_async_smem();
-                mbar_arrive_expect_tx(&full[slot], bytes);
-                if (ok) {
-                    const long long off = ((long long)page * Hkv + g) * (P * D);
-                    bulk_load_evict_first(s, static_cast<const T*>(p.k) + off, S::kChunk, &full[slot], policy);
-                    bulk_load_evict_first(s + S::kChunk, static_cast<const T*>(p.v) + off, S::kChunk, &full[slot],
-                                          policy);
-                }
-                if (seg_start)
-                    bulk_load(s + 2 * S::kChunk,
-                              static_cast<const T*>(p.q) + ((long long)b * p.q_heads + (long long)g * G) * D,
-                              S::kQBytes, &full[slot]);
-            }
-            __syncwarp();
-            next_unit(b, g, j, np, prefix, Hkv, p.batch);
+    unsigned char* ring = smem + warp * DEPTH * S::kSlot;
+
+    // ---- issue side: this warp's page k (iterator at unit r0 + warp + k NW)
+    int ib = 0, ig = 0, ij = 0, inp = 1, qb = -1, qg = -1;
+    if (n_mine > 0) {
+        locate_unit(r0 + warp, prefix, p.batch, Hkv, ib, ig, ij);
+        inp = prefix[ib + 1] - prefix[ib];
+    }
+    auto issue = [&](long long k) {
+        if (k >= win0 + 32) {
+            win0 = k;
+            win = load_window(k);
         }
-        if (lane == 0) *issued = it;
-    } else {
-        // ------------------------------------------------------------ consumers
-        constexpr int LPR = D / 8;            // lanes per K/V row (16 bytes each)
-        constexpr int RPI = 32 / LPR;         // rows per warp-wide load
-        constexpr int TPW = P / NW;           // token rows per warp per page
-        constexpr int NIT = TPW / RPI;
-        static_assert(TPW % RPI == 0, "page rows must split evenly over the warps");
-        const int r = lane / LPR, c = lane % LPR;
-        float qf[G][8], o[G][8], m[G], l[G];
-        int b, g, j;
-        locate_unit(r0, prefix, p.batch, Hkv, b, g, j);
-        int np = prefix[b + 1] - prefix[b];
-        int seg = 0;
-        int it = 0;
-        bool live = true;
-        for (long long u = r0; u < r1; ++u, ++it) {
-            const int slot = it % NST;
-            if (live) live = mbar_wait_bounded(&full[slot], (it / NST) & 1, abort_flag);
-            const unsigned char* s = smem + slot * S::kSlot;
-            const bool seg_start = (j == 0) || (it == 0);
-            if (seg_start) {
+        const int page = __shfl_sync(0xffffffffu, win, (int)(k - win0));
+        unsigned char* slot = ring + (int)(k % DEPTH) * S::kSlot;
+        if ((unsigned)page < (unsigned)p.num_pages) {
+            const long long off = ((long long)page * Hkv + ig) * (P * D);
+            const unsigned char* ks = reinterpret_cast<const unsigned char*>(static_cast<const T*>(p.k) + off);
+            const unsigned char* vs = reinterpret_cast<const unsigned char*>(static_cast<const T*>(p.v) + off);
+#pragma unroll
+            for (int n = 0; n < S::kChunk / 512; ++n) {
+                cp_async16(slot + n * 512 + lane * 16, ks + n * 512 + lane * 16);
+                cp_async16(slot + S::kChunk + n * 512 + lane * 16, vs + n * 512 + lane * 16);
+            }
+        } else if (lane == 0) {
+            atomicOr(&g_error_word, PKV_DEVERR_BAD_PAGE);   // never dereferenced
+        }
+        if (ib != qb || ig != qg) {           // first page of a (sequence, kv head) for this warp
+            qb = ib;
+            qg = ig;
+            const unsigned char* qs = reinterpret_cast<const unsigned char*>(
+                static_cast<const T*>(p.q) + ((long long)ib * p.q_heads + (long long)ig * G) * D);
+            for (int n = lane; n < QV; n += 32) cp_async16(slot + 2 * S::kChunk + n * 16, qs + n * 16);
+        }
+        if (ij + NW < inp) {
+            ij += NW;                          // common case: same (sequence, kv head)
+        } else {
+            for (int t = 0; t < NW; ++t) next_unit(ib, ig, ij, inp, prefix, Hkv, p.batch);
+        }
+    };
+#pragma unroll
+    for (int k = 0; k < DEPTH; ++k) {
+        if (k < n_mine) issue(k);
+        cp_async_commit();
+    }
+
+    // ---- compute side
+    const int r = lane / LPR, c = lane % LPR;
+    // After the transposed reduction lane holds the score of row i_own * RPI + r.
+    int i_own = 0;
+#pragma unroll
+    for (int m = LPR / 2, w8 = NIT / 2; w8 >= 1; m >>= 1, w8 >>= 1)
+        if (lane & m) i_own += w8;
+    const int tok_own = i_own * RPI + r;
+    // Lanes below the last halving mask hold duplicates; only the lowest counts in l.
+    const bool primary = (lane & (LPR / NIT - 1)) == 0;
+    float qf[G][8], o[G][8], m_run[G], l_run[G];
+#pragma unroll
+    for (int gi = 0; gi < G; ++gi) {
+        m_run[gi] = -INFINITY;
+        l_run[gi] = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o[gi][e] = 0.f;
+    }
+    int b, g, j;
+    locate_unit(r0, prefix, p.batch, Hkv, b, g, j);
+    int np = prefix[b + 1] - prefix[b];
+    int seg = 0, cb = -1, cg = -1;
+    long long kc = 0;                         // this warp's pages consumed
+    int it = 0;
+    for (long long u = r0; u < r1; ++u, ++it) {
+        if (it % NW == warp) {
+            cp_async_wait<DEPTH - 1>();         // page kc has landed (this lane's copies)
+            __syncwarp();                       // ... and every lane's (q is read across lanes)
+            const unsigned char* s = ring + (int)(kc % DEPTH) * S::kSlot;
+            if (b != cb || g != cg) {           // first page of this segment for this warp
+                cb = b;
+                cg = g;
 #pragma unroll
                 for (int gi = 0; gi < G; ++gi) {
                     const uint4 qu = *reinterpret_cast<const uint4*>(s + 2 * S::kChunk + (gi * D + c * 8) * 2);
                     unpack8<T>(qu, qf[gi]);
-                    m[gi] = -INFINITY;
-                    l[gi] = 0.f;
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) o[gi][e] = 0.f;
                 }
             }
             const int nvalid = min(P, lens[b] - j * P);
-            float kf[NIT][8], vf[NIT][8];
+            // ---- scores: partial dots over this lane's 8 columns, then a transposed
+            //      reduction that leaves one finished row score per lane
+            float sc[G];
+            {
+                float v[G][NIT];
 #pragma unroll
-            for (int n = 0; n < NIT; ++n) {
-                const int tok = warp * TPW + n * RPI + r;
-                const uint4 ku = *reinterpret_cast<const uint4*>(s + (tok * D + c * 8) * 2);
-                const uint4 vu = *reinterpret_cast<const uint4*>(s + S::kChunk + (tok * D + c * 8) * 2);
-                unpack8<T>(ku, kf[n]);
-                unpack8<T>(vu, vf[n]);
-                if (tok >= nvalid) {
+                for (int i = 0; i < NIT; ++i) {
+                    const uint4 ku = *reinterpret_cast<const uint4*>(s + i * 512 + lane * 16);
+                    float kf[8];
+                    unpack8<T>(ku, kf);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) vf[n][e] = 0.f;   // rows past the context may hold anything
+                    for (int gi = 0; gi < G; ++gi) {
+                        float2 a = make_float2(qf[gi][0] * kf[0], qf[gi][1] * kf[1]);
+#pragma unroll
+                        for (int e = 2; e < 8; e += 2)
+                            a = __ffma2_rn(make_float2(qf[gi][e], qf[gi][e + 1]), make_float2(kf[e], kf[e + 1]), a);
+                        v[gi][i] = a.x + a.y;
+                    }
                 }
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[slot]);
-#pragma unroll
-            for (int gi = 0; gi < G; ++gi) {
-                float sc[NIT];
-                float pm = -INFINITY;
-#pragma unroll
-                for (int n = 0; n < NIT; ++n) {
-                    float dot = 0.f;
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) dot = fmaf(qf[gi][e], kf[n][e], dot);
-#pragma unroll
-                    for (int mask = LPR / 2; mask > 0; mask >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, mask);
-                    const int tok = warp * TPW + n * RPI + r;
-                    sc[n] = tok < nvalid ? dot * p.scale_log2 : -INFINITY;
-                    pm = fmaxf(pm, sc[n]);
-                }
-#pragma unroll
-                for (int mask = LPR; mask < 32; mask <<= 1) pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, mask));
-                const float mn = fmaxf(m[gi], pm);
-                if (mn == -INFINITY) continue;        // no valid token seen yet by this warp
-                const float alpha = fast_exp2(m[gi] - mn);
-                m[gi] = mn;
-                float lsum = 0.f;
-#pragma unroll
-                for (int e = 0; e < 8; ++e) o[gi][e] *= alpha;
-#pragma unroll
-                for (int n = 0; n < NIT; ++n) {
-                    const float pr = fast_exp2(sc[n] - mn);
-                    lsum += pr;
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) o[gi][e] = fmaf(pr, vf[n][e], o[gi][e]);
-                }
-                l[gi] = l[gi] * alpha + lsum;
-            }
-            const bool seg_end = (j == np - 1) || (u == r1 - 1);
-            if (seg_end) {
-                float* buf = cmb + (seg & 1) * S::kCmbFloats;
 #pragma unroll
                 for (int gi = 0; gi < G; ++gi) {
-                    float lt = l[gi];
 #pragma unroll
-                    for (int mask = LPR; mask < 32; mask <<= 1) lt += __shfl_xor_sync(0xffffffffu, lt, mask);
+                    for (int n = NIT, m = LPR / 2; n > 1; n >>= 1, m >>= 1) {
+                        const bool up = (lane & m) != 0;
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        float ot = o[gi][e];
-#pragma unroll
-                        for (int mask = LPR; mask < 32; mask <<= 1) ot += __shfl_xor_sync(0xffffffffu, ot, mask);
-                        o[gi][e] = ot;
-                    }
-                    float* row = buf + (warp * G + gi) * (D + 2);
-                    if (r == 0) {
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) row[c * 8 + e] = o[gi][e];
-                        if (c == 0) {
-                            row[D] = m[gi];
-                            row[D + 1] = lt;
+                        for (int k = 0; k < n / 2; ++k) {
+                            const float send = up ? v[gi][k] : v[gi][k + n / 2];
+                            const float keep = up ? v[gi][k + n / 2] : v[gi][k];
+                            v[gi][k] = keep + __shfl_xor_sync(0xffffffffu, send, m);
                         }
                     }
-                }
-                named_barrier(1, NW * 32);
-                const long long seg0 = (long long)Hkv * prefix[b] + (long long)g * np;
-                const bool complete = seg0 >= r0 && seg0 + np <= r1;
-                const int pslot = seg0 < r0 ? 2 * blockIdx.x : 2 * blockIdx.x + 1;
-                for (int idx = tid; idx < G * D; idx += NW * 32) {
-                    const int gi = idx / D, dd = idx - gi * D;
-                    float M = -INFINITY;
 #pragma unroll
-                    for (int w = 0; w < NW; ++w) M = fmaxf(M, buf[(w * G + gi) * (D + 2) + D]);
-                    float num = 0.f, den = 0.f;
-#pragma unroll
-                    for (int w = 0; w < NW; ++w) {
-                        const float* row = buf + (w * G + gi) * (D + 2);
-                        const float wt = fast_exp2(row[D] - M);   // a warp with no tokens has m = -inf
-                        num = fmaf(wt, row[dd], num);
-                        den = fmaf(wt, row[D + 1], den);
-                    }
-                    if (complete) {
-                        T* dst = static_cast<T*>(p.out) + ((long long)b * p.q_heads + (long long)g * G + gi) * D + dd;
-                        *dst = Elt<T>::from_float(num / den);
-                    } else {
-                        p.part_o[((long long)pslot * G + gi) * D + dd] = num;
-                        if (dd == 0) {
-                            p.part_ml[((long long)pslot * G + gi) * 2 + 0] = M;
-                            p.part_ml[((long long)pslot * G + gi) * 2 + 1] = den;
-                        }
-                    }
+                    for (int m = LPR / (2 * NIT); m >= 1; m >>= 1)
+                        v[gi][0] += __shfl_xor_sync(0xffffffffu, v[gi][0], m);
+                    sc[gi] = tok_own < nvalid ? v[gi][0] * p.scale_log2 : -INFINITY;
                 }
-                ++seg;
             }
-            next_unit(b, g, j, np, prefix, Hkv, p.batch);
+            // ---- online softmax update (per query head of the group)
+            float pr[G], alpha[G];
+            bool rescale = false;
+#pragma unroll
+            for (int gi = 0; gi < G; ++gi) {
+                float pm = sc[gi];
+#pragma unroll
+                for (int m = 16; m >= LPR / NIT; m >>= 1) pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, m));
+                const float mn = fmaxf(m_run[gi], pm);   // finite: row 0 of a page is always valid
+                alpha[gi] = fast_exp2(m_run[gi] - mn);
+                rescale |= m_run[gi] != mn;
+                m_run[gi] = mn;
+                pr[gi] = fast_exp2(sc[gi] - mn);           // 0 for rows past the context
+                l_run[gi] = l_run[gi] * alpha[gi] + (primary ? pr[gi] : 0.f);
+            }
+            if (rescale) {
+#pragma unroll
+                for (int gi = 0; gi < G; ++gi)
+#pragma unroll
+                    for (int e = 0; e < 8; e += 2) {
+                        const float2 t = __fmul2_rn(make_float2(o[gi][e], o[gi][e + 1]), make_float2(alpha[gi], alpha[gi]));
+                        o[gi][e] = t.x;
+                        o[gi][e + 1] = t.y;
+                    }
+            }
+            // ---- o += p V over the page's rows
+#pragma unroll
+            for (int i = 0; i < NIT; ++i) {
+                const int row = i * RPI + r;
+                const uint4 vu = *reinterpret_cast<const uint4*>(s + S::kChunk + i * 512 + lane * 16);
+                float vf[8];
+                unpack8<T>(vu, vf);
+                if (nvalid < P && row >= nvalid) {             // only the last page of a sequence
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) vf[e] = 0.f;   // rows past the context may hold anything
+                }
+                int src = r * LPR;                              // the lane holding row i's score
+#pragma unroll
+                for (int m = LPR / 2, w8 = NIT / 2; w8 >= 1; m >>= 1, w8 >>= 1)
+                    if (i & w8) src += m;
+#pragma unroll
+                for (int gi = 0; gi < G; ++gi) {
+                    const float pi = __shfl_sync(0xffffffffu, pr[gi], src);
+#pragma unroll
+                    for (int e = 0; e < 8; e += 2) {
+                        const float2 acc = __ffma2_rn(make_float2(pi, pi), make_float2(vf[e], vf[e + 1]),
+                                                      make_float2(o[gi][e], o[gi][e + 1]));
+                        o[gi][e] = acc.x;
+                        o[gi][e + 1] = acc.y;
+                    }
+                }
+            }
+            __syncwarp();                         // every lane is done with the slot
+            if (kc + DEPTH < n_mine) issue(kc + DEPTH);
+            cp_async_commit();
+            ++kc;
         }
-    }
-    __syncthreads();
-    // Drain: a fill that no consumer waited for (only after a timeout) must land before
-    // the CTA's shared memory is released.
-    if (tid == 0) {
-        const int n = *issued;
-        for (int s = 0; s < NST && s < n; ++s) {
-            const int last = (n - 1 - s) / NST;          // index of the last fill of slot s
-            mbar_wait_bounded(&full[s], last & 1, drain_abort);
+        const bool seg_end = (j == np - 1) || (u == r1 - 1);
+        if (seg_end) {
+            // every warp publishes its (possibly empty) state of this segment
+            float* buf = cmb + (seg & 1) * S::kCmbFloats;
+#pragma unroll
+            for (int gi = 0; gi < G; ++gi) {
+                float lt = l_run[gi];
+#pragma unroll
+                for (int m = 16; m >= 1; m >>= 1) lt += __shfl_xor_sync(0xffffffffu, lt, m);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    float ot = o[gi][e];
+#pragma unroll
+                    for (int m = LPR; m < 32; m <<= 1) ot += __shfl_xor_sync(0xffffffffu, ot, m);
+                    o[gi][e] = ot;
+                }
+                float* row = buf + (warp * G + gi) * (D + 2);
+                if (r == 0) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) row[c * 8 + e] = o[gi][e];
+                    if (c == 0) {
+                        row[D] = m_run[gi];
+                        row[D + 1] = lt;
+                    }
+                }
+                m_run[gi] = -INFINITY;
+                l_run[gi] = 0.f;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) o[gi][e] = 0.f;
+            }
+            named_barrier(1, NW * 32);
+            const long long seg0 = (long long)Hkv * prefix[b] + (long long)g * np;
+            const bool complete = seg0 >= r0 && seg0 + np <= r1;
+            const int pslot = seg0 < r0 ? 2 * blockIdx.x : 2 * blockIdx.x + 1;
+            for (int idx = tid; idx < G * D; idx += NW * 32) {
+                const int gi = idx / D, dd = idx - gi * D;
+                float M = -INFINITY;
+#pragma unroll
+                for (int w = 0; w < NW; ++w) M = fmaxf(M, buf[(w * G + gi) * (D + 2) + D]);
+                float num = 0.f, den = 0.f;
+#pragma unroll
+                for (int w = 0; w < NW; ++w) {
+                    const float* row = buf + (w * G + gi) * (D + 2);
+                    const float wt = fast_exp2(row[D] - M);   // a warp with no page here has m = -inf
+                    num = fmaf(wt, row[dd], num);
+                    den = fmaf(wt, row[D + 1], den);
+                }
+                if (complete) {
+                    T* dst = static_cast<T*>(p.out) + ((long long)b * p.q_heads + (long long)g * G + gi) * D + dd;
+                    *dst = Elt<T>::from_float(num / den);
+                } else {
+                    p.part_o[((long long)pslot * G + gi) * D + dd] = num;
+                    if (dd == 0) {
+                        p.part_ml[((long long)pslot * G + gi) * 2 + 0] = M;
+                        p.part_ml[((long long)pslot * G + gi) * 2 + 1] = den;
+                    }
+                }
+            }
+            ++seg;
         }
+        next_unit(b, g, j, np, prefix, Hkv, p.batch);
     }
+    cp_async_wait<0>();
 }
 
 // One CTA per (sequence, kv head).  Sequences with no cached token get zeros; pairs

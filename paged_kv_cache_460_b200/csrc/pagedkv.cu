@@ -149,6 +149,46 @@ WorkspaceLayout workspace_layout(int batch, int group, int head_dim, int num_spl
 
 using namespace pkv;
 
+namespace pkv {
+namespace {
+
+int launch_rope_append(const RopeAppendParams& prm, int n_tokens, int dtype, cudaStream_t st)
+{
+    const int vph = prm.head_dim / 8;
+    const int nq = (prm.mode & kRopeRotate) ? prm.q_heads * vph : 0;
+    const int total = nq + ((prm.mode & kRopeAppend) ? 2 : 1) * prm.kv_heads * vph;
+    const int parts = (total + 255) / 256;
+    const dim3 grid(n_tokens, parts > 0 ? parts : 1);
+    cudaError_t e;
+    if (dtype == PKV_F16)
+        e = launch_pdl(rope_append_kernel<__half>, grid, dim3(256), 0, st, prm);
+    else
+        e = launch_pdl(rope_append_kernel<__nv_bfloat16>, grid, dim3(256), 0, st, prm);
+    return status_of(e);
+}
+
+RopeAppendParams pool_params(const pkv_pool* pool, int layer)
+{
+    RopeAppendParams prm;
+    std::memset(&prm, 0, sizeof(prm));
+    const size_t off = (size_t)layer * pool->layer_elems * 2;
+    prm.k_layer = static_cast<char*>(pool->k_base) + off;
+    prm.v_layer = static_cast<char*>(pool->v_base) + off;
+    prm.kv_heads = pool->kv_heads;
+    prm.head_dim = pool->head_dim;
+    prm.page_size = pool->page_size;
+    prm.num_slots = (int64_t)pool->num_pages * pool->page_size;
+    return prm;
+}
+
+bool misaligned16(const void* a, const void* b = nullptr, const void* c = nullptr)
+{
+    return ((reinterpret_cast<uintptr_t>(a) | reinterpret_cast<uintptr_t>(b) | reinterpret_cast<uintptr_t>(c)) & 15u) != 0;
+}
+
+}  // namespace
+}  // namespace pkv
+
 extern "C" int rope_apply(void* q, void* k, const int32_t* positions, int n_tokens, int q_heads, int kv_heads,
                           int head_dim, double theta, int dtype, pkv_stream_t stream)
 {
@@ -157,16 +197,18 @@ extern "C" int rope_apply(void* q, void* k, const int32_t* positions, int n_toke
     if (head_dim != 64 && head_dim != 128) return PKV_ERR_UNSUPPORTED;
     if (dtype != PKV_F16 && dtype != PKV_BF16) return PKV_ERR_UNSUPPORTED;
     if (n_tokens == 0 || q_heads + kv_heads == 0) return PKV_OK;
-    if (!positions) return PKV_ERR_INVALID_ARG;
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    cudaError_t e;
-    if (dtype == PKV_F16)
-        e = launch_pdl(rope_kernel<__half>, dim3(n_tokens), dim3(256), 0, st, static_cast<__half*>(q),
-                       static_cast<__half*>(k), positions, q_heads, kv_heads, head_dim, theta);
-    else
-        e = launch_pdl(rope_kernel<__nv_bfloat16>, dim3(n_tokens), dim3(256), 0, st, static_cast<__nv_bfloat16*>(q),
-                       static_cast<__nv_bfloat16*>(k), positions, q_heads, kv_heads, head_dim, theta);
-    return status_of(e);
+    if (!positions || misaligned16(q, k)) return PKV_ERR_INVALID_ARG;
+    RopeAppendParams prm;
+    std::memset(&prm, 0, sizeof(prm));
+    prm.q = q;
+    prm.k = k;
+    prm.positions = positions;
+    prm.q_heads = q_heads;
+    prm.kv_heads = kv_heads;
+    prm.head_dim = head_dim;
+    prm.theta = theta;
+    prm.mode = kRopeRotate;
+    return launch_rope_append(prm, n_tokens, dtype, reinterpret_cast<cudaStream_t>(stream));
 }
 
 extern "C" int paged_kv_append(const pkv_pool* pool, int layer, const void* k, const void* v,
@@ -175,15 +217,34 @@ extern "C" int paged_kv_append(const pkv_pool* pool, int layer, const void* k, c
     if (!pool || layer < 0 || layer >= pool->num_layers || n_tokens < 0) return PKV_ERR_INVALID_ARG;
     if (n_tokens == 0) return PKV_OK;
     if (!k || !v || !slot_mapping) return PKV_ERR_INVALID_ARG;
-    if ((reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v)) & 15u) return PKV_ERR_INVALID_ARG;
-    const size_t elt = 2;
-    uint4* kl = reinterpret_cast<uint4*>(static_cast<char*>(pool->k_base) + (size_t)layer * pool->layer_elems * elt);
-    uint4* vl = reinterpret_cast<uint4*>(static_cast<char*>(pool->v_base) + (size_t)layer * pool->layer_elems * elt);
-    const int64_t num_slots = (int64_t)pool->num_pages * pool->page_size;
-    cudaError_t e = launch_pdl(append_kernel, dim3(n_tokens), dim3(128), 0, reinterpret_cast<cudaStream_t>(stream), kl,
-                               vl, static_cast<const uint4*>(k), static_cast<const uint4*>(v), slot_mapping,
-                               pool->kv_heads, pool->head_dim, pool->page_size, num_slots);
-    return status_of(e);
+    if (misaligned16(k, v)) return PKV_ERR_INVALID_ARG;
+    RopeAppendParams prm = pool_params(pool, layer);
+    prm.k = const_cast<void*>(k);    // read only: no rotation in this mode
+    prm.v = v;
+    prm.slots = slot_mapping;
+    prm.mode = kRopeAppend;
+    return launch_rope_append(prm, n_tokens, pool->dtype, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int rope_append(const pkv_pool* pool, int layer, void* q, void* k, const void* v,
+                           const int32_t* positions, const int64_t* slot_mapping, int n_tokens, int q_heads,
+                           double theta, pkv_stream_t stream)
+{
+    if (!pool || layer < 0 || layer >= pool->num_layers || n_tokens < 0 || q_heads < 0 || !(theta > 0.0))
+        return PKV_ERR_INVALID_ARG;
+    if (n_tokens == 0) return PKV_OK;
+    if (!k || !v || !positions || !slot_mapping || (q_heads > 0 && !q)) return PKV_ERR_INVALID_ARG;
+    if (misaligned16(q, k, v)) return PKV_ERR_INVALID_ARG;
+    RopeAppendParams prm = pool_params(pool, layer);
+    prm.q = q;
+    prm.k = k;
+    prm.v = v;
+    prm.positions = positions;
+    prm.slots = slot_mapping;
+    prm.q_heads = q_heads;
+    prm.theta = theta;
+    prm.mode = kRopeRotate | kRopeAppend;
+    return launch_rope_append(prm, n_tokens, pool->dtype, reinterpret_cast<cudaStream_t>(stream));
 }
 
 extern "C" int pkv_decode_default_splits(int q_heads, int kv_heads, int head_dim, int page_size, int dtype,

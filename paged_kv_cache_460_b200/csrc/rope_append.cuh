@@ -1,9 +1,9 @@
-// RoPE and KV-append kernels of the decode step.
+// RoPE and KV append of the decode step's new token, one kernel for both.
 //
 // "为什么要自己动手写一个LLM推理引擎" (wzjinhao.cn/news/61427):
 //   s4.2  RoPE writes the position into q and k with a rotation;
 //   s4.3  apply_rotary_emb(q, k, start_pos), then the new k, v join the cache;
-//   s5.3  the cache is a preallocated pool (no concatenation).
+//   s5.3  the cache is a preallocated pool (no concatenation); fuse small kernels.
 #ifndef PKV_ROPE_APPEND_CUH_
 #define PKV_ROPE_APPEND_CUH_
 
@@ -11,84 +11,104 @@
 
 namespace pkv {
 
-// One CTA per token.  The head_dim/2 angles pos * theta^(-2i/d) and their cosines and
-// sines are evaluated once per token in fp64 and shared through shared memory; every
-// (head, pair) of q and k is then rotated in fp64 and rounded once to the storage type.
-// Products and differences use explicit _rn intrinsics, so no fused multiply-add changes
-// the rounding of the rotation.
+constexpr int kRopeRotate = 1;   // turn q and k in place
+constexpr int kRopeAppend = 2;   // write k and v into their pool slots
+
+struct RopeAppendParams {
+    void* q;                 // [n][q_heads][d]   (rotated in place)
+    void* k;                 // [n][kv_heads][d]  (rotated in place)
+    const void* v;           // [n][kv_heads][d]
+    const int32_t* positions;
+    const int64_t* slots;
+    void* k_layer;           // this layer's K pool [pages][kv_heads][P][d]
+    void* v_layer;
+    int q_heads;
+    int kv_heads;
+    int head_dim;
+    int page_size;
+    int64_t num_slots;
+    double theta;
+    int mode;
+};
+
+// Grid: (token, part).  Each thread handles one 16-byte vector (8 elements, 4 pairs)
+// of the token's q, k or v rows.  The head_dim/2 angles pos * theta^(-2i/d) and their
+// cosines and sines are evaluated once per CTA in fp64 before griddepcontrol.wait, so
+// this prologue overlaps the previous kernel on the stream; each pair is then turned in
+// fp64 (explicit _rn products: no fused rounding) and rounded once to the storage type.
+// Appending copies the rotated k and the v vector bit for bit into row slot % P of page
+// slot / P; a negative slot skips the token, a slot past the pool is skipped and flagged.
 template <typename T>
-__global__ void __launch_bounds__(256) rope_kernel(T* __restrict__ q, T* __restrict__ k,
-                                                   const int32_t* __restrict__ positions, int q_heads,
-                                                   int kv_heads, int head_dim, double theta)
+__global__ void __launch_bounds__(256) rope_append_kernel(const RopeAppendParams p)
 {
     __shared__ double cs[64][2];
-    pdl_wait();
-    pdl_launch_dependents();
     const int t = blockIdx.x;
-    const int pos = positions[t];
-    if (pos < 0) return;
-    const int half = head_dim >> 1;
-    for (int i = threadIdx.x; i < half; i += blockDim.x) {
-        const double freq = pow(theta, -2.0 * (double)i / (double)head_dim);
-        double s, c;
-        sincos((double)pos * freq, &s, &c);
-        cs[i][0] = c;
-        cs[i][1] = s;
+    const int pos = (p.mode & kRopeRotate) ? p.positions[t] : -1;
+    const int half = p.head_dim >> 1;
+    if (pos >= 0) {
+        for (int i = threadIdx.x; i < half; i += blockDim.x) {
+            const double freq = pow(p.theta, -2.0 * (double)i / (double)p.head_dim);
+            double sn, cn;
+            sincos((double)pos * freq, &sn, &cn);
+            cs[i][0] = cn;
+            cs[i][1] = sn;
+        }
     }
     __syncthreads();
-    const int nq = q_heads * half;
-    const int total = (q_heads + kv_heads) * half;
-    for (int idx = threadIdx.x; idx < total; idx += blockDim.x) {
-        T* x;
-        int i;
-        if (idx < nq) {
-            const int h = idx / half;
-            i = idx - h * half;
-            x = q + ((size_t)t * q_heads + h) * head_dim + 2 * i;
-        } else {
-            const int rel = idx - nq;
-            const int h = rel / half;
-            i = rel - h * half;
-            x = k + ((size_t)t * kv_heads + h) * head_dim + 2 * i;
-        }
-        const double x0 = Elt<T>::to_double(x[0]);
-        const double x1 = Elt<T>::to_double(x[1]);
-        const double c = cs[i][0], s = cs[i][1];
-        const double y0 = __dsub_rn(__dmul_rn(x0, c), __dmul_rn(x1, s));
-        const double y1 = __dadd_rn(__dmul_rn(x0, s), __dmul_rn(x1, c));
-        x[0] = Elt<T>::from_double(y0);
-        x[1] = Elt<T>::from_double(y1);
-    }
-}
-
-// One CTA per token: copy the token's k and v rows (kv_heads x head_dim elements each,
-// 16-byte vectors) into row slot % page_size of page slot / page_size.  A negative
-// slot skips the token; a slot past the pool is skipped and flagged.
-__global__ void __launch_bounds__(128) append_kernel(uint4* __restrict__ k_layer, uint4* __restrict__ v_layer,
-                                                     const uint4* __restrict__ k, const uint4* __restrict__ v,
-                                                     const int64_t* __restrict__ slots, int kv_heads,
-                                                     int head_dim, int page_size, int64_t num_slots)
-{
     pdl_wait();
     pdl_launch_dependents();
-    const int t = blockIdx.x;
-    const int64_t s = slots[t];
-    if (s < 0) return;
-    if (s >= num_slots) {
-        if (threadIdx.x == 0) atomicOr(&g_error_word, PKV_DEVERR_BAD_SLOT);
-        return;
+    int64_t slot = -1;
+    if (p.mode & kRopeAppend) {
+        slot = p.slots[t];
+        if (slot >= p.num_slots) {
+            if (blockIdx.y == 0 && threadIdx.x == 0) atomicOr(&g_error_word, PKV_DEVERR_BAD_SLOT);
+            slot = -1;
+        }
     }
-    const int64_t page = s / page_size;
-    const int row = (int)(s - page * page_size);
-    const int vec_per_row = head_dim / 8;          // 8 two-byte elements per 16 bytes
-    const int total = kv_heads * vec_per_row;
-    for (int idx = threadIdx.x; idx < total; idx += blockDim.x) {
-        const int h = idx / vec_per_row;
-        const int c = idx - h * vec_per_row;
-        const int64_t dst = ((page * kv_heads + h) * page_size + row) * vec_per_row + c;
-        const int64_t src = ((int64_t)t * kv_heads + h) * vec_per_row + c;
-        k_layer[dst] = k[src];
-        v_layer[dst] = v[src];
+    const int vph = p.head_dim / 8;                      // 16-byte vectors per head row
+    const int nq = (p.mode & kRopeRotate) ? p.q_heads * vph : 0;
+    const int nk = p.kv_heads * vph;
+    const int total = nq + ((p.mode & kRopeAppend) ? 2 * nk : nk);
+    const int64_t page = slot >= 0 ? slot / p.page_size : 0;
+    const int row = slot >= 0 ? (int)(slot - page * p.page_size) : 0;
+    for (int idx = blockIdx.y * blockDim.x + threadIdx.x; idx < total; idx += gridDim.y * blockDim.x) {
+        uint4* src;
+        int h, c;
+        bool is_v = false;
+        if (idx < nq) {
+            h = idx / vph;
+            c = idx - h * vph;
+            src = reinterpret_cast<uint4*>(static_cast<T*>(p.q) + ((int64_t)t * p.q_heads + h) * p.head_dim) + c;
+        } else if (idx < nq + nk) {
+            h = (idx - nq) / vph;
+            c = (idx - nq) - h * vph;
+            src = reinterpret_cast<uint4*>(static_cast<T*>(p.k) + ((int64_t)t * p.kv_heads + h) * p.head_dim) + c;
+        } else {
+            h = (idx - nq - nk) / vph;
+            c = (idx - nq - nk) - h * vph;
+            src = const_cast<uint4*>(reinterpret_cast<const uint4*>(static_cast<const T*>(p.v) +
+                                                                    ((int64_t)t * p.kv_heads + h) * p.head_dim)) + c;
+            is_v = true;
+        }
+        uint4 u = *src;
+        if (!is_v && pos >= 0) {
+            T* e = reinterpret_cast<T*>(&u);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int i = c * 4 + k;                    // pair index within the head
+                const double x0 = Elt<T>::to_double(e[2 * k]);
+                const double x1 = Elt<T>::to_double(e[2 * k + 1]);
+                const double cn = cs[i][0], sn = cs[i][1];
+                e[2 * k] = Elt<T>::from_double(__dsub_rn(__dmul_rn(x0, cn), __dmul_rn(x1, sn)));
+                e[2 * k + 1] = Elt<T>::from_double(__dadd_rn(__dmul_rn(x0, sn), __dmul_rn(x1, cn)));
+            }
+            *src = u;
+        }
+        if (slot >= 0 && idx >= nq) {
+            uint4* dst = static_cast<uint4*>(is_v ? p.v_layer : p.k_layer) +
+                         ((page * p.kv_heads + h) * p.page_size + row) * vph + c;
+            *dst = u;
+        }
     }
 }
 

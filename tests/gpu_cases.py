@@ -56,13 +56,17 @@ class Case:
         self.slots_t = torch.from_numpy(self.slots).cuda()
         self.scale = 1.0 / math.sqrt(s.head_dim)
 
-    def gpu_layer(self, layer, num_splits=0, workspace=None):
+    def gpu_layer(self, layer, num_splits=0, workspace=None, fused=False):
         s = self.s
         q_t = to_dev(self.q[layer], s.dtype)
         k_t = to_dev(self.k[layer], s.dtype)
         v_t = to_dev(self.v[layer], s.dtype)
-        pkv.rope_apply(q_t, k_t, self.pos_t, s.theta)
-        pkv.paged_kv_append(self.pool, layer, k_t, v_t, self.slots_t)
+        if fused:
+            pkv.rope_append(self.pool, layer, q_t, k_t, v_t, self.pos_t, self.slots_t, s.theta)
+        else:
+            pkv.rope_apply(q_t, k_t, self.pos_t, s.theta)
+            pkv.paged_kv_append(self.pool, layer, k_t, v_t, self.slots_t)
+        self.last_q = q_t
         out = torch.empty_like(q_t)
         pkv.paged_decode_attention(self.pool, layer, out, q_t, self.bt_t, self.cl_t, self.scale,
                                    num_splits=num_splits, workspace=workspace)

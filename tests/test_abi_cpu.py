@@ -194,3 +194,14 @@ def test_workspace_size_and_host_validation(L):
     assert L.rope_apply(None, f(), f(), 1, 2, 2, 64, 10000.0, 0, None) == _lib.PKV_ERR_INVALID_ARG
     assert L.rope_apply(f(), f(), f(), 0, 2, 2, 64, 10000.0, 0, None) == 0
     L.kv_pool_destroy(h)
+
+
+def test_rope_append_validates(L):
+    h = _pool(L, num_pages=8, page_size=16, kv_heads=2, head_dim=64)
+    f = _fake_ptr
+    assert L.rope_append(h, 1, f(), f(), f(), f(), f(), 1, 2, 10000.0, None) == _lib.PKV_ERR_INVALID_ARG
+    assert L.rope_append(h, 0, f(), f(), f(), None, f(), 1, 2, 10000.0, None) == _lib.PKV_ERR_INVALID_ARG
+    assert L.rope_append(h, 0, f(0x10004), f(), f(), f(), f(), 1, 2, 10000.0, None) == _lib.PKV_ERR_INVALID_ARG
+    assert L.rope_append(h, 0, f(), f(), f(), f(), f(), 1, 2, 0.0, None) == _lib.PKV_ERR_INVALID_ARG
+    assert L.rope_append(h, 0, f(), f(), f(), f(), f(), 0, 2, 10000.0, None) == 0
+    L.kv_pool_destroy(h)

@@ -85,6 +85,21 @@ def test_append_out_of_range_slot_is_skipped_and_flagged():
     assert (got[0, 0, :, 3] == 0x3C00).all() and got.sum() == 2 * d * 0x3C00
 
 
+@pytest.mark.parametrize("d,P,Hq,Hkv,dtype", [(128, 16, 8, 8, "f16"), (128, 32, 8, 2, "bf16"), (64, 16, 4, 1, "f16")])
+def test_fused_rope_append_equals_separate_calls(d, P, Hq, Hkv, dtype):
+    cached = [0, 5, P - 1, P, 3 * P + 2, -1, 100]
+    s = synth.random_spec(250 + d + P, len(cached), Hq, Hkv, d, P, cached, dtype=dtype)
+    a, b = Case(s), Case(s)
+    out_a = to_bits(a.gpu_layer(0))
+    out_b = to_bits(b.gpu_layer(0, fused=True))
+    assert np.array_equal(to_bits(a.kp_t), to_bits(b.kp_t))
+    assert np.array_equal(to_bits(a.vp_t), to_bits(b.vp_t))
+    assert np.array_equal(to_bits(a.last_q), to_bits(b.last_q))
+    assert np.array_equal(out_a, out_b)
+    _expect_close(out_b, b.oracle_layer(0), dtype, "fused step")
+    assert pkv.kv_get_device_error() == 0
+
+
 # ------------------------------------------------------------------ whole step, small workloads
 @pytest.mark.parametrize("name", ["tiny", "layer7b"])
 def test_step_matches_oracle_on_workload(name):
@@ -196,7 +211,7 @@ def test_full_size_workload_sampled(name, layers, check_layers):
     ws = pkv.DecodeWorkspace(s.batch, s.q_heads, s.kv_heads, s.head_dim, s.page_size, TDT[s.dtype])
     outs = {}
     for L in range(layers):                      # the step as the benchmark runs it
-        out = c.gpu_layer(L, workspace=ws)
+        out = c.gpu_layer(L, workspace=ws, fused=True)
         if L in snaps:
             outs[L] = to_bits(out)
     for L, sn in snaps.items():
