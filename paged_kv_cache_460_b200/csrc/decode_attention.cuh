@@ -39,7 +39,9 @@ namespace pkv {
 
 constexpr int kDecodeWarps = 4;
 constexpr int kDecodeThreads = kDecodeWarps * 32;
-constexpr int kRingBudgetBytes = 68 * 1024;    // three CTAs per SM at page 16, head_dim 128
+// Two ring slots per warp at page 16 / head_dim 128.  Deeper rings (3-5 slots) and a
+// third CTA per SM were measured slower on the 10-request, 32-layer decode workload.
+constexpr int kRingBudgetBytes = 68 * 1024;
 constexpr int kMetaHeaderBytes = 16;   // int64 chunk, int64 total units
 
 struct DecodeParams {
@@ -73,7 +75,8 @@ struct DecodeShape {
     static constexpr int kRingBytes = kDecodeWarps * kDepth * kSlot;
     static constexpr int kCmbOffset = kRingBytes;
     static constexpr int kCmbFloats = kDecodeWarps * G * (D + 2);
-    static constexpr int kWarpTotOffset = kCmbOffset + 2 * kCmbFloats * 4;
+    static constexpr int kPbufOffset = kCmbOffset + 2 * kCmbFloats * 4;     // [warps][G][P] floats
+    static constexpr int kWarpTotOffset = kPbufOffset + kDecodeWarps * G * P * 4;
     static constexpr int kScanOffset = kWarpTotOffset + 64;
     // prefix[batch+1] and lens[batch] follow
     static int smem_bytes(int batch) { return kScanOffset + 4 * (2 * batch + 1); }
@@ -147,13 +150,17 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_pass1_kernel(const Deco
     using S = DecodeShape<D, P, G>;
     constexpr int NW = kDecodeWarps;
     constexpr int DEPTH = S::kDepth;
-    constexpr int LPR = D / 8;            // lanes per K/V row (16 bytes each)
-    constexpr int RPI = 32 / LPR;         // rows covered by one warp-wide 16-byte access
-    constexpr int NIT = P / RPI;          // accesses per page chunk
+    constexpr int CPR = D / 8;            // 16-byte chunks per K/V row
+    constexpr int LPRK = 2;               // lanes sharing one K row in q.k
+    constexpr int RPL = P / 16;           // K rows per lane per page (rows t and t + 16)
+    constexpr int CPL = CPR / LPRK;       // K chunks per lane per row
+    constexpr int EPL = D / 32;           // output columns owned by each lane in p.V
     constexpr int QV = S::kQBytes / 16;   // 16-byte pieces of the group's q rows
-    static_assert(NIT <= LPR, "a page's rows must fit the transposed reduction");
+    static_assert(P == 16 || P == 32, "page size");
+    static_assert(EPL == 2 || EPL == 4, "head_dim");
     extern __shared__ __align__(128) unsigned char smem[];
     float* cmb = reinterpret_cast<float*>(smem + S::kCmbOffset);
+    float* pbuf_all = reinterpret_cast<float*>(smem + S::kPbufOffset);
     int* warp_tot = reinterpret_cast<int*>(smem + S::kWarpTotOffset);
     int* prefix = reinterpret_cast<int*>(smem + S::kScanOffset);
     int* lens = prefix + p.batch + 1;
@@ -198,8 +205,12 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_pass1_kernel(const Deco
     if (r0 >= r1) return;
 
     unsigned char* ring = smem + warp * DEPTH * S::kSlot;
+    float* pbuf = pbuf_all + warp * G * P;
 
-    // ---- issue side: this warp's page k (iterator at unit r0 + warp + k NW)
+    // ---- issue side: this warp's page k (iterator at unit r0 + warp + k NW).
+    // K rows land XOR-swizzled by 16-byte chunk -- chunk c of row t at position
+    // c ^ ((2 t + c / CPL) & 7) -- so that the lanes reading different rows at the same
+    // column hit different banks; V rows land as they are.
     int ib = 0, ig = 0, ij = 0, inp = 1, qb = -1, qg = -1;
     if (n_mine > 0) {
         locate_unit(r0 + warp, prefix, p.batch, Hkv, ib, ig, ij);
@@ -218,8 +229,11 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_pass1_kernel(const Deco
             const unsigned char* vs = reinterpret_cast<const unsigned char*>(static_cast<const T*>(p.v) + off);
 #pragma unroll
             for (int n = 0; n < S::kChunk / 512; ++n) {
-                cp_async16(slot + n * 512 + lane * 16, ks + n * 512 + lane * 16);
-                cp_async16(slot + S::kChunk + n * 512 + lane * 16, vs + n * 512 + lane * 16);
+                const int gidx = n * 32 + lane;               // 16-byte chunk of the page
+                const int t = gidx / CPR, c = gidx % CPR;
+                const int pos = c ^ ((t * LPRK + c / CPL) & 7);
+                cp_async16(slot + t * (2 * D) + pos * 16, ks + gidx * 16);
+                cp_async16(slot + S::kChunk + gidx * 16, vs + gidx * 16);
             }
         } else if (lane == 0) {
             atomicOr(&g_error_word, PKV_DEVERR_BAD_PAGE);   // never dereferenced
@@ -243,200 +257,193 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_pass1_kernel(const Deco
         cp_async_commit();
     }
 
-    // ---- compute side
-    const int r = lane / LPR, c = lane % LPR;
-    // After the transposed reduction lane holds the score of row i_own * RPI + r.
-    int i_own = 0;
-#pragma unroll
-    for (int m = LPR / 2, w8 = NIT / 2; w8 >= 1; m >>= 1, w8 >>= 1)
-        if (lane & m) i_own += w8;
-    const int tok_own = i_own * RPI + r;
-    // Lanes below the last halving mask hold duplicates; only the lowest counts in l.
-    const bool primary = (lane & (LPR / NIT - 1)) == 0;
-    float qf[G][8], o[G][8], m_run[G], l_run[G];
+    // ---- compute side.  q.k: lane (t, h) = (lane / 2, lane % 2) dots rows t (and t + 16
+    // at P = 32) over chunks h*CPL .. h*CPL+CPL-1; p.V: lane owns output columns
+    // lane*EPL .. lane*EPL+EPL-1.
+    const int t_own = lane / LPRK, h_own = lane % LPRK;
+    const int sw_own = (t_own * LPRK + h_own) & 7;
+    uint4 qraw[G][CPL];
+    float o[G][EPL], m_run[G], l_run[G];
 #pragma unroll
     for (int gi = 0; gi < G; ++gi) {
         m_run[gi] = -INFINITY;
         l_run[gi] = 0.f;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) o[gi][e] = 0.f;
+        for (int e = 0; e < EPL; ++e) o[gi][e] = 0.f;
     }
+    long long kc = 0;                         // this warp's pages consumed
     int b, g, j;
     locate_unit(r0, prefix, p.batch, Hkv, b, g, j);
     int np = prefix[b + 1] - prefix[b];
-    int seg = 0, cb = -1, cg = -1;
-    long long kc = 0;                         // this warp's pages consumed
-    int it = 0;
-    for (long long u = r0; u < r1; ++u, ++it) {
-        if (it % NW == warp) {
+    int seg = 0;
+    // One pass per segment (the range's part of one (sequence, kv head)): this warp's
+    // pages of it, then the combine of all warps.
+    for (long long u = r0; u < r1; ++seg) {
+        const long long u_end = min(r1, u + (np - j));
+        const long long first = u + ((warp - (int)((u - r0) % NW)) + NW) % NW;
+        bool have_q = false;
+        for (long long uu = first; uu < u_end; uu += NW) {
             cp_async_wait<DEPTH - 1>();         // page kc has landed (this lane's copies)
-            __syncwarp();                       // ... and every lane's (q is read across lanes)
+            __syncwarp();                       // ... and every lane's
             const unsigned char* s = ring + (int)(kc % DEPTH) * S::kSlot;
-            if (b != cb || g != cg) {           // first page of this segment for this warp
-                cb = b;
-                cg = g;
+            if (!have_q) {                      // first page of this segment for this warp
+                have_q = true;
 #pragma unroll
-                for (int gi = 0; gi < G; ++gi) {
-                    const uint4 qu = *reinterpret_cast<const uint4*>(s + 2 * S::kChunk + (gi * D + c * 8) * 2);
-                    unpack8<T>(qu, qf[gi]);
-                }
+                for (int gi = 0; gi < G; ++gi)
+#pragma unroll
+                    for (int i = 0; i < CPL; ++i)
+                        qraw[gi][i] = *reinterpret_cast<const uint4*>(s + 2 * S::kChunk + gi * (2 * D) +
+                                                                      (h_own * CPL + i) * 16);
             }
-            const int nvalid = min(P, lens[b] - j * P);
-            // ---- scores: partial dots over this lane's 8 columns, then a transposed
-            //      reduction that leaves one finished row score per lane
-            float sc[G];
-            {
-                float v[G][NIT];
+            const int nvalid = min(P, lens[b] - (j + (int)(uu - u)) * P);
+            // ---- scores: lane's partial dots over its chunks of rows t_own (+ 16)
+            float sc[G][RPL];
 #pragma unroll
-                for (int i = 0; i < NIT; ++i) {
-                    const uint4 ku = *reinterpret_cast<const uint4*>(s + i * 512 + lane * 16);
-                    float kf[8];
-                    unpack8<T>(ku, kf);
+            for (int rr = 0; rr < RPL; ++rr) {
+                float acc[G];
 #pragma unroll
-                    for (int gi = 0; gi < G; ++gi) {
-                        float2 a = make_float2(qf[gi][0] * kf[0], qf[gi][1] * kf[1]);
+                for (int gi = 0; gi < G; ++gi) acc[gi] = 0.f;
+                const int t = t_own + 16 * rr;
 #pragma unroll
-                        for (int e = 2; e < 8; e += 2)
-                            a = __ffma2_rn(make_float2(qf[gi][e], qf[gi][e + 1]), make_float2(kf[e], kf[e + 1]), a);
-                        v[gi][i] = a.x + a.y;
-                    }
+                for (int i = 0; i < CPL; ++i) {
+                    const int pos = (h_own * CPL + i) ^ sw_own;
+                    const uint4 ku = *reinterpret_cast<const uint4*>(s + t * (2 * D) + pos * 16);
+#pragma unroll
+                    for (int gi = 0; gi < G; ++gi) acc[gi] += dot8<T>(qraw[gi][i], ku);
                 }
 #pragma unroll
                 for (int gi = 0; gi < G; ++gi) {
-#pragma unroll
-                    for (int n = NIT, m = LPR / 2; n > 1; n >>= 1, m >>= 1) {
-                        const bool up = (lane & m) != 0;
-#pragma unroll
-                        for (int k = 0; k < n / 2; ++k) {
-                            const float send = up ? v[gi][k] : v[gi][k + n / 2];
-                            const float keep = up ? v[gi][k + n / 2] : v[gi][k];
-                            v[gi][k] = keep + __shfl_xor_sync(0xffffffffu, send, m);
-                        }
-                    }
-#pragma unroll
-                    for (int m = LPR / (2 * NIT); m >= 1; m >>= 1)
-                        v[gi][0] += __shfl_xor_sync(0xffffffffu, v[gi][0], m);
-                    sc[gi] = tok_own < nvalid ? v[gi][0] * p.scale_log2 : -INFINITY;
+                    acc[gi] += __shfl_xor_sync(0xffffffffu, acc[gi], 1);
+                    sc[gi][rr] = t < nvalid ? acc[gi] * p.scale_log2 : -INFINITY;
                 }
             }
-            // ---- online softmax update (per query head of the group)
-            float pr[G], alpha[G];
+            // ---- online softmax update; p of every row published to the warp's buffer
+            float alpha[G];
             bool rescale = false;
 #pragma unroll
             for (int gi = 0; gi < G; ++gi) {
-                float pm = sc[gi];
+                float pm = sc[gi][0];
 #pragma unroll
-                for (int m = 16; m >= LPR / NIT; m >>= 1) pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, m));
+                for (int rr = 1; rr < RPL; ++rr) pm = fmaxf(pm, sc[gi][rr]);
+#pragma unroll
+                for (int m = 16; m >= 2; m >>= 1) pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, m));
                 const float mn = fmaxf(m_run[gi], pm);   // finite: row 0 of a page is always valid
                 alpha[gi] = fast_exp2(m_run[gi] - mn);
                 rescale |= m_run[gi] != mn;
                 m_run[gi] = mn;
-                pr[gi] = fast_exp2(sc[gi] - mn);           // 0 for rows past the context
-                l_run[gi] = l_run[gi] * alpha[gi] + (primary ? pr[gi] : 0.f);
+                float ls = 0.f;
+#pragma unroll
+                for (int rr = 0; rr < RPL; ++rr) {
+                    const float pr = fast_exp2(sc[gi][rr] - mn);   // 0 for rows past the context
+                    ls += pr;
+                    if (h_own == 0) pbuf[gi * P + t_own + 16 * rr] = pr;
+                }
+                l_run[gi] = l_run[gi] * alpha[gi] + (h_own == 0 ? ls : 0.f);
             }
             if (rescale) {
 #pragma unroll
                 for (int gi = 0; gi < G; ++gi)
 #pragma unroll
-                    for (int e = 0; e < 8; e += 2) {
-                        const float2 t = __fmul2_rn(make_float2(o[gi][e], o[gi][e + 1]), make_float2(alpha[gi], alpha[gi]));
-                        o[gi][e] = t.x;
-                        o[gi][e + 1] = t.y;
+                    for (int e = 0; e < EPL; e += 2) {
+                        const float2 t2 = __fmul2_rn(make_float2(o[gi][e], o[gi][e + 1]), make_float2(alpha[gi], alpha[gi]));
+                        o[gi][e] = t2.x;
+                        o[gi][e + 1] = t2.y;
                     }
             }
-            // ---- o += p V over the page's rows
-#pragma unroll
-            for (int i = 0; i < NIT; ++i) {
-                const int row = i * RPI + r;
-                const uint4 vu = *reinterpret_cast<const uint4*>(s + S::kChunk + i * 512 + lane * 16);
-                float vf[8];
-                unpack8<T>(vu, vf);
-                if (nvalid < P && row >= nvalid) {             // only the last page of a sequence
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) vf[e] = 0.f;   // rows past the context may hold anything
+            __syncwarp();                         // p of all rows visible to the warp
+            // ---- o += p V: row t's EPL columns of this lane (rows past the context skipped)
+            const unsigned char* vbase = s + S::kChunk + lane * (EPL * 2);
+            auto pv_row = [&](int t) {
+                float vf[EPL];
+                if constexpr (EPL == 4) {
+                    const uint2 w = *reinterpret_cast<const uint2*>(vbase + t * (2 * D));
+                    const float2 a = Elt<T>::to_float2(w.x), c2 = Elt<T>::to_float2(w.y);
+                    vf[0] = a.x; vf[1] = a.y; vf[2] = c2.x; vf[3] = c2.y;
+                } else {
+                    const uint32_t w = *reinterpret_cast<const uint32_t*>(vbase + t * (2 * D));
+                    const float2 a = Elt<T>::to_float2(w);
+                    vf[0] = a.x; vf[1] = a.y;
                 }
-                int src = r * LPR;                              // the lane holding row i's score
-#pragma unroll
-                for (int m = LPR / 2, w8 = NIT / 2; w8 >= 1; m >>= 1, w8 >>= 1)
-                    if (i & w8) src += m;
 #pragma unroll
                 for (int gi = 0; gi < G; ++gi) {
-                    const float pi = __shfl_sync(0xffffffffu, pr[gi], src);
+                    const float pt = pbuf[gi * P + t];
 #pragma unroll
-                    for (int e = 0; e < 8; e += 2) {
-                        const float2 acc = __ffma2_rn(make_float2(pi, pi), make_float2(vf[e], vf[e + 1]),
-                                                      make_float2(o[gi][e], o[gi][e + 1]));
-                        o[gi][e] = acc.x;
-                        o[gi][e + 1] = acc.y;
+                    for (int e = 0; e < EPL; e += 2) {
+                        const float2 r2 = __ffma2_rn(make_float2(pt, pt), make_float2(vf[e], vf[e + 1]),
+                                                     make_float2(o[gi][e], o[gi][e + 1]));
+                        o[gi][e] = r2.x;
+                        o[gi][e + 1] = r2.y;
                     }
                 }
+            };
+            if (nvalid == P) {
+#pragma unroll
+                for (int t = 0; t < P; ++t) pv_row(t);
+            } else {
+                for (int t = 0; t < nvalid; ++t) pv_row(t);   // last page of a sequence
             }
-            __syncwarp();                         // every lane is done with the slot
+            __syncwarp();                         // every lane is done with the slot and p
             if (kc + DEPTH < n_mine) issue(kc + DEPTH);
             cp_async_commit();
             ++kc;
         }
-        const bool seg_end = (j == np - 1) || (u == r1 - 1);
-        if (seg_end) {
-            // every warp publishes its (possibly empty) state of this segment
-            float* buf = cmb + (seg & 1) * S::kCmbFloats;
+        // ---- every warp publishes its (possibly empty) state of this segment
+        float* buf = cmb + (seg & 1) * S::kCmbFloats;
 #pragma unroll
-            for (int gi = 0; gi < G; ++gi) {
-                float lt = l_run[gi];
+        for (int gi = 0; gi < G; ++gi) {
+            float lt = l_run[gi];
 #pragma unroll
-                for (int m = 16; m >= 1; m >>= 1) lt += __shfl_xor_sync(0xffffffffu, lt, m);
+            for (int m = 16; m >= 1; m >>= 1) lt += __shfl_xor_sync(0xffffffffu, lt, m);
+            float* row = buf + (warp * G + gi) * (D + 2);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    float ot = o[gi][e];
-#pragma unroll
-                    for (int m = LPR; m < 32; m <<= 1) ot += __shfl_xor_sync(0xffffffffu, ot, m);
-                    o[gi][e] = ot;
-                }
-                float* row = buf + (warp * G + gi) * (D + 2);
-                if (r == 0) {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) row[c * 8 + e] = o[gi][e];
-                    if (c == 0) {
-                        row[D] = m_run[gi];
-                        row[D + 1] = lt;
-                    }
-                }
-                m_run[gi] = -INFINITY;
-                l_run[gi] = 0.f;
-#pragma unroll
-                for (int e = 0; e < 8; ++e) o[gi][e] = 0.f;
+            for (int e = 0; e < EPL; ++e) row[lane * EPL + e] = o[gi][e];
+            if (lane == 0) {
+                row[D] = m_run[gi];
+                row[D + 1] = lt;
             }
-            named_barrier(1, NW * 32);
-            const long long seg0 = (long long)Hkv * prefix[b] + (long long)g * np;
-            const bool complete = seg0 >= r0 && seg0 + np <= r1;
-            const int pslot = seg0 < r0 ? 2 * blockIdx.x : 2 * blockIdx.x + 1;
-            for (int idx = tid; idx < G * D; idx += NW * 32) {
-                const int gi = idx / D, dd = idx - gi * D;
-                float M = -INFINITY;
+            m_run[gi] = -INFINITY;
+            l_run[gi] = 0.f;
 #pragma unroll
-                for (int w = 0; w < NW; ++w) M = fmaxf(M, buf[(w * G + gi) * (D + 2) + D]);
-                float num = 0.f, den = 0.f;
-#pragma unroll
-                for (int w = 0; w < NW; ++w) {
-                    const float* row = buf + (w * G + gi) * (D + 2);
-                    const float wt = fast_exp2(row[D] - M);   // a warp with no page here has m = -inf
-                    num = fmaf(wt, row[dd], num);
-                    den = fmaf(wt, row[D + 1], den);
-                }
-                if (complete) {
-                    T* dst = static_cast<T*>(p.out) + ((long long)b * p.q_heads + (long long)g * G + gi) * D + dd;
-                    *dst = Elt<T>::from_float(num / den);
-                } else {
-                    p.part_o[((long long)pslot * G + gi) * D + dd] = num;
-                    if (dd == 0) {
-                        p.part_ml[((long long)pslot * G + gi) * 2 + 0] = M;
-                        p.part_ml[((long long)pslot * G + gi) * 2 + 1] = den;
-                    }
-                }
-            }
-            ++seg;
+            for (int e = 0; e < EPL; ++e) o[gi][e] = 0.f;
         }
-        next_unit(b, g, j, np, prefix, Hkv, p.batch);
+        named_barrier(1, NW * 32);
+        const long long seg0 = (long long)Hkv * prefix[b] + (long long)g * np;
+        const bool complete = seg0 >= r0 && seg0 + np <= r1;
+        const int pslot = seg0 < r0 ? 2 * blockIdx.x : 2 * blockIdx.x + 1;
+        for (int idx = tid; idx < G * D; idx += NW * 32) {
+            const int gi = idx / D, dd = idx - gi * D;
+            float M = -INFINITY;
+#pragma unroll
+            for (int w = 0; w < NW; ++w) M = fmaxf(M, buf[(w * G + gi) * (D + 2) + D]);
+            float num = 0.f, den = 0.f;
+#pragma unroll
+            for (int w = 0; w < NW; ++w) {
+                const float* row = buf + (w * G + gi) * (D + 2);
+                const float wt = fast_exp2(row[D] - M);   // a warp with no page here has m = -inf
+                num = fmaf(wt, row[dd], num);
+                den = fmaf(wt, row[D + 1], den);
+            }
+            if (complete) {
+                T* dst = static_cast<T*>(p.out) + ((long long)b * p.q_heads + (long long)g * G + gi) * D + dd;
+                *dst = Elt<T>::from_float(num / den);
+            } else {
+                p.part_o[((long long)pslot * G + gi) * D + dd] = num;
+                if (dd == 0) {
+                    p.part_ml[((long long)pslot * G + gi) * 2 + 0] = M;
+                    p.part_ml[((long long)pslot * G + gi) * 2 + 1] = den;
+                }
+            }
+        }
+        // next segment: the next kv head of this sequence, or the next non-empty sequence
+        u = u_end;
+        j = 0;
+        if (++g == Hkv) {
+            g = 0;
+            do {
+                ++b;
+                np = b < p.batch ? prefix[b + 1] - prefix[b] : 1;
+            } while (np == 0);
+        }
     }
     cp_async_wait<0>();
 }

@@ -80,7 +80,8 @@ struct DecodeImpl {
         return status_of(e);
     }
 
-    // SMs x resident CTAs per SM at the shared-memory size of a 64-row batch.
+    // SMs x resident CTAs per SM (at the shared-memory size of a 64-row batch), at most
+    // two per SM: a third CTA per SM measured slower on the 10-request decode workload.
     static int splits(int* out)
     {
         int dev = 0, sms = 0, per_sm = 0;
@@ -91,7 +92,7 @@ struct DecodeImpl {
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_pass1_kernel<D, P, G, T>, kDecodeThreads,
                                                           smem) != cudaSuccess)
             return PKV_ERR_CUDA;
-        *out = sms * (per_sm > 0 ? per_sm : 1);
+        *out = sms * (per_sm > 2 ? 2 : (per_sm > 0 ? per_sm : 1));
         return PKV_OK;
     }
 };

@@ -168,6 +168,28 @@ template <> struct Elt<__nv_bfloat16> {
     static __device__ __forceinline__ double to_double(__nv_bfloat16 x) { return (double)__bfloat162float(x); }
 };
 
+// Dot product of 8 storage elements with fp32 accumulation.  sm_100's mixed-precision
+// fma (16-bit multiplicands, fp32 addend and result) rounds exactly like widening both
+// operands to fp32 and calling fmaf, since the 16-bit product is exact in fp32.
+template <typename T> __device__ __forceinline__ float dot8(const uint4& q, const uint4& k);
+
+#define PKV_DOT8_ASM(TYPE)                                                                                     \
+    float a = 0.f, b = 0.f;                                                                                    \
+    asm("{ .reg .b16 q0,q1,q2,q3,q4,q5,q6,q7,k0,k1,k2,k3,k4,k5,k6,k7;\n\t"                                      \
+        "mov.b32 {q0,q1}, %2; mov.b32 {q2,q3}, %3; mov.b32 {q4,q5}, %4; mov.b32 {q6,q7}, %5;\n\t"                 \
+        "mov.b32 {k0,k1}, %6; mov.b32 {k2,k3}, %7; mov.b32 {k4,k5}, %8; mov.b32 {k6,k7}, %9;\n\t"                 \
+        "fma.rn.f32." TYPE " %0, q0, k0, %0; fma.rn.f32." TYPE " %1, q1, k1, %1;\n\t"                            \
+        "fma.rn.f32." TYPE " %0, q2, k2, %0; fma.rn.f32." TYPE " %1, q3, k3, %1;\n\t"                            \
+        "fma.rn.f32." TYPE " %0, q4, k4, %0; fma.rn.f32." TYPE " %1, q5, k5, %1;\n\t"                            \
+        "fma.rn.f32." TYPE " %0, q6, k6, %0; fma.rn.f32." TYPE " %1, q7, k7, %1; }"                                \
+        : "+f"(a), "+f"(b)                                                                                     \
+        : "r"(q.x), "r"(q.y), "r"(q.z), "r"(q.w), "r"(k.x), "r"(k.y), "r"(k.z), "r"(k.w));                    \
+    return a + b;
+
+template <> __device__ __forceinline__ float dot8<__half>(const uint4& q, const uint4& k) { PKV_DOT8_ASM("f16") }
+template <> __device__ __forceinline__ float dot8<__nv_bfloat16>(const uint4& q, const uint4& k) { PKV_DOT8_ASM("bf16") }
+#undef PKV_DOT8_ASM
+
 template <typename T>
 __device__ __forceinline__ void unpack8(const uint4& u, float (&f)[8])
 {
@@ -176,6 +198,8 @@ __device__ __forceinline__ void unpack8(const uint4& u, float (&f)[8])
     f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
     f[4] = c.x; f[5] = c.y; f[6] = d.x; f[7] = d.y;
 }
+
+
 
 }  // namespace pkv
 
