@@ -5,7 +5,7 @@
 
 A step is one pass of the whole hot path over one batch: for every layer, RoPE on
 the new token's q and k, the KV append through the slot mapping, and paged decode
-attention (streaming pass + merge).  The default workload is the batch-10,
+attention (one streaming kernel that also merges cut segments).  The default workload is the batch-10,
 32-layer, 32-head, head_dim-128, fp16 decode step with context lengths uniform in
 [128, 2048] and 16-token pages interleaved across the requests.
 
@@ -386,7 +386,7 @@ def run_ours(args):
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": profiled_traffic(args.workload),
                          "peak_source": "%s copy bandwidth" % peak_kind,
-                         "kernel": "paged_decode_attention (streaming pass + merge), per call",
+                         "kernel": "paged_decode_attention (one kernel per call)",
                          "frac_of_8tbs": achieved / NOMINAL_HBM_GBS},
             "cpu_baseline": cpu,
             "e2e": e2e,

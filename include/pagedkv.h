@@ -176,10 +176,10 @@ int pkv_decode_default_splits(int q_heads, int kv_heads, int head_dim, int page_
                               int* num_splits_out);
 
 /*
- * Workspace bytes paged_decode_attention needs for `num_splits` (>= 1) partitions and a
- * batch of `batch` rows: per partition two fp32 partial results (running max, sum and the
- * unnormalised output of every query head of a kv-head group) plus the batch's page
- * prefix sums.  0 on bad input.
+ * Workspace bytes paged_decode_attention needs for `num_splits` (>= 1) partitions: per
+ * partition two fp32 partial results (running max, sum and the unnormalised output of every
+ * query head of a kv-head group) and one int32 counter.  `batch` is accepted for
+ * compatibility and does not change the size.  0 on bad input.
  */
 size_t pkv_decode_workspace_size(int batch, int q_heads, int kv_heads, int head_dim,
                                  int num_splits);
@@ -201,11 +201,13 @@ size_t pkv_decode_workspace_size(int batch, int q_heads, int kv_heads, int head_
  *   {1, 2, 4, 8}.
  *   num_splits: number of work partitions (0 = pkv_decode_default_splits).  The batch's
  *           pages x kv heads are laid end to end and cut into num_splits equal ranges, one
- *           per CTA; a (sequence, kv head) cut by a range boundary is finished by a second
- *           merge kernel that rescales the partial softmax sums (log-sum-exp).
+ *           per CTA; a (sequence, kv head) cut by a range boundary is finished by the CTA
+ *           that delivers its last partial, which rescales the partial softmax sums
+ *           (log-sum-exp).  One kernel launch per call.
  *   workspace: device scratch of >= pkv_decode_workspace_size(batch, q_heads, kv_heads,
- *           head_dim, num_splits) bytes, 256-byte aligned; no initial contents needed;
- *           calls that share a workspace must be ordered on one stream.
+ *           head_dim, num_splits) bytes, 256-byte aligned, zero-filled before its first use
+ *           (pkv_decode_workspace_clear or any memset); every call leaves it ready for the
+ *           next one.  Calls that share a workspace must be ordered on one stream.
  * Errors: INVALID_ARG (bad pointer/shape/layer), UNSUPPORTED (group/head_dim/page/dtype
  * combination), NO_SPACE (workspace too small), CUDA (launch failure).
  */
@@ -225,21 +227,28 @@ int paged_decode_attention(const pkv_pool* pool, int layer, void* out, const voi
  * workspace: the scratch is a fixed 4 MiB array inside the library, in device memory
  * that every GPU which loads the library holds until the process exits.
  *   - A call whose scratch would exceed 4 MiB (2 x num_splits x (q_heads / kv_heads) x
- *     (head_dim + 2) fp32 values plus the batch's page prefix sums) is rejected with
+ *     (head_dim + 2) fp32 values plus num_splits counters) is rejected with
  *     PKV_ERR_NO_SPACE and launches nothing.  On B200 the automatic split count
- *     (num_splits = 0) fits for every shape and batch size the kernels accept.
+ *     (num_splits = 0) fits for every shape the kernels accept.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call before any
  *     stream capture begins.
  *   - All calls on a device share the one array, which keeps the previous call's
- *     contents; nothing in it needs clearing.  Calls that overlap on the GPU (different
- *     streams, or several host threads) race on it: order them on one stream.
+ *     contents; nothing in it needs clearing (its counters are zero when the library is
+ *     loaded and every call leaves them at zero).  Calls that overlap on the GPU
+ *     (different streams, or several host threads) race on it: order them on one stream.
  *   - No cudaMalloc, cudaFree or allocating library routine is called.
  */
 int paged_decode_attention_noalloc(const pkv_pool* pool, int layer, void* out, const void* q,
                                    const int32_t* block_tables, int max_pages_per_seq,
                                    const int32_t* context_lens, int batch, int q_heads, int kv_heads,
                                    float scale, int num_splits, pkv_stream_t stream);
+
+/*
+ * Zero-fill a decode workspace (cudaMemsetAsync on `stream`) before its first use with
+ * paged_decode_attention.  INVALID_ARG for a NULL workspace with a non-zero size.
+ */
+int pkv_decode_workspace_clear(void* workspace, size_t workspace_bytes, pkv_stream_t stream);
 
 /*
  * Read and clear the device error word (PKV_DEVERR_* bits) of the current device.

@@ -196,7 +196,9 @@ def rope_append(pool, layer, q, k, v, positions, slot_mapping, theta=10000.0, st
 
 
 class DecodeWorkspace:
-    """Device scratch for paged_decode_attention, sized for a batch and a split count."""
+    """Device scratch for paged_decode_attention, sized for a batch and a split count.
+    Allocated zero-filled, as the kernel's per-partition counters require; every call
+    leaves it ready for the next one."""
 
     def __init__(self, batch, q_heads, kv_heads, head_dim, page_size, dtype, num_splits=0, device=None):
         torch = _torch()
@@ -204,7 +206,7 @@ class DecodeWorkspace:
             num_splits = pkv_decode_default_splits(q_heads, kv_heads, head_dim, page_size, dtype_code(dtype))
         self.num_splits = num_splits
         self.nbytes = pkv_decode_workspace_size(batch, q_heads, kv_heads, head_dim, num_splits)
-        self.buffer = torch.empty(self.nbytes, dtype=torch.uint8, device=device or "cuda")
+        self.buffer = torch.zeros(self.nbytes, dtype=torch.uint8, device=device or "cuda")
 
 
 def paged_decode_attention(pool, layer, out, q, block_tables, context_lens, scale, kv_heads=None,

@@ -28,8 +28,10 @@
 // the log2 domain, and accumulates p.V with packed fp32 FMAs.  At the end of a segment
 // the warps' (m, l, o) are combined through shared memory: a segment wholly inside the
 // range is normalised and written as the output; a cut one is written to one of the
-// CTA's two partial slots (2c: it began before the range, 2c+1: it continues after it)
-// for the merge kernel.
+// CTA's two partial slots (2c: it began before the range, 2c+1: it continues after it),
+// and the CTA that delivers the last partial of a cut segment (counted with an atomic in
+// the workspace, indexed by the segment's first CTA) merges them: M = max m_k,
+// out = sum_k 2^(m_k - M) o_k / sum_k 2^(m_k - M) l_k, and resets the counter.
 #ifndef PKV_DECODE_ATTENTION_CUH_
 #define PKV_DECODE_ATTENTION_CUH_
 
@@ -39,10 +41,11 @@ namespace pkv {
 
 constexpr int kDecodeWarps = 4;
 constexpr int kDecodeThreads = kDecodeWarps * 32;
-// Two ring slots per warp at page 16 / head_dim 128.  Deeper rings (3-5 slots) and a
-// third CTA per SM were measured slower on the 10-request, 32-layer decode workload.
+// Two ring slots per warp at page 16 / head_dim 128, three CTAs per SM (the MHA kernel
+// is held to 128 registers so that a RoPE/append CTA still fits beside them).  Deeper
+// rings (3-5 slots) measured slower on the 10-request, 32-layer decode workload.
 constexpr int kRingBudgetBytes = 68 * 1024;
-constexpr int kMetaHeaderBytes = 16;   // int64 chunk, int64 total units
+constexpr int kMaxMergeParts = 4;   // partials loaded per merge round
 
 struct DecodeParams {
     const void* k;              // this layer's K pool  [pages][kv_heads][P][D]
@@ -53,7 +56,7 @@ struct DecodeParams {
     const int32_t* context_lens;
     float* part_o;              // [2 * num_splits][G][D]
     float* part_ml;             // [2 * num_splits][G][2]
-    unsigned char* meta;        // chunk, W, prefix[batch + 1]
+    int* counters;              // [num_splits]: partials delivered per cut segment (zero between calls)
     int batch;
     int max_pages;
     int q_heads;
@@ -145,7 +148,7 @@ __device__ __forceinline__ void next_unit(int& b, int& g, int& j, int& np, const
 }
 
 template <int D, int P, int G, typename T>
-__global__ void __launch_bounds__(kDecodeThreads) decode_pass1_kernel(const DecodeParams p)
+__global__ void __launch_bounds__(kDecodeThreads, G == 1 ? 4 : 1) decode_pass1_kernel(const DecodeParams p)
 {
     using S = DecodeShape<D, P, G>;
     constexpr int NW = kDecodeWarps;
@@ -162,12 +165,17 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_pass1_kernel(const Deco
     float* cmb = reinterpret_cast<float*>(smem + S::kCmbOffset);
     float* pbuf_all = reinterpret_cast<float*>(smem + S::kPbufOffset);
     int* warp_tot = reinterpret_cast<int*>(smem + S::kWarpTotOffset);
+    volatile int* last_flag = warp_tot + 8;
     int* prefix = reinterpret_cast<int*>(smem + S::kScanOffset);
     int* lens = prefix + p.batch + 1;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-    // Prologue: reads only the caller's lengths and page table, which the previous
-    // kernel on the stream does not write; pool, q and workspace wait for pdl_wait.
+    // Prologue, before waiting on the previous kernel of the stream: the caller's lengths
+    // and page table, and the first cached pages (see below).  Library kernels only let
+    // their successor start once their own predecessor has finished (RoPE/append, which
+    // writes just the newest token of each sequence, is the one that lets it start
+    // earlier), so none of these is still being written; q, the newest tokens, the
+    // outputs and the workspace are touched only after pdl_wait.
     block_page_prefix<P>(p.context_lens, p.batch, prefix, lens, warp_tot);
     __syncthreads();
     const int Hkv = p.kv_heads;
@@ -190,22 +198,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_pass1_kernel(const Deco
     };
     long long win0 = 0;
     int win = load_window(0);
-
-    pdl_wait();
-    pdl_launch_dependents();
-    if (blockIdx.x == 0) {
-        long long* hdr = reinterpret_cast<long long*>(p.meta);
-        int* pre = reinterpret_cast<int*>(p.meta + kMetaHeaderBytes);
-        if (tid == 0) {
-            hdr[0] = chunk;
-            hdr[1] = W;
-        }
-        for (int b = tid; b <= p.batch; b += blockDim.x) pre[b] = prefix[b];
-    }
-    if (r0 >= r1) return;
-
-    unsigned char* ring = smem + warp * DEPTH * S::kSlot;
-    float* pbuf = pbuf_all + warp * G * P;
+    const int ring_off = warp * DEPTH * S::kSlot;
 
     // ---- issue side: this warp's page k (iterator at unit r0 + warp + k NW).
     // K rows land XOR-swizzled by 16-byte chunk -- chunk c of row t at position
@@ -216,13 +209,13 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_pass1_kernel(const Deco
         locate_unit(r0 + warp, prefix, p.batch, Hkv, ib, ig, ij);
         inp = prefix[ib + 1] - prefix[ib];
     }
-    auto issue = [&](long long k) {
+    auto issue_kv = [&](long long k) {
         if (k >= win0 + 32) {
             win0 = k;
             win = load_window(k);
         }
         const int page = __shfl_sync(0xffffffffu, win, (int)(k - win0));
-        unsigned char* slot = ring + (int)(k % DEPTH) * S::kSlot;
+        unsigned char* slot = smem + ring_off + (int)(k % DEPTH) * S::kSlot;
         if ((unsigned)page < (unsigned)p.num_pages) {
             const long long off = ((long long)page * Hkv + ig) * (P * D);
             const unsigned char* ks = reinterpret_cast<const unsigned char*>(static_cast<const T*>(p.k) + off);
@@ -238,24 +231,67 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_pass1_kernel(const Deco
         } else if (lane == 0) {
             atomicOr(&g_error_word, PKV_DEVERR_BAD_PAGE);   // never dereferenced
         }
-        if (ib != qb || ig != qg) {           // first page of a (sequence, kv head) for this warp
-            qb = ib;
-            qg = ig;
-            const unsigned char* qs = reinterpret_cast<const unsigned char*>(
-                static_cast<const T*>(p.q) + ((long long)ib * p.q_heads + (long long)ig * G) * D);
-            for (int n = lane; n < QV; n += 32) cp_async16(slot + 2 * S::kChunk + n * 16, qs + n * 16);
-        }
+    };
+    auto issue_q = [&](long long k, int bq, int gq) {    // the group's q rows into page k's slot
+        unsigned char* slot = smem + ring_off + (int)(k % DEPTH) * S::kSlot;
+        const unsigned char* qs = reinterpret_cast<const unsigned char*>(
+            static_cast<const T*>(p.q) + ((long long)bq * p.q_heads + (long long)gq * G) * D);
+        for (int n = lane; n < QV; n += 32) cp_async16(slot + 2 * S::kChunk + n * 16, qs + n * 16);
+    };
+    auto advance = [&]() {
         if (ij + NW < inp) {
             ij += NW;                          // common case: same (sequence, kv head)
         } else {
             for (int t = 0; t < NW; ++t) next_unit(ib, ig, ij, inp, prefix, Hkv, p.batch);
         }
     };
-#pragma unroll
-    for (int k = 0; k < DEPTH; ++k) {
+    auto issue = [&](long long k) {
+        issue_kv(k);
+        if (ib != qb || ig != qg) {           // first page of a (sequence, kv head) for this warp
+            qb = ib;
+            qg = ig;
+            issue_q(k, ib, ig);
+        }
+        advance();
+    };
+    // Before waiting on the previous kernel: prefetch this warp's first pages, except a
+    // page holding a sequence's newest token (the append before this kernel may still be
+    // writing it) and the q rows (the kernel before may still be producing them).
+    int m_pre = 0, pre_qb[DEPTH], pre_qg[DEPTH];
+    for (; m_pre < DEPTH && m_pre < n_mine; ++m_pre) {
+        if (ij == inp - 1) break;
+        issue_kv(m_pre);
+        pre_qb[m_pre] = -1;
+        if (ib != qb || ig != qg) {
+            qb = ib;
+            qg = ig;
+            pre_qb[m_pre] = ib;
+            pre_qg[m_pre] = ig;
+        }
+        advance();
+        cp_async_commit();
+    }
+
+    pdl_wait();
+    pdl_launch_dependents();
+    // rows with no cached token get zeros (spread over the CTAs)
+    for (int b = blockIdx.x; b < p.batch; b += gridDim.x) {
+        if (prefix[b + 1] != prefix[b]) continue;
+        T* row = static_cast<T*>(p.out) + (long long)b * p.q_heads * D;
+        for (int idx = tid; idx < p.q_heads * D; idx += blockDim.x) row[idx] = Elt<T>::from_float(0.f);
+    }
+    if (r0 >= r1) return;
+
+    unsigned char* ring = smem + ring_off;
+    float* pbuf = pbuf_all + warp * G * P;
+    for (int k = 0; k < m_pre; ++k)
+        if (pre_qb[k] >= 0) issue_q(k, pre_qb[k], pre_qg[k]);
+    if (m_pre == DEPTH) cp_async_commit();
+    for (int k = m_pre; k < DEPTH; ++k) {
         if (k < n_mine) issue(k);
         cp_async_commit();
     }
+    cp_async_wait<0>();
 
     // ---- compute side.  q.k: lane (t, h) = (lane / 2, lane % 2) dots rows t (and t + 16
     // at P = 32) over chunks h*CPL .. h*CPL+CPL-1; p.V: lane owns output columns
@@ -434,6 +470,53 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_pass1_kernel(const Deco
                 }
             }
         }
+        if (!complete) {
+            // Deliver this partial; the CTA that delivers the last one merges the segment.
+            // One thread publishes the CTA's writes (a gpu-scope fence is cumulative over
+            // the barrier) and counts them in; the merging CTA reads the other partials
+            // through L2.
+            const int c0 = (int)(seg0 / chunk), c1 = (int)((seg0 + np - 1) / chunk);
+            named_barrier(1, NW * 32);
+            if (tid == 0) {
+                __threadfence();
+                const bool last = atomicAdd(&p.counters[c0], 1) == c1 - c0;
+                if (last) __threadfence();
+                *last_flag = last;
+            }
+            named_barrier(1, NW * 32);
+            if (*last_flag) {
+                for (int idx = tid; idx < G * D; idx += NW * 32) {
+                    const int gi = idx / D, dd = idx - gi * D;
+                    float mk[kMaxMergeParts], lk[kMaxMergeParts], ok[kMaxMergeParts];
+                    float M = -INFINITY, num = 0.f, den = 0.f;
+                    for (int c = c0; c <= c1; c += kMaxMergeParts) {
+                        const int n = min(kMaxMergeParts, c1 + 1 - c);
+#pragma unroll
+                        for (int q = 0; q < kMaxMergeParts; ++q) {      // independent loads
+                            if (q < n) {
+                                const int sl = c + q == c0 ? 2 * c0 + 1 : 2 * (c + q);
+                                mk[q] = __ldcg(&p.part_ml[((long long)sl * G + gi) * 2]);
+                                lk[q] = __ldcg(&p.part_ml[((long long)sl * G + gi) * 2 + 1]);
+                                ok[q] = __ldcg(&p.part_o[((long long)sl * G + gi) * D + dd]);
+                            }
+                        }
+#pragma unroll
+                        for (int q = 0; q < kMaxMergeParts; ++q) {      // running log-sum-exp
+                            if (q < n) {
+                                const float Mn = fmaxf(M, mk[q]);
+                                const float a = fast_exp2(M - Mn), w = fast_exp2(mk[q] - Mn);
+                                num = num * a + w * ok[q];
+                                den = den * a + w * lk[q];
+                                M = Mn;
+                            }
+                        }
+                    }
+                    T* dst = static_cast<T*>(p.out) + ((long long)b * p.q_heads + (long long)g * G + gi) * D + dd;
+                    *dst = Elt<T>::from_float(num / den);
+                }
+                if (tid == 0) p.counters[c0] = 0;   // ready for the next call
+            }
+        }
         // next segment: the next kv head of this sequence, or the next non-empty sequence
         u = u_end;
         j = 0;
@@ -446,46 +529,6 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_pass1_kernel(const Deco
         }
     }
     cp_async_wait<0>();
-}
-
-// One CTA per (sequence, kv head).  Sequences with no cached token get zeros; pairs
-// finished inside one partition were written by pass 1; the others are merged from the
-// partial slots of the partitions c0..c1 that cover them: M = max m_k,
-// out = sum_k 2^(m_k - M) o_k / sum_k 2^(m_k - M) l_k.
-template <int D, int G, typename T>
-__global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeParams p)
-{
-    pdl_wait();
-    pdl_launch_dependents();
-    const int Hkv = p.kv_heads;
-    const int b = blockIdx.x / Hkv, g = blockIdx.x - b * Hkv;
-    const long long chunk = reinterpret_cast<const long long*>(p.meta)[0];
-    const int* pre = reinterpret_cast<const int*>(p.meta + kMetaHeaderBytes);
-    const int np = pre[b + 1] - pre[b];
-    T* out = static_cast<T*>(p.out) + ((long long)b * p.q_heads + (long long)g * G) * D;
-    if (np == 0) {
-        for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) out[idx] = Elt<T>::from_float(0.f);
-        return;
-    }
-    const long long seg0 = (long long)Hkv * pre[b] + (long long)g * np;
-    const int c0 = (int)(seg0 / chunk), c1 = (int)((seg0 + np - 1) / chunk);
-    if (c0 == c1) return;
-    for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
-        const int gi = idx / D, dd = idx - gi * D;
-        float M = -INFINITY;
-        for (int c = c0; c <= c1; ++c) {
-            const int slot = c == c0 ? 2 * c0 + 1 : 2 * c;
-            M = fmaxf(M, p.part_ml[((long long)slot * G + gi) * 2]);
-        }
-        float num = 0.f, den = 0.f;
-        for (int c = c0; c <= c1; ++c) {
-            const int slot = c == c0 ? 2 * c0 + 1 : 2 * c;
-            const float wt = fast_exp2(p.part_ml[((long long)slot * G + gi) * 2] - M);
-            num = fmaf(wt, p.part_o[((long long)slot * G + gi) * D + dd], num);
-            den = fmaf(wt, p.part_ml[((long long)slot * G + gi) * 2 + 1], den);
-        }
-        out[idx] = Elt<T>::from_float(num / den);
-    }
 }
 
 }  // namespace pkv

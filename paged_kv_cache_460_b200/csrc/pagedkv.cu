@@ -75,13 +75,11 @@ struct DecodeImpl {
         cudaError_t e = ensure_smem(decode_pass1_kernel<D, P, G, T>, smem, configured);
         if (e != cudaSuccess) return PKV_ERR_CUDA;
         e = launch_pdl(decode_pass1_kernel<D, P, G, T>, dim3(prm.num_splits), dim3(kDecodeThreads), smem, st, prm);
-        if (e != cudaSuccess) return PKV_ERR_CUDA;
-        e = launch_pdl(decode_merge_kernel<D, G, T>, dim3(prm.batch * prm.kv_heads), dim3(128), 0, st, prm);
         return status_of(e);
     }
 
     // SMs x resident CTAs per SM (at the shared-memory size of a 64-row batch), at most
-    // two per SM: a third CTA per SM measured slower on the 10-request decode workload.
+    // three per SM: a fourth did not fit beside the RoPE/append kernel and ran slower.
     static int splits(int* out)
     {
         int dev = 0, sms = 0, per_sm = 0;
@@ -92,7 +90,7 @@ struct DecodeImpl {
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_pass1_kernel<D, P, G, T>, kDecodeThreads,
                                                           smem) != cudaSuccess)
             return PKV_ERR_CUDA;
-        *out = sms * (per_sm > 2 ? 2 : (per_sm > 0 ? per_sm : 1));
+        *out = sms * (per_sm > 3 ? 3 : (per_sm > 0 ? per_sm : 1));
         return PKV_OK;
     }
 };
@@ -132,14 +130,15 @@ bool pick_decode(int head_dim, int page_size, int group, int dtype, DecodeOps& o
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct WorkspaceLayout {
-    size_t meta, part_o, part_ml, total;
+    size_t counters, part_o, part_ml, total;
 };
 
 WorkspaceLayout workspace_layout(int batch, int group, int head_dim, int num_splits)
 {
+    (void)batch;
     WorkspaceLayout w;
-    w.meta = 0;
-    w.part_o = align256(kMetaHeaderBytes + sizeof(int) * ((size_t)batch + 1));
+    w.counters = 0;
+    w.part_o = align256(sizeof(int) * (size_t)num_splits);
     w.part_ml = w.part_o + align256(sizeof(float) * 2 * (size_t)num_splits * group * head_dim);
     w.total = w.part_ml + align256(sizeof(float) * 2 * (size_t)num_splits * group * 2);
     return w;
@@ -294,7 +293,7 @@ extern "C" int paged_decode_attention(const pkv_pool* pool, int layer, void* out
     prm.block_tables = block_tables;
     prm.context_lens = context_lens;
     unsigned char* ws = static_cast<unsigned char*>(workspace);
-    prm.meta = ws + wl.meta;
+    prm.counters = reinterpret_cast<int*>(ws + wl.counters);
     prm.part_o = reinterpret_cast<float*>(ws + wl.part_o);
     prm.part_ml = reinterpret_cast<float*>(ws + wl.part_ml);
     prm.batch = batch;
@@ -305,6 +304,13 @@ extern "C" int paged_decode_attention(const pkv_pool* pool, int layer, void* out
     prm.num_splits = num_splits;
     prm.scale_log2 = scale * 1.4426950408889634f;
     return ops.launch(prm, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int pkv_decode_workspace_clear(void* workspace, size_t workspace_bytes, pkv_stream_t stream)
+{
+    if (!workspace && workspace_bytes) return PKV_ERR_INVALID_ARG;
+    if (!workspace_bytes) return PKV_OK;
+    return status_of(cudaMemsetAsync(workspace, 0, workspace_bytes, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 extern "C" int kv_get_device_error(uint32_t* err_out)
@@ -371,8 +377,8 @@ extern "C" int paged_decode_attention_noalloc(const pkv_pool* pool, int layer, v
     void* scratch = nullptr;
     const int st = static_scratch_address(&scratch);
     if (st != PKV_OK) return st;
-    // Nothing in the scratch has to start at zero: every value a call reads was written
-    // earlier in the same call, so the previous call's contents do no harm.
+    // The scratch's only state that outlives a call is its counters, which are zero when
+    // the library is loaded and which every call leaves at zero.
     return paged_decode_attention(pool, layer, out, q, block_tables, max_pages_per_seq, context_lens, batch,
                                   q_heads, kv_heads, scale, num_splits, scratch, kStaticScratchBytes, stream);
 }

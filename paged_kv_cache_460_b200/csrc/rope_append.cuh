@@ -34,7 +34,8 @@ struct RopeAppendParams {
 // Grid: (token, part).  Each thread handles one 16-byte vector (8 elements, 4 pairs)
 // of the token's q, k or v rows.  The head_dim/2 angles pos * theta^(-2i/d) and their
 // cosines and sines are evaluated once per CTA in fp64 before griddepcontrol.wait, so
-// this prologue overlaps the previous kernel on the stream; each pair is then turned in
+// this prologue overlaps the previous kernel on the stream (and the attention kernel
+// after it may start its prefetch during this one); each pair is then turned in
 // fp64 (explicit _rn products: no fused rounding) and rounded once to the storage type.
 // Appending copies the rotated k and the v vector bit for bit into row slot % P of page
 // slot / P; a negative slot skips the token, a slot past the pool is skipped and flagged.
@@ -55,8 +56,10 @@ __global__ void __launch_bounds__(256) rope_append_kernel(const RopeAppendParams
         }
     }
     __syncthreads();
-    pdl_wait();
+    // Let the attention kernel that follows start now: before its own wait it reads only
+    // pages that this kernel does not write (it skips those holding a newest token).
     pdl_launch_dependents();
+    pdl_wait();
     int64_t slot = -1;
     if (p.mode & kRopeAppend) {
         slot = p.slots[t];

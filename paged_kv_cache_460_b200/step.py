@@ -2,9 +2,9 @@
 
 "为什么要自己动手写一个LLM推理引擎" (wzjinhao.cn/news/61427) s5.3 names per-call launch
 and CPU-sync overhead as a decode bottleneck.  DecodeStep issues every layer's
-RoPE + KV append (one fused kernel) and paged attention (streaming pass and merge)
-from one CUDA graph, so a step costs one graph launch instead of three kernel
-launches per layer from Python.  The graph
+RoPE + KV append (one fused kernel) and paged attention (one kernel) from one
+CUDA graph, so a step costs one graph launch instead of two kernel launches per
+layer from Python.  The graph
 reads fixed device buffers; `run` copies a step's inputs from (pinned) host memory
 into them, replays the graph and copies the outputs back.  All arithmetic stays in
 the library's kernels; this module only orders the calls.
@@ -45,11 +45,11 @@ class DecodeStep:
         self.theta = theta
         self.workspace = DecodeWorkspace(batch, q_heads, Hkv, d, pool.page_size, dt, num_splits, device=dev)
         self.graph = None
-        self.kernels_per_step = 3 * L
+        self.kernels_per_step = 2 * L
 
     def layer(self, i, stream=None):
         """Enqueue layer i of the step on the current stream: RoPE + KV append (one
-        kernel), then attention (streaming pass + merge)."""
+        kernel), then attention (one kernel)."""
         rope_append(self.pool, i, self.q[i], self.k[i], self.v[i], self.positions, self.slot_mapping, self.theta,
                     stream)
         paged_decode_attention(self.pool, i, self.out[i], self.q[i], self.block_tables, self.context_lens,

@@ -147,6 +147,23 @@ def test_split_count_sweep():
     assert np.array_equal(to_bits(c3.gpu_layer(0, num_splits=7)), outs[3])
 
 
+def test_reused_workspace_gives_identical_bits():
+    """The merge counters in the workspace are back at zero after every call."""
+    s = synth.random_spec(450, 5, 8, 4, 128, 16, [900, 33, 0, 300, 1500], dtype="bf16")
+    c = Case(s)
+    c.gpu_layer(0)                               # the append has happened; now attention only
+    ws = pkv.DecodeWorkspace(s.batch, s.q_heads, s.kv_heads, s.head_dim, s.page_size, TDT[s.dtype], 7)
+    q = c.last_q
+    outs = []
+    for _ in range(3):
+        out = torch.empty_like(q)
+        pkv.paged_decode_attention(c.pool, 0, out, q, c.bt_t, c.cl_t, c.scale, num_splits=7, workspace=ws)
+        outs.append(to_bits(out))
+    assert np.array_equal(outs[0], outs[1]) and np.array_equal(outs[1], outs[2])
+    assert (ws.buffer[:7 * 4].view(torch.int32) == 0).all().item()
+    _expect_close(outs[0], c.oracle_layer(0), "bf16", "reused workspace")
+
+
 def test_physical_page_permutation_gives_identical_bits():
     s = synth.random_spec(500, 4, 8, 4, 128, 16, [500, 77, 16, 1200], dtype="bf16")
     c = Case(s)
