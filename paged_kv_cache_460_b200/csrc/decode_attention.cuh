@@ -147,6 +147,99 @@ __device__ __forceinline__ void next_unit(int& b, int& g, int& j, int& np, const
     } while (np == 0);
 }
 
+// End of a segment, after every warp has published its (m, l, o) of it in `buf`
+// ([warps][G][D + 2]: o, then m and l): combine the warps; a segment wholly inside the
+// CTA's range [r0, r1) is normalised and written as the output, a cut one leaves a
+// partial in one of the CTA's two slots (2c: it began before the range, 2c+1: it goes on
+// after it), and the CTA that delivers the last partial of a segment merges them:
+// M = max m_k, out = sum_k 2^(m_k - M) o_k / sum_k 2^(m_k - M) l_k.  The delivery is
+// counted with an atomic in the workspace (indexed by the segment's first CTA); one
+// thread publishes the CTA's writes with a gpu-scope fence (cumulative over the barrier)
+// and the merging CTA reads the other partials through L2, then resets the counter.
+template <int D, int G, typename T>
+__device__ __forceinline__ void segment_epilogue(const DecodeParams& p, const float* buf, int b, int g, int np,
+                                                 const int* prefix, long long r0, long long r1, long long chunk,
+                                                 volatile int* last_flag)
+{
+    constexpr int NW = kDecodeWarps;
+    const int tid = threadIdx.x;
+    named_barrier(1, kDecodeThreads);
+    const long long seg0 = (long long)p.kv_heads * prefix[b] + (long long)g * np;
+    const bool complete = seg0 >= r0 && seg0 + np <= r1;
+    const int pslot = seg0 < r0 ? 2 * blockIdx.x : 2 * blockIdx.x + 1;
+    for (int idx = tid; idx < G * D; idx += kDecodeThreads) {
+        const int gi = idx / D, dd = idx - gi * D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) M = fmaxf(M, buf[(w * G + gi) * (D + 2) + D]);
+        float num = 0.f, den = 0.f;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+            const float* row = buf + (w * G + gi) * (D + 2);
+            const float wt = fast_exp2(row[D] - M);   // a warp with no page here has m = -inf
+            num = fmaf(wt, row[dd], num);
+            den = fmaf(wt, row[D + 1], den);
+        }
+        if (complete) {
+            T* dst = static_cast<T*>(p.out) + ((long long)b * p.q_heads + (long long)g * G + gi) * D + dd;
+            *dst = Elt<T>::from_float(num / den);
+        } else {
+            p.part_o[((long long)pslot * G + gi) * D + dd] = num;
+            if (dd == 0) {
+                p.part_ml[((long long)pslot * G + gi) * 2 + 0] = M;
+                p.part_ml[((long long)pslot * G + gi) * 2 + 1] = den;
+            }
+        }
+    }
+    if (!complete) {
+        // Deliver this partial; the CTA that delivers the last one merges the segment.
+        // One thread publishes the CTA's writes (a gpu-scope fence is cumulative over
+        // the barrier) and counts them in; the merging CTA reads the other partials
+        // through L2.
+        const int c0 = (int)(seg0 / chunk), c1 = (int)((seg0 + np - 1) / chunk);
+        named_barrier(1, kDecodeThreads);
+        if (tid == 0) {
+            __threadfence();
+            const bool last = atomicAdd(&p.counters[c0], 1) == c1 - c0;
+            if (last) __threadfence();
+            *last_flag = last;
+        }
+        named_barrier(1, kDecodeThreads);
+        if (*last_flag) {
+            for (int idx = tid; idx < G * D; idx += kDecodeThreads) {
+                const int gi = idx / D, dd = idx - gi * D;
+                float mk[kMaxMergeParts], lk[kMaxMergeParts], ok[kMaxMergeParts];
+                float M = -INFINITY, num = 0.f, den = 0.f;
+                for (int c = c0; c <= c1; c += kMaxMergeParts) {
+                    const int n = min(kMaxMergeParts, c1 + 1 - c);
+#pragma unroll
+                    for (int q = 0; q < kMaxMergeParts; ++q) {      // independent loads
+                        if (q < n) {
+                            const int sl = c + q == c0 ? 2 * c0 + 1 : 2 * (c + q);
+                            mk[q] = __ldcg(&p.part_ml[((long long)sl * G + gi) * 2]);
+                            lk[q] = __ldcg(&p.part_ml[((long long)sl * G + gi) * 2 + 1]);
+                            ok[q] = __ldcg(&p.part_o[((long long)sl * G + gi) * D + dd]);
+                        }
+                    }
+#pragma unroll
+                    for (int q = 0; q < kMaxMergeParts; ++q) {      // running log-sum-exp
+                        if (q < n) {
+                            const float Mn = fmaxf(M, mk[q]);
+                            const float a = fast_exp2(M - Mn), w = fast_exp2(mk[q] - Mn);
+                            num = num * a + w * ok[q];
+                            den = den * a + w * lk[q];
+                            M = Mn;
+                        }
+                    }
+                }
+                T* dst = static_cast<T*>(p.out) + ((long long)b * p.q_heads + (long long)g * G + gi) * D + dd;
+                *dst = Elt<T>::from_float(num / den);
+            }
+            if (tid == 0) p.counters[c0] = 0;   // ready for the next call
+        }
+    }
+}
+
 template <int D, int P, int G, typename T>
 __global__ void __launch_bounds__(kDecodeThreads, G == 1 ? 4 : 1) decode_pass1_kernel(const DecodeParams p)
 {
@@ -442,81 +535,7 @@ __global__ void __launch_bounds__(kDecodeThreads, G == 1 ? 4 : 1) decode_pass1_k
 #pragma unroll
             for (int e = 0; e < EPL; ++e) o[gi][e] = 0.f;
         }
-        named_barrier(1, NW * 32);
-        const long long seg0 = (long long)Hkv * prefix[b] + (long long)g * np;
-        const bool complete = seg0 >= r0 && seg0 + np <= r1;
-        const int pslot = seg0 < r0 ? 2 * blockIdx.x : 2 * blockIdx.x + 1;
-        for (int idx = tid; idx < G * D; idx += NW * 32) {
-            const int gi = idx / D, dd = idx - gi * D;
-            float M = -INFINITY;
-#pragma unroll
-            for (int w = 0; w < NW; ++w) M = fmaxf(M, buf[(w * G + gi) * (D + 2) + D]);
-            float num = 0.f, den = 0.f;
-#pragma unroll
-            for (int w = 0; w < NW; ++w) {
-                const float* row = buf + (w * G + gi) * (D + 2);
-                const float wt = fast_exp2(row[D] - M);   // a warp with no page here has m = -inf
-                num = fmaf(wt, row[dd], num);
-                den = fmaf(wt, row[D + 1], den);
-            }
-            if (complete) {
-                T* dst = static_cast<T*>(p.out) + ((long long)b * p.q_heads + (long long)g * G + gi) * D + dd;
-                *dst = Elt<T>::from_float(num / den);
-            } else {
-                p.part_o[((long long)pslot * G + gi) * D + dd] = num;
-                if (dd == 0) {
-                    p.part_ml[((long long)pslot * G + gi) * 2 + 0] = M;
-                    p.part_ml[((long long)pslot * G + gi) * 2 + 1] = den;
-                }
-            }
-        }
-        if (!complete) {
-            // Deliver this partial; the CTA that delivers the last one merges the segment.
-            // One thread publishes the CTA's writes (a gpu-scope fence is cumulative over
-            // the barrier) and counts them in; the merging CTA reads the other partials
-            // through L2.
-            const int c0 = (int)(seg0 / chunk), c1 = (int)((seg0 + np - 1) / chunk);
-            named_barrier(1, NW * 32);
-            if (tid == 0) {
-                __threadfence();
-                const bool last = atomicAdd(&p.counters[c0], 1) == c1 - c0;
-                if (last) __threadfence();
-                *last_flag = last;
-            }
-            named_barrier(1, NW * 32);
-            if (*last_flag) {
-                for (int idx = tid; idx < G * D; idx += NW * 32) {
-                    const int gi = idx / D, dd = idx - gi * D;
-                    float mk[kMaxMergeParts], lk[kMaxMergeParts], ok[kMaxMergeParts];
-                    float M = -INFINITY, num = 0.f, den = 0.f;
-                    for (int c = c0; c <= c1; c += kMaxMergeParts) {
-                        const int n = min(kMaxMergeParts, c1 + 1 - c);
-#pragma unroll
-                        for (int q = 0; q < kMaxMergeParts; ++q) {      // independent loads
-                            if (q < n) {
-                                const int sl = c + q == c0 ? 2 * c0 + 1 : 2 * (c + q);
-                                mk[q] = __ldcg(&p.part_ml[((long long)sl * G + gi) * 2]);
-                                lk[q] = __ldcg(&p.part_ml[((long long)sl * G + gi) * 2 + 1]);
-                                ok[q] = __ldcg(&p.part_o[((long long)sl * G + gi) * D + dd]);
-                            }
-                        }
-#pragma unroll
-                        for (int q = 0; q < kMaxMergeParts; ++q) {      // running log-sum-exp
-                            if (q < n) {
-                                const float Mn = fmaxf(M, mk[q]);
-                                const float a = fast_exp2(M - Mn), w = fast_exp2(mk[q] - Mn);
-                                num = num * a + w * ok[q];
-                                den = den * a + w * lk[q];
-                                M = Mn;
-                            }
-                        }
-                    }
-                    T* dst = static_cast<T*>(p.out) + ((long long)b * p.q_heads + (long long)g * G + gi) * D + dd;
-                    *dst = Elt<T>::from_float(num / den);
-                }
-                if (tid == 0) p.counters[c0] = 0;   // ready for the next call
-            }
-        }
+        segment_epilogue<D, G, T>(p, buf, b, g, np, prefix, r0, r1, chunk, last_flag);
         // next segment: the next kv head of this sequence, or the next non-empty sequence
         u = u_end;
         j = 0;

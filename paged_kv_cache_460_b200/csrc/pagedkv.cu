@@ -13,6 +13,7 @@
 #include <mutex>
 
 #include "decode_attention.cuh"
+#include "decode_attention_mma.cuh"
 #include "pagedkv.h"
 #include "pkv_internal.h"
 #include "rope_append.cuh"
@@ -63,18 +64,31 @@ struct DecodeOps {
     int group;
 };
 
+// One query head per kv head: the CUDA-core kernel; 2 to 8 heads sharing a kv head: the
+// tensor-core kernel.
+template <int D, int P, int G, typename T, bool kMma = (G > 1)>
+struct DecodeKernel {
+    static constexpr auto fn = decode_pass1_kernel<D, P, G, T>;
+    static int smem(int batch) { return DecodeShape<D, P, G>::smem_bytes(batch); }
+};
+template <int D, int P, int G, typename T>
+struct DecodeKernel<D, P, G, T, true> {
+    static constexpr auto fn = decode_pass1_mma_kernel<D, P, G, T>;
+    static int smem(int batch) { return MmaShape<D, G>::smem_bytes(batch); }
+};
+
 template <int D, int P, int G, typename T>
 struct DecodeImpl {
-    using S = DecodeShape<D, P, G>;
+    using K = DecodeKernel<D, P, G, T>;
     static int configured[kMaxDevices];
 
     static int launch(const DecodeParams& prm, cudaStream_t st)
     {
-        const int smem = S::smem_bytes(prm.batch);
+        const int smem = K::smem(prm.batch);
         if (smem > kMaxSmemPerCta) return PKV_ERR_UNSUPPORTED;
-        cudaError_t e = ensure_smem(decode_pass1_kernel<D, P, G, T>, smem, configured);
+        cudaError_t e = ensure_smem(K::fn, smem, configured);
         if (e != cudaSuccess) return PKV_ERR_CUDA;
-        e = launch_pdl(decode_pass1_kernel<D, P, G, T>, dim3(prm.num_splits), dim3(kDecodeThreads), smem, st, prm);
+        e = launch_pdl(K::fn, dim3(prm.num_splits), dim3(kDecodeThreads), smem, st, prm);
         return status_of(e);
     }
 
@@ -85,10 +99,9 @@ struct DecodeImpl {
         int dev = 0, sms = 0, per_sm = 0;
         if (cudaGetDevice(&dev) != cudaSuccess) return PKV_ERR_CUDA;
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return PKV_ERR_CUDA;
-        const int smem = S::smem_bytes(64);
-        if (ensure_smem(decode_pass1_kernel<D, P, G, T>, smem, configured) != cudaSuccess) return PKV_ERR_CUDA;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_pass1_kernel<D, P, G, T>, kDecodeThreads,
-                                                          smem) != cudaSuccess)
+        const int smem = K::smem(64);
+        if (ensure_smem(K::fn, smem, configured) != cudaSuccess) return PKV_ERR_CUDA;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, K::fn, kDecodeThreads, smem) != cudaSuccess)
             return PKV_ERR_CUDA;
         *out = sms * (per_sm > 3 ? 3 : (per_sm > 0 ? per_sm : 1));
         return PKV_OK;
