@@ -161,6 +161,11 @@ def dist_setup(args):
     return world, rank, local
 
 
+def throughput(world, bytes_per_step, steps, ms):
+    """Whole-job GB/s: the bytes of all `world` replicas over the slowest rank's time."""
+    return world * bytes_per_step * steps / (ms * 1e-3) / 1e9
+
+
 def max_over_ranks(value, world, device=None):
     """Max of a per-rank float across the process group (the identity with one rank)."""
     if world == 1:
@@ -364,7 +369,7 @@ def run_ours(args):
         saved, args.steps = args.steps, n_e2e
         ms_e2e = max_over_ranks(timed(e2e_step), world, dev)
         args.steps = saved
-        e2e = {"value": world * s.kv_bytes_read() * L * n_e2e / (ms_e2e * 1e-3) / 1e9, "unit": UNIT,
+        e2e = {"value": throughput(world, s.kv_bytes_read() * L, n_e2e, ms_e2e), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e / n_e2e}
 
     err = pkv.kv_get_device_error()
@@ -373,7 +378,7 @@ def run_ours(args):
 
     if rank == 0:
         per_step_ms = ms_total / args.steps
-        value = world * s.kv_bytes_read() * L * args.steps / (ms_total * 1e-3) / 1e9
+        value = throughput(world, s.kv_bytes_read() * L, args.steps, ms_total)
         peak, peak_kind = measured_peaks()
         achieved = s.kv_bytes_read() / (attn_ms_mean * 1e-3) / 1e9
         cpu = None
