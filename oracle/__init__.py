@@ -54,6 +54,7 @@ def _load():
         lib.ora_decode_attention.argtypes = [P, P, P, P, I, P, I, I, I, I, I, D, I, P, P, I]
         lib.ora_decode_attention_pairs.argtypes = [P, P, P, P, I, P, I, I, I, I, D, I, P, P, I, P]
         lib.ora_causal_attention_full.argtypes = [P, P, P, I, I, I, I, D, P]
+        lib.ora_rms_norm.argtypes = [P, P, P, I, I, D, I, P, P, P]
         lib.ora_kv_cache_bytes.argtypes = [I, I, I, I64, I]
         lib.ora_kv_cache_bytes.restype = I64
         _lib = lib
@@ -188,3 +189,19 @@ def causal_attention_full(q, k, v, scale):
 
 def kv_cache_bytes(layers, heads, head_dim, tokens, elt_bytes):
     return int(_load().ora_kv_cache_bytes(layers, heads, head_dim, tokens, elt_bytes))
+
+
+# ----------------------------------------------------------------- RMSNorm
+def rms_norm(x, w, eps, dtype, residual=None):
+    """x: uint16 [rows, hidden]; w: uint16 [hidden].  Returns (rounded bits, exact float64,
+    rounded residual sums or None)."""
+    x = _c(x, np.uint16)
+    w = _c(w, np.uint16)
+    rows, hidden = x.shape
+    out = np.empty_like(x)
+    exact = np.empty(x.shape, np.float64)
+    res = _c(residual, np.uint16) if residual is not None else None
+    res_out = np.empty_like(x) if residual is not None else None
+    _load().ora_rms_norm(_p(x), _p(res) if res is not None else None, _p(w), rows, hidden, float(eps),
+                         _DT[dtype], _p(out), _p(exact), _p(res_out) if res_out is not None else None)
+    return out, exact, res_out

@@ -428,3 +428,43 @@ int64_t ora_kv_cache_bytes(int layers, int heads, int head_dim, int64_t tokens, 
 {
     return (int64_t)layers * 2 * heads * head_dim * tokens * elt_bytes;
 }
+
+/* ------------------------------------------------------------------------- */
+/* RMSNorm  [ENGINE] s4.2                                                      */
+/* ------------------------------------------------------------------------- */
+
+/*
+ * RMSNorm of each row, in double: y = x / sqrt(mean(x^2) + eps) * w.  The page is
+ * explicit that eps is added to the mean square before the square root (not to the
+ * root).  With a residual (optional), the row first becomes h = x + residual, rounded
+ * once to the storage type (that rounded sum is also returned), and h is normalised.
+ *   x, residual, out: [rows][hidden] storage; w: [hidden]; exact_out (optional): the
+ *   unrounded doubles of y; residual_out (when residual is given): the rounded sums.
+ */
+void ora_rms_norm(const uint16_t* x, const uint16_t* residual, const uint16_t* w, int rows, int hidden,
+                  double eps, int dtype, uint16_t* out, double* exact_out, uint16_t* residual_out)
+{
+    for (int r = 0; r < rows; ++r) {
+        const int64_t base = (int64_t)r * hidden;
+        double* h = (double*)malloc(sizeof(double) * (size_t)hidden);
+        for (int i = 0; i < hidden; ++i) {
+            double v = dec(x[base + i], dtype);
+            if (residual) {
+                uint16_t sum = enc(v + dec(residual[base + i], dtype), dtype);
+                residual_out[base + i] = sum;
+                v = dec(sum, dtype);
+            }
+            h[i] = v;
+        }
+        double ms = 0.0;
+        for (int i = 0; i < hidden; ++i) ms += h[i] * h[i];
+        ms /= hidden;
+        double inv = 1.0 / sqrt(ms + eps);
+        for (int i = 0; i < hidden; ++i) {
+            double y = h[i] * inv * dec(w[i], dtype);
+            out[base + i] = enc(y, dtype);
+            if (exact_out) exact_out[base + i] = y;
+        }
+        free(h);
+    }
+}

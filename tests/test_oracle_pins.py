@@ -358,3 +358,47 @@ def test_workload_kv_bytes_match_size_model():
     s = synth.spec("layer7b")
     assert s.kv_bytes_read() == 2049 * 2 * 32 * 128 * 2
     assert oracle.kv_cache_bytes(1, 32, 128, 2049, 2) == s.kv_bytes_read()
+
+
+# ------------------------------------------------------------------ RMSNorm
+def test_rms_norm_eps_sits_inside_the_root():
+    """[ENGINE] s4.2: eps is added to the mean square, then the root is taken.  A constant
+    row c makes both placements closed forms that differ clearly for small c."""
+    c, eps, hidden = 1e-3, 1e-6, 64
+    x = np.full((1, hidden), c)
+    bits = oracle.encode(x, "f16")
+    cd = oracle.decode(bits[0, :1], "f16")[0]
+    w = oracle.encode(np.ones(hidden), "f16")
+    _, exact, _ = oracle.rms_norm(bits, w, eps, "f16")
+    inside = cd / math.sqrt(cd * cd + eps)
+    outside = cd / (math.sqrt(cd * cd) + eps)
+    assert np.allclose(exact, inside, rtol=1e-12, atol=0)
+    assert abs(inside - outside) > 0.2
+
+
+def test_rms_norm_brute_force_and_unit_rms():
+    r = np.random.Generator(np.random.PCG64(70))
+    x = synth.round_f32(r.standard_normal((3, 24), dtype=np.float32), "bf16")
+    w = synth.round_f32(r.standard_normal(24, dtype=np.float32), "bf16")
+    _, exact, _ = oracle.rms_norm(x, w, 1e-6, "bf16")
+    xd, wd = oracle.decode(x, "bf16"), oracle.decode(w, "bf16")
+    for i in range(3):
+        row = [float(v) for v in xd[i]]
+        inv = 1.0 / math.sqrt(math.fsum(v * v for v in row) / len(row) + 1e-6)
+        ref = [row[k] * inv * float(wd[k]) for k in range(24)]
+        assert np.allclose(exact[i], ref, rtol=1e-12, atol=1e-15)
+    ones = oracle.encode(np.ones(24), "bf16")
+    _, unit, _ = oracle.rms_norm(x, ones, 0.0, "bf16")
+    assert np.allclose((unit ** 2).mean(axis=1), 1.0, rtol=1e-12)
+
+
+def test_rms_norm_residual_is_summed_and_rounded_first():
+    r = np.random.Generator(np.random.PCG64(71))
+    x = synth.round_f32(r.standard_normal((2, 16), dtype=np.float32), "f16")
+    res = synth.round_f32(r.standard_normal((2, 16), dtype=np.float32), "f16")
+    w = oracle.encode(np.ones(16), "f16")
+    y, exact, summed = oracle.rms_norm(x, w, 1e-6, "f16", residual=res)
+    expect_sum = (oracle.decode(x, "f16") + oracle.decode(res, "f16")).astype(np.float16).view(np.uint16)
+    assert np.array_equal(summed, expect_sum)
+    y2, exact2, _ = oracle.rms_norm(summed, w, 1e-6, "f16")
+    assert np.array_equal(y, y2) and np.array_equal(exact, exact2)
