@@ -53,6 +53,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the CPU-baseline sample")
+    ap.add_argument("--op", choices=("decode", "rms_norm"), default="decode",
+                    help="decode: the decode step (default); rms_norm: the RMSNorm kernel alone")
     return ap.parse_args(argv)
 
 
@@ -413,10 +415,57 @@ def run_ours(args):
     return 0
 
 
+def run_rms_norm(args):
+    """RMSNorm (fused residual add) on the decode hidden state of the workload's batch:
+    rows = batch, hidden = q_heads * head_dim; 32 calls per step (one per layer) in a graph."""
+    import torch
+    import paged_kv_cache_460_b200 as pkv
+    s = synth.spec(args.workload, num_layers=args.layers)
+    dev = torch.device("cuda", 0)
+    tdt = torch.float16 if s.dtype == "f16" else torch.bfloat16
+    rows, hidden, L = s.batch, s.q_heads * s.head_dim, s.num_layers
+    g = torch.Generator(device=dev)
+    g.manual_seed(4242)
+    x = torch.randn((L, rows, hidden), generator=g, device=dev).to(tdt)
+    res = torch.randn((L, rows, hidden), generator=g, device=dev).to(tdt)
+    w = torch.randn((L, hidden), generator=g, device=dev).to(tdt)
+    out = torch.empty_like(x)
+    for layer in range(L):
+        pkv.rms_norm(out[layer], x[layer], w[layer], 1e-6, residual=res[layer])
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    cs = torch.cuda.Stream()
+    cs.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(cs), torch.cuda.graph(graph, stream=cs):
+        for layer in range(L):
+            pkv.rms_norm(out[layer], x[layer], w[layer], 1e-6, residual=res[layer])
+    torch.cuda.current_stream().wait_stream(cs)
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        graph.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    per_call_us = 1000.0 * ms / (args.steps * L)
+    bytes_per_call = (4 * rows * hidden + hidden) * 2          # x, residual in; residual, out back; weight
+    print(json.dumps({"metric": "rms_norm (fused residual) us per call", "value": per_call_us, "unit": "us",
+                      "higher_is_better": False, "steps": args.steps, "warmup": args.warmup,
+                      "config": {"workload": "rows %d x hidden %d, %s" % (rows, hidden, s.dtype)},
+                      "bytes_per_call": bytes_per_call, "GB_per_s": bytes_per_call / (per_call_us * 1e-6) / 1e9,
+                      "gpu_launches": args.steps * L}), flush=True)
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.op == "rms_norm":
+        return run_rms_norm(args)
     return run_ours(args)
 
 

@@ -7,7 +7,8 @@
  *            s3.4  KV-cache management: size formula; the cache cut into fixed pages of
  *                  16 or 32 tokens, allocated from a free list and given back when a
  *                  request ends; attention locates a token's block through a page index.
- *            s4.2  RoPE: position enters q and k through a rotation.
+ *            s4.2  RoPE: position enters q and k through a rotation; RMSNorm with eps
+ *                  added to the mean square before the root.
  *            s4.3  forward with a cache: n_heads / n_kv_heads views,
  *                  apply_rotary_emb(q, k, start_pos), cache update, q k^T / sqrt(head_dim)
  *                  plus causal mask, softmax, times v.
@@ -166,6 +167,19 @@ int paged_kv_append(const pkv_pool* pool, int layer, const void* k, const void* 
 int rope_append(const pkv_pool* pool, int layer, void* q, void* k, const void* v,
                 const int32_t* positions, const int64_t* slot_mapping, int n_tokens, int q_heads,
                 double theta, pkv_stream_t stream);
+
+/*
+ * RMSNorm of each row of the decode hidden state ([ENGINE] s4.2: root mean square only,
+ * eps added to the mean square before the root):
+ *   out[r][i] = h[r][i] * rsqrt(mean_i(h[r][i]^2) + eps) * weight[i]
+ * with h = x, or, when `residual` is not NULL, h = x + residual rounded once to the element
+ * type and written back to `residual` (the fused residual add of a decoder block).
+ *   out, x, residual: device [rows][hidden]; weight: device [hidden]; all 16-byte aligned;
+ *   out may be x.  hidden a multiple of 8, at most 16384; sum of squares and scaling in fp32,
+ *   one rounding of the result.
+ */
+int rms_norm(void* out, const void* x, void* residual, const void* weight, int rows, int hidden,
+             float eps, int dtype, pkv_stream_t stream);
 
 /*
  * Number of work partitions paged_decode_attention uses when called with num_splits = 0 on

@@ -55,6 +55,7 @@ def _load():
         lib.ora_decode_attention_pairs.argtypes = [P, P, P, P, I, P, I, I, I, I, D, I, P, P, I, P]
         lib.ora_causal_attention_full.argtypes = [P, P, P, I, I, I, I, D, P]
         lib.ora_rms_norm.argtypes = [P, P, P, I, I, D, I, P, P, P]
+        lib.ora_prefill_attention.argtypes = [P, P, P, P, I, P, P, I, I, I, I, I, D, I, P]
         lib.ora_kv_cache_bytes.argtypes = [I, I, I, I64, I]
         lib.ora_kv_cache_bytes.restype = I64
         _lib = lib
@@ -205,3 +206,21 @@ def rms_norm(x, w, eps, dtype, residual=None):
     _load().ora_rms_norm(_p(x), _p(res) if res is not None else None, _p(w), rows, hidden, float(eps),
                          _DT[dtype], _p(out), _p(exact), _p(res_out) if res_out is not None else None)
     return out, exact, res_out
+
+
+# ----------------------------------------------------------------- chunked prefill
+def prefill_attention(q, k_pool, v_pool, block_tables, cu_q, context_lens, scale, dtype):
+    """q: uint16 [total_q, Hq, d]; query rows of sequence b are cu_q[b] .. cu_q[b+1]-1 and
+    sit at positions context_lens[b] - n_b ... context_lens[b] - 1.  Returns float64."""
+    q = _c(q, np.uint16)
+    kp = _c(k_pool, np.uint16)
+    vp = _c(v_pool, np.uint16)
+    bt = _c(block_tables, np.int32)
+    cq = _c(cu_q, np.int32)
+    cl = _c(context_lens, np.int32)
+    total, Hq, d = q.shape
+    _, Hkv, P, _ = kp.shape
+    out = np.zeros((total, Hq, d), np.float64)
+    _load().ora_prefill_attention(_p(q), _p(kp), _p(vp), _p(bt), bt.shape[1], _p(cq), _p(cl), cl.shape[0], Hq,
+                                  Hkv, d, P, float(scale), _DT[dtype], _p(out))
+    return out

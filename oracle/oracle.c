@@ -468,3 +468,61 @@ void ora_rms_norm(const uint16_t* x, const uint16_t* residual, const uint16_t* w
         free(h);
     }
 }
+
+/* ------------------------------------------------------------------------- */
+/* chunked prefill  [ENGINE] s4.3                                              */
+/* ------------------------------------------------------------------------- */
+
+/*
+ * Attention of a chunk of new query tokens per sequence over the paged cache, with
+ * the causal mask slice [start_pos, start_pos + seq_len) of the page's forward:
+ * sequence b contributes the query rows cu_q[b] .. cu_q[b+1]-1 (n_b = cu_q[b+1] - cu_q[b]);
+ * its cache already holds the chunk (context_lens[b] = L_b tokens), so query row i sits at
+ * position start_pos + i with start_pos = L_b - n_b and sees keys 0 .. start_pos + i.
+ *   q: [cu_q[batch]][q_heads][head_dim] storage; pools and block tables as in
+ *   ora_decode_attention; out: [cu_q[batch]][q_heads][head_dim] double.
+ */
+void ora_prefill_attention(const uint16_t* q, const uint16_t* k_pool, const uint16_t* v_pool,
+                           const int32_t* block_tables, int max_pages_per_seq, const int32_t* cu_q,
+                           const int32_t* context_lens, int batch, int q_heads, int kv_heads,
+                           int head_dim, int page_size, double scale, int dtype, double* out)
+{
+    int group = q_heads / kv_heads;
+    for (int b = 0; b < batch; ++b) {
+        int n = cu_q[b + 1] - cu_q[b];
+        int len = context_lens[b];
+        if (n <= 0) continue;
+        int start = len - n;
+        double* s = (double*)malloc(sizeof(double) * (size_t)(len > 0 ? len : 1));
+        for (int i = 0; i < n; ++i) {
+            int pos = start + i;                     /* keys 0 .. pos are visible */
+            for (int h = 0; h < q_heads; ++h) {
+                int g = h / group;
+                const uint16_t* qh = q + ((int64_t)(cu_q[b] + i) * q_heads + h) * head_dim;
+                double* o = out + ((int64_t)(cu_q[b] + i) * q_heads + h) * head_dim;
+                double mx = -INFINITY;
+                for (int t = 0; t <= pos; ++t) {
+                    int64_t page = block_tables[(int64_t)b * max_pages_per_seq + t / page_size];
+                    const uint16_t* kr = k_pool + ((page * kv_heads + g) * page_size + t % page_size) * head_dim;
+                    double dot = 0.0;
+                    for (int e = 0; e < head_dim; ++e) dot += dec(qh[e], dtype) * dec(kr[e], dtype);
+                    s[t] = scale * dot;
+                    if (s[t] > mx) mx = s[t];
+                }
+                double z = 0.0;
+                for (int t = 0; t <= pos; ++t) {
+                    s[t] = exp(s[t] - mx);
+                    z += s[t];
+                }
+                for (int e = 0; e < head_dim; ++e) o[e] = 0.0;
+                for (int t = 0; t <= pos; ++t) {
+                    int64_t page = block_tables[(int64_t)b * max_pages_per_seq + t / page_size];
+                    const uint16_t* vr = v_pool + ((page * kv_heads + g) * page_size + t % page_size) * head_dim;
+                    for (int e = 0; e < head_dim; ++e) o[e] += s[t] * dec(vr[e], dtype);
+                }
+                for (int e = 0; e < head_dim; ++e) o[e] /= z;
+            }
+        }
+        free(s);
+    }
+}

@@ -23,7 +23,7 @@ from ._lib import (PKV_BF16, PKV_DEVERR_BAD_PAGE, PKV_DEVERR_BAD_SLOT, PKV_DEVER
                    PagedKVError, lib)
 
 __all__ = [
-    "KVPool", "rope_apply", "paged_kv_append", "rope_append", "paged_decode_attention", "pkv_slot_mapping",
+    "KVPool", "rope_apply", "paged_kv_append", "rope_append", "paged_decode_attention", "rms_norm", "pkv_slot_mapping",
     "pkv_kv_cache_bytes", "pkv_decode_workspace_size", "pkv_decode_default_splits",
     "kv_get_device_error", "DecodeWorkspace", "PagedKVError", "PKV_F16", "PKV_BF16",
     "PKV_DEVERR_BAD_PAGE", "PKV_DEVERR_BAD_SLOT", "PKV_DEVERR_TIMEOUT",
@@ -193,6 +193,20 @@ def rope_append(pool, layer, q, k, v, positions, slot_mapping, theta=10000.0, st
     st = lib().rope_append(pool.handle, layer, _ptr(q), _ptr(k), _ptr(v), _ptr(positions), _ptr(slot_mapping),
                            k.shape[0], q.shape[1], float(theta), _stream(stream))
     _lib.check("rope_append", st)
+
+
+def rms_norm(out, x, weight, eps=1e-6, residual=None, stream=None):
+    """out = x * rsqrt(mean(x^2) + eps) * weight per row of x [rows, hidden]; with a residual,
+    x + residual (rounded) is written back to the residual and normalised instead."""
+    _need(out, "out", x.dtype)
+    _need(x, "x", x.dtype)
+    _need(weight, "weight", x.dtype)
+    _need(residual, "residual", x.dtype)
+    rows, hidden = x.shape
+    st = lib().rms_norm(_ptr(out), _ptr(x), _ptr(residual), _ptr(weight), rows, hidden, float(eps),
+                        dtype_code(x.dtype), _stream(stream))
+    _lib.check("rms_norm", st)
+    return out
 
 
 class DecodeWorkspace:

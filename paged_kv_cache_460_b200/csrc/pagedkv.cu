@@ -16,6 +16,7 @@
 #include "decode_attention_mma.cuh"
 #include "pagedkv.h"
 #include "pkv_internal.h"
+#include "rms_norm.cuh"
 #include "rope_append.cuh"
 
 namespace pkv {
@@ -258,6 +259,28 @@ extern "C" int rope_append(const pkv_pool* pool, int layer, void* q, void* k, co
     prm.theta = theta;
     prm.mode = kRopeRotate | kRopeAppend;
     return launch_rope_append(prm, n_tokens, pool->dtype, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int rms_norm(void* out, const void* x, void* residual, const void* weight, int rows, int hidden,
+                        float eps, int dtype, pkv_stream_t stream)
+{
+    if (rows < 0 || hidden <= 0 || hidden % 8 || !(eps >= 0.f)) return PKV_ERR_INVALID_ARG;
+    if (hidden > kNormThreads * kNormMaxVecPerThread * 8) return PKV_ERR_UNSUPPORTED;
+    if (dtype != PKV_F16 && dtype != PKV_BF16) return PKV_ERR_UNSUPPORTED;
+    if (rows == 0) return PKV_OK;
+    if (!out || !x || !weight) return PKV_ERR_INVALID_ARG;
+    if (misaligned16(out, x, weight) || misaligned16(residual)) return PKV_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if (dtype == PKV_F16)
+        e = launch_pdl(rms_norm_kernel<__half>, dim3(rows), dim3(kNormThreads), 0, st, static_cast<__half*>(out),
+                       static_cast<const __half*>(x), static_cast<__half*>(residual),
+                       static_cast<const __half*>(weight), hidden, eps);
+    else
+        e = launch_pdl(rms_norm_kernel<__nv_bfloat16>, dim3(rows), dim3(kNormThreads), 0, st,
+                       static_cast<__nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(x),
+                       static_cast<__nv_bfloat16*>(residual), static_cast<const __nv_bfloat16*>(weight), hidden, eps);
+    return status_of(e);
 }
 
 extern "C" int pkv_decode_default_splits(int q_heads, int kv_heads, int head_dim, int page_size, int dtype,

@@ -205,3 +205,13 @@ def test_rope_append_validates(L):
     assert L.rope_append(h, 0, f(), f(), f(), f(), f(), 1, 2, 0.0, None) == _lib.PKV_ERR_INVALID_ARG
     assert L.rope_append(h, 0, f(), f(), f(), f(), f(), 0, 2, 10000.0, None) == 0
     L.kv_pool_destroy(h)
+
+
+def test_rms_norm_validates(L):
+    f = _fake_ptr
+    assert L.rms_norm(f(), f(), None, f(), 2, 4100, 1e-6, 0, None) == _lib.PKV_ERR_INVALID_ARG    # hidden % 8
+    assert L.rms_norm(f(), f(), None, f(), 2, 32768, 1e-6, 0, None) == _lib.PKV_ERR_UNSUPPORTED
+    assert L.rms_norm(f(), f(), None, f(), 2, 4096, -1.0, 0, None) == _lib.PKV_ERR_INVALID_ARG
+    assert L.rms_norm(None, f(), None, f(), 2, 4096, 1e-6, 0, None) == _lib.PKV_ERR_INVALID_ARG
+    assert L.rms_norm(f(), f(), f(0x10004), f(), 2, 4096, 1e-6, 0, None) == _lib.PKV_ERR_INVALID_ARG
+    assert L.rms_norm(f(), f(), None, f(), 0, 4096, 1e-6, 0, None) == 0

@@ -236,3 +236,22 @@ def test_full_size_workload_sampled(name, layers, check_layers):
         got = np.stack([outs[L][b, g * G:(g + 1) * G] for b, g, _, _ in sn])
         _expect_close(got, ref, s.dtype, "%s layer %d" % (name, L))
     assert pkv.kv_get_device_error() == 0
+
+
+# ------------------------------------------------------------------ RMSNorm
+@pytest.mark.parametrize("dtype,rows,hidden,fused", [("f16", 10, 4096, False), ("bf16", 64, 4096, True),
+                                                     ("f16", 3, 4104, True), ("bf16", 1, 16384, False)])
+def test_rms_norm_matches_oracle(dtype, rows, hidden, fused):
+    r = np.random.Generator(np.random.PCG64(900 + hidden + rows))
+    x = synth.round_f32(r.standard_normal((rows, hidden), dtype=np.float32) * 3, dtype)
+    w = synth.round_f32(1 + 0.1 * r.standard_normal(hidden, dtype=np.float32), dtype)
+    res = synth.round_f32(r.standard_normal((rows, hidden), dtype=np.float32), dtype) if fused else None
+    x_t, w_t = to_dev(x, dtype), to_dev(w, dtype)
+    res_t = to_dev(res, dtype) if fused else None
+    out = torch.empty_like(x_t)
+    pkv.rms_norm(out, x_t, w_t, 1e-6, residual=res_t)
+    ref_bits, ref_exact, ref_res = oracle.rms_norm(x, w, 1e-6, dtype, residual=res)
+    _expect_close(out, ref_exact, dtype, "rms_norm")
+    if fused:
+        assert np.array_equal(to_bits(res_t), ref_res)        # the rounded sum is bit-exact
+    assert (to_bits(out) == ref_bits).mean() > 0.99

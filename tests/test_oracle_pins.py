@@ -402,3 +402,50 @@ def test_rms_norm_residual_is_summed_and_rounded_first():
     assert np.array_equal(summed, expect_sum)
     y2, exact2, _ = oracle.rms_norm(summed, w, 1e-6, "f16")
     assert np.array_equal(y, y2) and np.array_equal(exact, exact2)
+
+
+# ------------------------------------------------------------------ chunked prefill
+def test_prefill_of_one_token_is_the_decode_step():
+    sp, q, kp, vp, _, _, scale = _logical_case(80, 3, 8, 2, 16, 4, [9, 30, 1])
+    cl = np.array([9, 30, 1], np.int32)
+    dec = oracle.decode_attention(q, kp, vp, sp.block_tables, cl, scale, "f16")
+    pre = oracle.prefill_attention(q, kp, vp, sp.block_tables, np.arange(4, dtype=np.int32), cl, scale, "f16")
+    assert np.array_equal(pre, dec)
+
+
+@pytest.mark.parametrize("T,chunk,Hq,Hkv", [(23, 23, 2, 2), (40, 9, 4, 2), (17, 5, 8, 1)])
+def test_prefill_equals_full_causal_recompute(T, chunk, Hq, Hkv):
+    """The cache check of s5.2 for a chunk: the last `chunk` rows of the full causal
+    recompute, computed from the paged cache with the mask slice [T-chunk, T)."""
+    d, P = 8, 4
+    r = np.random.Generator(np.random.PCG64(T + chunk))
+    qs = synth.round_f32(r.standard_normal((T, Hq, d), dtype=np.float32), "bf16")
+    ks = synth.round_f32(r.standard_normal((T, Hkv, d), dtype=np.float32), "bf16")
+    vs = synth.round_f32(r.standard_normal((T, Hkv, d), dtype=np.float32), "bf16")
+    full = oracle.causal_attention_full(oracle.decode(qs, "bf16"), oracle.decode(ks, "bf16"),
+                                        oracle.decode(vs, "bf16"), 1 / math.sqrt(d))
+    sp = synth.random_spec(T, 1, Hq, Hkv, d, P, [T - 1])
+    kp = np.zeros((sp.num_pages, Hkv, P, d), np.uint16)
+    vp = np.zeros_like(kp)
+    for t in range(T):
+        page = sp.block_tables[0][t // P]
+        kp[page, :, t % P] = ks[t]
+        vp[page, :, t % P] = vs[t]
+    pre = oracle.prefill_attention(qs[T - chunk:], kp, vp, sp.block_tables, np.array([0, chunk], np.int32),
+                                   np.array([T], np.int32), 1 / math.sqrt(d), "bf16")
+    assert np.allclose(pre, full[T - chunk:], rtol=1e-12, atol=1e-14)
+
+
+def test_prefill_matches_brute_force():
+    sp, q, kp, vp, Kl, Vl, scale = _logical_case(81, 2, 4, 2, 8, 4, [13, 7])
+    cq = np.array([0, 3, 5], np.int32)                     # 3 new tokens of seq 0, 2 of seq 1
+    qq = np.concatenate([q, q[:1], q[1:], q[:1]])[:5]      # any 5 query rows
+    pre = oracle.prefill_attention(qq, kp, vp, sp.block_tables, cq, np.array([13, 7], np.int32), scale, "f16")
+    for b, (lo, hi, L) in enumerate([(0, 3, 13), (3, 5, 7)]):
+        for i in range(hi - lo):
+            pos = L - (hi - lo) + i
+            for h in range(4):
+                qv = list(oracle.decode(qq[lo + i, h], "f16"))
+                ref = brute.attention_one(qv, [Kl[b][t][h // 2] for t in range(pos + 1)],
+                                          [Vl[b][t][h // 2] for t in range(pos + 1)], scale)
+                assert np.allclose(pre[lo + i, h], ref, rtol=1e-12, atol=1e-14)
