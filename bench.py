@@ -53,8 +53,9 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the CPU-baseline sample")
-    ap.add_argument("--op", choices=("decode", "rms_norm"), default="decode",
-                    help="decode: the decode step (default); rms_norm: the RMSNorm kernel alone")
+    ap.add_argument("--op", choices=("decode", "rms_norm", "prefill"), default="decode",
+                    help="decode: the decode step (default); rms_norm / prefill: that kernel alone")
+    ap.add_argument("--chunk", type=int, default=512, help="prefill: new tokens per sequence")
     return ap.parse_args(argv)
 
 
@@ -460,12 +461,84 @@ def run_rms_norm(args):
     return 0
 
 
+def run_prefill(args):
+    """Chunked prefill attention on the workload's sequences: the last `--chunk` tokens of
+    each context are the chunk (causal over the whole cached prefix); 32 calls per step, one
+    per layer, in a graph.  Reports us per call and tensor TFLOP/s (4 flops per q.k / p.V
+    multiply-add pair element) against the measured bf16 GEMM peak."""
+    import torch
+    import paged_kv_cache_460_b200 as pkv
+    s = synth.spec(args.workload, num_layers=args.layers)
+    dev = torch.device("cuda", 0)
+    tdt = torch.float16 if s.dtype == "f16" else torch.bfloat16
+    L = s.num_layers
+    kp, vp = synth.pool_values_torch(s, dev)
+    pool = pkv.KVPool(kp, vp)
+    ctx = s.context_lens.astype(np.int64)
+    chunk = np.minimum(ctx, args.chunk)
+    cu_q = np.concatenate([[0], np.cumsum(chunk)]).astype(np.int32)
+    total = int(cu_q[-1])
+    g = torch.Generator(device=dev)
+    g.manual_seed(5150)
+    q = torch.randn((L, total, s.q_heads, s.head_dim), generator=g, device=dev).to(tdt)
+    out = torch.empty_like(q)
+    cu_t = torch.from_numpy(cu_q).to(dev)
+    bt = torch.from_numpy(s.block_tables).to(dev)
+    cl = torch.from_numpy(s.context_lens).to(dev)
+    scale = 1.0 / math.sqrt(s.head_dim)
+
+    def step():
+        for layer in range(L):
+            pkv.paged_prefill_attention(pool, layer, out[layer], q[layer], cu_t, bt, cl, scale)
+
+    step()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    cs = torch.cuda.Stream()
+    cs.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(cs), torch.cuda.graph(graph, stream=cs):
+        step()
+    torch.cuda.current_stream().wait_stream(cs)
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        graph.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    per_call_us = 1000.0 * e0.elapsed_time(e1) / (args.steps * L)
+    # visible keys of row i of sequence b: L_b - n_b + i + 1
+    keys = sum(int(n) * int(c - n) + int(n) * (int(n) + 1) // 2 for c, n in zip(ctx, chunk))
+    flops = 4.0 * keys * s.head_dim * s.q_heads
+    tflops = flops / (per_call_us * 1e-6) / 1e12
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peak = float(json.load(f)["bf16_tflops"])
+        kind = "measured"
+    except Exception:
+        peak, kind = 1590.0, "fallback"
+    print(json.dumps({"metric": "paged chunked-prefill attention us per call", "value": per_call_us, "unit": "us",
+                      "higher_is_better": False, "steps": args.steps, "warmup": args.warmup,
+                      "config": {"workload": "%s contexts, last %d tokens of each as the chunk (%d rows), %d q / %d kv "
+                                             "heads, d %d, page %d, %s" % (s.name, args.chunk, total, s.q_heads,
+                                                                          s.kv_heads, s.head_dim, s.page_size,
+                                                                          s.dtype)},
+                      "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
+                                   "frac": tflops / peak, "peak_source": "%s bf16 GEMM" % kind},
+                      "gpu_launches": args.steps * L}), flush=True)
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
     if args.op == "rms_norm":
         return run_rms_norm(args)
+    if args.op == "prefill":
+        return run_prefill(args)
     return run_ours(args)
 
 

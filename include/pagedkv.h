@@ -259,6 +259,27 @@ int paged_decode_attention_noalloc(const pkv_pool* pool, int layer, void* out, c
                                    float scale, int num_splits, pkv_stream_t stream);
 
 /*
+ * Chunked prefill attention over the paged cache ([ENGINE] s4.3: a chunk of seq_len tokens
+ * at start_pos with the causal mask slice [start_pos : start_pos + seq_len]).  The chunk's
+ * k and v must already be in the pool (rope_apply / paged_kv_append take any number of
+ * tokens with their positions and slots).
+ *   q, out: device [total_q][q_heads][head_dim] (pool's dtype), 16-byte aligned; the rows of
+ *           sequence b are cu_q[b] .. cu_q[b+1] - 1 (cu_q: device [batch + 1] int32, cu_q[0] = 0,
+ *           cu_q[batch] = total_q, non-decreasing).
+ *   context_lens: device [batch] int32, the cached tokens of each sequence with the chunk
+ *           included (L_b >= n_b); row i of sequence b sits at position L_b - n_b + i and
+ *           attends to tokens 0 .. L_b - n_b + i.
+ *   block_tables, max_pages_per_seq, kv_heads, scale: as for paged_decode_attention;
+ *   q_heads / kv_heads in {1, 2, 4, 8}.
+ * One warp per (sequence, kv head, 16 query rows) on the tensor cores (mma.sync, fp32
+ * accumulation and softmax); no workspace.  Errors as for paged_decode_attention.
+ */
+int paged_prefill_attention(const pkv_pool* pool, int layer, void* out, const void* q, const int32_t* cu_q,
+                            int total_q, const int32_t* block_tables, int max_pages_per_seq,
+                            const int32_t* context_lens, int batch, int q_heads, int kv_heads, float scale,
+                            pkv_stream_t stream);
+
+/*
  * Zero-fill a decode workspace (cudaMemsetAsync on `stream`) before its first use with
  * paged_decode_attention.  INVALID_ARG for a NULL workspace with a non-zero size.
  */

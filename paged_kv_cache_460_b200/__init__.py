@@ -23,7 +23,7 @@ from ._lib import (PKV_BF16, PKV_DEVERR_BAD_PAGE, PKV_DEVERR_BAD_SLOT, PKV_DEVER
                    PagedKVError, lib)
 
 __all__ = [
-    "KVPool", "rope_apply", "paged_kv_append", "rope_append", "paged_decode_attention", "rms_norm", "pkv_slot_mapping",
+    "KVPool", "rope_apply", "paged_kv_append", "rope_append", "paged_decode_attention", "paged_prefill_attention", "rms_norm", "pkv_slot_mapping",
     "pkv_kv_cache_bytes", "pkv_decode_workspace_size", "pkv_decode_default_splits",
     "kv_get_device_error", "DecodeWorkspace", "PagedKVError", "PKV_F16", "PKV_BF16",
     "PKV_DEVERR_BAD_PAGE", "PKV_DEVERR_BAD_SLOT", "PKV_DEVERR_TIMEOUT",
@@ -193,6 +193,24 @@ def rope_append(pool, layer, q, k, v, positions, slot_mapping, theta=10000.0, st
     st = lib().rope_append(pool.handle, layer, _ptr(q), _ptr(k), _ptr(v), _ptr(positions), _ptr(slot_mapping),
                            k.shape[0], q.shape[1], float(theta), _stream(stream))
     _lib.check("rope_append", st)
+
+
+def paged_prefill_attention(pool, layer, out, q, cu_q, block_tables, context_lens, scale, kv_heads=None,
+                            stream=None):
+    """Chunked prefill: rows cu_q[b] .. cu_q[b+1]-1 of q [total_q, q_heads, d] are the new tokens
+    of sequence b at positions context_lens[b] - n_b ...; each attends causally over the pages."""
+    torch = _torch()
+    _need(out, "out", pool.dtype)
+    _need(q, "q", pool.dtype)
+    _need(cu_q, "cu_q", torch.int32)
+    _need(block_tables, "block_tables", torch.int32)
+    _need(context_lens, "context_lens", torch.int32)
+    total_q, Hq, _ = q.shape
+    st = lib().paged_prefill_attention(pool.handle, layer, _ptr(out), _ptr(q), _ptr(cu_q), total_q, _ptr(block_tables),
+                                       block_tables.shape[1], _ptr(context_lens), context_lens.shape[0], Hq,
+                                       pool.kv_heads if kv_heads is None else kv_heads, float(scale), _stream(stream))
+    _lib.check("paged_prefill_attention", st)
+    return out
 
 
 def rms_norm(out, x, weight, eps=1e-6, residual=None, stream=None):

@@ -14,6 +14,7 @@
 
 #include "decode_attention.cuh"
 #include "decode_attention_mma.cuh"
+#include "prefill_attention.cuh"
 #include "pagedkv.h"
 #include "pkv_internal.h"
 #include "rms_norm.cuh"
@@ -340,6 +341,83 @@ extern "C" int paged_decode_attention(const pkv_pool* pool, int layer, void* out
     prm.num_splits = num_splits;
     prm.scale_log2 = scale * 1.4426950408889634f;
     return ops.launch(prm, reinterpret_cast<cudaStream_t>(stream));
+}
+
+namespace pkv {
+namespace {
+
+template <int D, int P, int G, typename T>
+int launch_prefill(const PrefillParams& prm, int grid, cudaStream_t st)
+{
+    static int configured[kMaxDevices] = {0};
+    const int smem = PrefillShape<D>::smem_bytes(prm.batch);
+    if (smem > kMaxSmemPerCta) return PKV_ERR_UNSUPPORTED;
+    if (ensure_smem(prefill_attention_kernel<D, P, G, T>, smem, configured) != cudaSuccess) return PKV_ERR_CUDA;
+    return status_of(launch_pdl(prefill_attention_kernel<D, P, G, T>, dim3(grid), dim3(kPrefillThreads), smem, st,
+                                prm));
+}
+
+template <int D, int P, typename T>
+int prefill_group(int group, const PrefillParams& prm, int grid, cudaStream_t st)
+{
+    switch (group) {
+    case 1: return launch_prefill<D, P, 1, T>(prm, grid, st);
+    case 2: return launch_prefill<D, P, 2, T>(prm, grid, st);
+    case 4: return launch_prefill<D, P, 4, T>(prm, grid, st);
+    case 8: return launch_prefill<D, P, 8, T>(prm, grid, st);
+    default: return PKV_ERR_UNSUPPORTED;
+    }
+}
+
+template <typename T>
+int prefill_shape(int head_dim, int page_size, int group, const PrefillParams& prm, int grid, cudaStream_t st)
+{
+    if (head_dim == 128 && page_size == 16) return prefill_group<128, 16, T>(group, prm, grid, st);
+    if (head_dim == 128 && page_size == 32) return prefill_group<128, 32, T>(group, prm, grid, st);
+    if (head_dim == 64 && page_size == 16) return prefill_group<64, 16, T>(group, prm, grid, st);
+    if (head_dim == 64 && page_size == 32) return prefill_group<64, 32, T>(group, prm, grid, st);
+    return PKV_ERR_UNSUPPORTED;
+}
+
+}  // namespace
+}  // namespace pkv
+
+extern "C" int paged_prefill_attention(const pkv_pool* pool, int layer, void* out, const void* q, const int32_t* cu_q,
+                                       int total_q, const int32_t* block_tables, int max_pages_per_seq,
+                                       const int32_t* context_lens, int batch, int q_heads, int kv_heads, float scale,
+                                       pkv_stream_t stream)
+{
+    if (!pool || layer < 0 || layer >= pool->num_layers) return PKV_ERR_INVALID_ARG;
+    if (batch < 0 || total_q < 0 || q_heads <= 0 || kv_heads != pool->kv_heads || q_heads % kv_heads)
+        return PKV_ERR_INVALID_ARG;
+    if (max_pages_per_seq <= 0 || !(scale == scale)) return PKV_ERR_INVALID_ARG;
+    if (batch == 0 || total_q == 0) return PKV_OK;
+    if (!out || !q || !cu_q || !block_tables || !context_lens) return PKV_ERR_INVALID_ARG;
+    if (misaligned16(out, q)) return PKV_ERR_INVALID_ARG;
+    const int group = q_heads / kv_heads;
+    PrefillParams prm;
+    const size_t elt = 2;
+    prm.k = static_cast<const char*>(pool->k_base) + (size_t)layer * pool->layer_elems * elt;
+    prm.v = static_cast<const char*>(pool->v_base) + (size_t)layer * pool->layer_elems * elt;
+    prm.q = q;
+    prm.out = out;
+    prm.cu_q = cu_q;
+    prm.block_tables = block_tables;
+    prm.context_lens = context_lens;
+    prm.batch = batch;
+    prm.max_pages = max_pages_per_seq;
+    prm.q_heads = q_heads;
+    prm.kv_heads = kv_heads;
+    prm.num_pages = pool->num_pages;
+    prm.scale_log2 = scale * 1.4426950408889634f;
+    // work items: kv_heads * sum_b ceil(n_b * group / 16) <= kv_heads * ((total_q * group + 15 * batch) / 16 + 1)
+    const long long bound = (long long)kv_heads * (((long long)total_q * group + 15LL * batch) / 16 + 1);
+    const long long grid = (bound + kPrefillWarps - 1) / kPrefillWarps;
+    if (grid > 0x7fffffffLL) return PKV_ERR_UNSUPPORTED;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (pool->dtype == PKV_F16)
+        return prefill_shape<__half>(pool->head_dim, pool->page_size, group, prm, (int)grid, st);
+    return prefill_shape<__nv_bfloat16>(pool->head_dim, pool->page_size, group, prm, (int)grid, st);
 }
 
 extern "C" int pkv_decode_workspace_clear(void* workspace, size_t workspace_bytes, pkv_stream_t stream)

@@ -215,3 +215,14 @@ def test_rms_norm_validates(L):
     assert L.rms_norm(None, f(), None, f(), 2, 4096, 1e-6, 0, None) == _lib.PKV_ERR_INVALID_ARG
     assert L.rms_norm(f(), f(), f(0x10004), f(), 2, 4096, 1e-6, 0, None) == _lib.PKV_ERR_INVALID_ARG
     assert L.rms_norm(f(), f(), None, f(), 0, 4096, 1e-6, 0, None) == 0
+
+
+def test_prefill_validates(L):
+    h = _pool(L, num_pages=8, page_size=16, kv_heads=2, head_dim=64)
+    f = _fake_ptr
+    assert L.paged_prefill_attention(h, 0, f(), f(), f(), 4, f(), 4, f(), 1, 3, 2, 0.1, None) == _lib.PKV_ERR_INVALID_ARG
+    assert L.paged_prefill_attention(h, 0, f(), f(), f(), 4, f(), 4, f(), 1, 32, 2, 0.1, None) == _lib.PKV_ERR_UNSUPPORTED
+    assert L.paged_prefill_attention(h, 1, f(), f(), f(), 4, f(), 4, f(), 1, 2, 2, 0.1, None) == _lib.PKV_ERR_INVALID_ARG
+    assert L.paged_prefill_attention(h, 0, None, f(), f(), 4, f(), 4, f(), 1, 2, 2, 0.1, None) == _lib.PKV_ERR_INVALID_ARG
+    assert L.paged_prefill_attention(h, 0, f(), f(), f(), 0, f(), 4, f(), 1, 2, 2, 0.1, None) == 0
+    L.kv_pool_destroy(h)
