@@ -56,6 +56,9 @@ def _load():
         lib.ora_causal_attention_full.argtypes = [P, P, P, I, I, I, I, D, P]
         lib.ora_rms_norm.argtypes = [P, P, P, I, I, D, I, P, P, P]
         lib.ora_prefill_attention.argtypes = [P, P, P, P, I, P, P, I, I, I, I, I, D, I, P]
+        lib.ora_quantize_row_i8.argtypes = [P, I, I, P, P]
+        lib.ora_kv_append_i8.argtypes = [P, P, P, P, P, P, P, I, P, I, I, I, I, I]
+        lib.ora_decode_attention_i8_pairs.argtypes = [P, P, P, P, P, P, I, P, I, I, I, I, D, I, P, P, I, P]
         lib.ora_kv_cache_bytes.argtypes = [I, I, I, I64, I]
         lib.ora_kv_cache_bytes.restype = I64
         _lib = lib
@@ -223,4 +226,56 @@ def prefill_attention(q, k_pool, v_pool, block_tables, cu_q, context_lens, scale
     out = np.zeros((total, Hq, d), np.float64)
     _load().ora_prefill_attention(_p(q), _p(kp), _p(vp), _p(bt), bt.shape[1], _p(cq), _p(cl), cl.shape[0], Hq,
                                   Hkv, d, P, float(scale), _DT[dtype], _p(out))
+    return out
+
+
+# ----------------------------------------------------------------- int8 KV pages
+def quantize_rows_i8(x, dtype):
+    """x: uint16 [..., d] storage rows -> (int8 codes [..., d], float32 scales [...])."""
+    x = _c(x, np.uint16)
+    d = x.shape[-1]
+    flat = x.reshape(-1, d)
+    codes = np.empty(flat.shape, np.int8)
+    scales = np.empty(flat.shape[0], np.float32)
+    lib = _load()
+    for r in range(flat.shape[0]):
+        lib.ora_quantize_row_i8(_p(flat[r]), d, _DT[dtype], _p(codes[r]), _p(scales[r:r + 1]))
+    return codes.reshape(x.shape), scales.reshape(x.shape[:-1])
+
+
+def kv_append_i8(k_codes, v_codes, k_scales, v_scales, k, v, block_tables, positions, dtype):
+    """Quantising append into copies of one layer's int8 pool (codes [pages, Hkv, P, d],
+    scales [pages, Hkv, P])."""
+    kc = np.array(k_codes, dtype=np.int8, copy=True, order="C")
+    vc = np.array(v_codes, dtype=np.int8, copy=True, order="C")
+    ks = np.array(k_scales, dtype=np.float32, copy=True, order="C")
+    vs = np.array(v_scales, dtype=np.float32, copy=True, order="C")
+    k = _c(k, np.uint16)
+    v = _c(v, np.uint16)
+    bt = _c(block_tables, np.int32)
+    pos = _c(positions, np.int32)
+    _, kvh, P, d = kc.shape
+    _load().ora_kv_append_i8(_p(kc), _p(vc), _p(ks), _p(vs), _p(k), _p(v), _p(bt), bt.shape[1], _p(pos),
+                             pos.shape[0], kvh, P, d, _DT[dtype])
+    return kc, vc, ks, vs
+
+
+def decode_attention_i8_pairs(q, k_codes, v_codes, k_scales, v_scales, block_tables, context_lens, scale, dtype,
+                              pairs):
+    q = _c(q, np.uint16)
+    kc = _c(k_codes, np.int8)
+    vc = _c(v_codes, np.int8)
+    ks = _c(k_scales, np.float32)
+    vs = _c(v_scales, np.float32)
+    bt = _c(block_tables, np.int32)
+    cl = _c(context_lens, np.int32)
+    _, Hq, d = q.shape
+    _, Hkv, P, _ = kc.shape
+    pairs = np.asarray(pairs, dtype=np.int64).reshape(-1, 2)
+    pb = _c(pairs[:, 0], np.int32)
+    ph = _c(pairs[:, 1], np.int32)
+    out = np.empty((pairs.shape[0], d), np.float64)
+    _load().ora_decode_attention_i8_pairs(_p(q), _p(kc), _p(vc), _p(ks), _p(vs), _p(bt), bt.shape[1], _p(cl), Hq,
+                                          Hkv, d, P, float(scale), _DT[dtype], _p(pb), _p(ph), pairs.shape[0],
+                                          _p(out))
     return out

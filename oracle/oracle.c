@@ -526,3 +526,107 @@ void ora_prefill_attention(const uint16_t* q, const uint16_t* k_pool, const uint
         free(s);
     }
 }
+
+/* ------------------------------------------------------------------------- */
+/* int8 KV pages  [ENGINE] s3.4 (compression: store the cache in a smaller type) */
+/* ------------------------------------------------------------------------- */
+
+/*
+ * Symmetric int8 quantisation of one head row of k or v (head_dim storage values):
+ * amax = max |x_i|; codes q_i = round_half_even(x_i * (127 / amax)) in [-127, 127];
+ * scale = amax / 127, so x_i ~ q_i * scale.  An all-zero row gets scale 0 and codes 0.
+ * The decisions are taken in fp32 (each operation correctly rounded), the kernel's
+ * precision, so that both sides produce the same codes.
+ */
+void ora_quantize_row_i8(const uint16_t* x, int head_dim, int dtype, int8_t* codes, float* scale_out)
+{
+    float amax = 0.0f;
+    for (int i = 0; i < head_dim; ++i) {
+        float a = (float)fabs(dec(x[i], dtype));
+        if (a > amax) amax = a;
+    }
+    if (amax == 0.0f) {
+        for (int i = 0; i < head_dim; ++i) codes[i] = 0;
+        *scale_out = 0.0f;
+        return;
+    }
+    volatile float inv = 127.0f / amax;
+    for (int i = 0; i < head_dim; ++i) {
+        volatile float prod = (float)dec(x[i], dtype) * inv;
+        float r = rintf(prod);
+        if (r > 127.0f) r = 127.0f;
+        if (r < -127.0f) r = -127.0f;
+        codes[i] = (int8_t)r;
+    }
+    volatile float sc = amax / 127.0f;
+    *scale_out = sc;
+}
+
+/*
+ * Cache update into an int8 pool: the token of row b (k, v: [n][kv_heads][head_dim]
+ * storage values) goes to position positions[b] of sequence b; each head row is quantised
+ * with ora_quantize_row_i8.  Pools: codes [num_pages][kv_heads][page_size][head_dim],
+ * scales [num_pages][kv_heads][page_size].
+ */
+void ora_kv_append_i8(int8_t* k_codes, int8_t* v_codes, float* k_scales, float* v_scales, const uint16_t* k,
+                      const uint16_t* v, const int32_t* block_tables, int max_pages_per_seq, const int32_t* positions,
+                      int n, int kv_heads, int page_size, int head_dim, int dtype)
+{
+    for (int b = 0; b < n; ++b) {
+        int pos = positions[b];
+        if (pos < 0) continue;
+        int64_t page = block_tables[(int64_t)b * max_pages_per_seq + pos / page_size];
+        int row = pos % page_size;
+        for (int h = 0; h < kv_heads; ++h) {
+            int64_t dst = (page * kv_heads + h) * page_size + row;
+            int64_t src = ((int64_t)b * kv_heads + h) * head_dim;
+            ora_quantize_row_i8(k + src, head_dim, dtype, k_codes + dst * head_dim, k_scales + dst);
+            ora_quantize_row_i8(v + src, head_dim, dtype, v_codes + dst * head_dim, v_scales + dst);
+        }
+    }
+}
+
+/*
+ * Decode attention over an int8 pool: token t's key is k_code * k_scale (and likewise v),
+ * taken exactly in double; otherwise as ora_decode_attention_pairs.  q: storage values.
+ */
+void ora_decode_attention_i8_pairs(const uint16_t* q, const int8_t* k_codes, const int8_t* v_codes,
+                                   const float* k_scales, const float* v_scales, const int32_t* block_tables,
+                                   int max_pages_per_seq, const int32_t* context_lens, int q_heads, int kv_heads,
+                                   int head_dim, int page_size, double scale, int dtype, const int32_t* pair_b,
+                                   const int32_t* pair_h, int n_pairs, double* out)
+{
+    int group = q_heads / kv_heads;
+    for (int p = 0; p < n_pairs; ++p) {
+        int b = pair_b[p], h = pair_h[p], g = h / group;
+        int len = context_lens[b];
+        double* o = out + (int64_t)p * head_dim;
+        for (int i = 0; i < head_dim; ++i) o[i] = 0.0;
+        if (len <= 0) continue;
+        const uint16_t* qh = q + ((int64_t)b * q_heads + h) * head_dim;
+        double* s = (double*)malloc(sizeof(double) * (size_t)len);
+        double mx = -INFINITY;
+        for (int t = 0; t < len; ++t) {
+            int64_t row = (block_tables[(int64_t)b * max_pages_per_seq + t / page_size] * kv_heads + g) * page_size +
+                          t % page_size;
+            double dot = 0.0;
+            for (int i = 0; i < head_dim; ++i)
+                dot += dec(qh[i], dtype) * ((double)k_codes[row * head_dim + i] * (double)k_scales[row]);
+            s[t] = scale * dot;
+            if (s[t] > mx) mx = s[t];
+        }
+        double z = 0.0;
+        for (int t = 0; t < len; ++t) {
+            s[t] = exp(s[t] - mx);
+            z += s[t];
+        }
+        for (int t = 0; t < len; ++t) {
+            int64_t row = (block_tables[(int64_t)b * max_pages_per_seq + t / page_size] * kv_heads + g) * page_size +
+                          t % page_size;
+            for (int i = 0; i < head_dim; ++i)
+                o[i] += s[t] * ((double)v_codes[row * head_dim + i] * (double)v_scales[row]);
+        }
+        for (int i = 0; i < head_dim; ++i) o[i] /= z;
+        free(s);
+    }
+}

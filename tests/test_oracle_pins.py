@@ -449,3 +449,68 @@ def test_prefill_matches_brute_force():
                 ref = brute.attention_one(qv, [Kl[b][t][h // 2] for t in range(pos + 1)],
                                           [Vl[b][t][h // 2] for t in range(pos + 1)], scale)
                 assert np.allclose(pre[lo + i, h], ref, rtol=1e-12, atol=1e-14)
+
+
+# ------------------------------------------------------------------ int8 KV pages
+def test_int8_codes_match_a_float32_reference():
+    """The quantiser's fp32 steps, redone with numpy float32 (each op rounded to nearest)."""
+    r = np.random.Generator(np.random.PCG64(90))
+    for dtype in ("f16", "bf16"):
+        x = synth.round_f32(r.standard_normal((50, 128), dtype=np.float32) * 2, dtype)
+        codes, scales = oracle.quantize_rows_i8(x, dtype)
+        xf = oracle.decode(x, dtype).astype(np.float32)
+        amax = np.abs(xf).max(axis=1)
+        inv = (np.float32(127.0) / amax).astype(np.float32)
+        ref = np.clip(np.rint((xf * inv[:, None]).astype(np.float32)), -127, 127).astype(np.int8)
+        assert np.array_equal(codes, ref)
+        assert np.array_equal(scales, (amax / np.float32(127.0)).astype(np.float32))
+        # the largest element maps to +-127 and every element is within half a step, plus the
+        # fp32 roundings of the scale and of x * inv (each 2^-24 relative, times |code| <= 127)
+        assert np.all(np.abs(codes).max(axis=1) == 127)
+        err = np.abs(codes.astype(np.float64) * scales[:, None] - oracle.decode(x, dtype))
+        assert np.all(err <= scales[:, None] * (0.5 + 2 * 127 * 2.0 ** -24))
+
+
+def test_int8_zero_row_and_attention_on_dequantised_values():
+    codes, scales = oracle.quantize_rows_i8(np.zeros((1, 16), np.uint16), "f16")
+    assert np.all(codes == 0) and scales[0] == 0
+    sp, q, kp, vp, _, _, scale = _logical_case(91, 2, 4, 2, 16, 4, [19, 6])
+    kc, ks = oracle.quantize_rows_i8(kp, "f16")
+    vc, vs = oracle.quantize_rows_i8(vp, "f16")
+    cl = np.array([19, 6], np.int32)
+    pairs = [(b, h) for b in range(2) for h in range(4)]
+    got = oracle.decode_attention_i8_pairs(q, kc, vc, ks, vs, sp.block_tables, cl, scale, "f16", pairs)
+    # brute force on the dequantised cache (exact products code * scale in double)
+    kd = kc.astype(np.float64) * ks[..., None].astype(np.float64)
+    vd = vc.astype(np.float64) * vs[..., None].astype(np.float64)
+    for n, (b, h) in enumerate(pairs):
+        keys, vals = [], []
+        for t in range(cl[b]):
+            page = sp.block_tables[b][t // 4]
+            keys.append(list(kd[page, h // 2, t % 4]))
+            vals.append(list(vd[page, h // 2, t % 4]))
+        ref = brute.attention_one(list(oracle.decode(q[b, h], "f16")), keys, vals, scale)
+        assert np.allclose(got[n], ref, rtol=1e-12, atol=1e-14)
+
+
+def test_int8_append_lands_where_the_fp16_append_does():
+    """Quantising append == plain append (pinned above) followed by row-wise quantisation of
+    the written rows; untouched rows keep their codes and scales."""
+    r = np.random.Generator(np.random.PCG64(92))
+    pages, kvh, P, d, n = 6, 2, 4, 16, 3
+    kp = synth.round_f32(r.standard_normal((pages, kvh, P, d), dtype=np.float32), "f16")
+    vp = synth.round_f32(r.standard_normal((pages, kvh, P, d), dtype=np.float32), "f16")
+    k = synth.round_f32(r.standard_normal((n, kvh, d), dtype=np.float32), "f16")
+    v = synth.round_f32(r.standard_normal((n, kvh, d), dtype=np.float32), "f16")
+    bt = np.array([[5, 2], [0, 1], [3, 4]], np.int32)
+    pos = np.array([6, 0, -1], np.int32)
+    kc, ks = oracle.quantize_rows_i8(kp, "f16")
+    vc, vs = oracle.quantize_rows_i8(vp, "f16")
+    kc2, vc2, ks2, vs2 = oracle.kv_append_i8(kc, vc, ks, vs, k, v, bt, pos, "f16")
+    kp2, vp2 = oracle.kv_append(kp, vp, k, v, bt, pos)
+    kc_ref, ks_ref = oracle.quantize_rows_i8(kp2, "f16")
+    vc_ref, vs_ref = oracle.quantize_rows_i8(vp2, "f16")
+    assert np.array_equal(kc2, kc_ref) and np.array_equal(ks2, ks_ref)
+    assert np.array_equal(vc2, vc_ref) and np.array_equal(vs2, vs_ref)
+    assert not np.array_equal(kc2, kc)                  # something was written
+    assert np.array_equal(kc2[2, :, 2], kc_ref[2, :, 2])  # page 2 row 2 (token 6 of seq 0)
