@@ -56,6 +56,9 @@ def parse_args(argv=None):
     ap.add_argument("--op", choices=("decode", "rms_norm", "prefill"), default="decode",
                     help="decode: the decode step (default); rms_norm / prefill: that kernel alone")
     ap.add_argument("--chunk", type=int, default=512, help="prefill: new tokens per sequence")
+    ap.add_argument("--kv", choices=("native", "int8"), default="native",
+                    help="decode: page storage -- the workload's 16-bit type, or int8 codes with a fp32 "
+                         "scale per (token, head) row")
     return ap.parse_args(argv)
 
 
@@ -78,10 +81,19 @@ def kernel_source_digest():
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload):
+def kv_bytes_per_layer(s, kv):
+    """Algorithmic KV bytes one attention call reads: every cached token's K and V row of
+    every kv head -- head_dim elements, or head_dim int8 codes plus a 4-byte scale."""
+    if kv == "int8":
+        return int(s.context_lens.astype(np.int64).sum()) * s.kv_heads * 2 * (s.head_dim + 4)
+    return s.kv_bytes_read()
+
+
+def profiled_traffic(workload, kv="native"):
     """DRAM bytes per attention launch from the committed ncu summary, if it was taken
     on the kernel source as it is now (else None)."""
-    path = os.path.join(ROOT, "profiles", "decode_attention_%s.md" % workload)
+    name = workload if kv == "native" else "int8_" + workload
+    path = os.path.join(ROOT, "profiles", "decode_attention_%s.md" % name)
     if not os.path.exists(path):
         return None
     vals = {}
@@ -181,7 +193,7 @@ def max_over_ranks(value, world, device=None):
 
 
 # ------------------------------------------------------------------ CPU oracle timing
-def time_oracle_sample(s, seconds, seed=0, max_pairs=None):
+def time_oracle_sample(s, seconds, seed=0, max_pairs=None, kv="native"):
     """Time the fp64 oracle (single thread) on (b, kv head) pairs of the workload, each
     pair a standalone mini pool, until ~`seconds` have passed.  Returns
     (GB/s of algorithmic KV bytes, description)."""
@@ -199,14 +211,23 @@ def time_oracle_sample(s, seconds, seed=0, max_pairs=None):
         table = np.arange(kmini.shape[0], dtype=np.int32)[None, :]
         cl = np.array([s.context_lens[b]], np.int32)
         pairs = [(0, h) for h in range(G)]
+        if kv == "int8":
+            codes = r.integers(-127, 128, size=(2,) + kmini.shape, dtype=np.int8)
+            sc = (r.uniform(1.5, 2.5, size=(2,) + kmini.shape[:-1]) / 127.0).astype(np.float32)
+            t0 = time.perf_counter()
+            oracle.decode_attention_i8_pairs(q, codes[0], codes[1], sc[0], sc[1], table, cl, scale, s.dtype, pairs)
+            total_t += time.perf_counter() - t0
+            total_bytes += int(cl[0]) * 2 * (s.head_dim + 4)
+            n += 1
+            continue
         t0 = time.perf_counter()
         oracle.decode_attention_pairs(q, kmini, vmini, table, cl, scale, s.dtype, pairs)
         total_t += time.perf_counter() - t0
         total_bytes += int(cl[0]) * 2 * s.head_dim * s.elt_bytes
         n += 1
     gbs = total_bytes / total_t / 1e9
-    return gbs, "%d random (sequence, kv head) pairs of one %s layer (%d query heads each), %.1f s" % (
-        n, s.name, G, total_t)
+    return gbs, "%d random (sequence, kv head) pairs of one %s layer (%d query heads each%s), %.1f s" % (
+        n, s.name, G, ", int8 pages" if kv == "int8" else "", total_t)
 
 
 def run_reference(args):
@@ -216,12 +237,12 @@ def run_reference(args):
     s = synth.spec(args.workload, num_layers=args.layers)
     per_step = max(0.02, min(2.0, 150.0 / max(1, args.steps + args.warmup)))
     for i in range(args.warmup):
-        time_oracle_sample(s, per_step, seed=i)
+        time_oracle_sample(s, per_step, seed=i, kv=args.kv)
     vals, t_all = [], 0.0
     import oracle  # noqa: F401
     for i in range(args.steps):
         t0 = time.perf_counter()
-        g, _ = time_oracle_sample(s, per_step, seed=1000 + i)
+        g, _ = time_oracle_sample(s, per_step, seed=1000 + i, kv=args.kv)
         t_all += time.perf_counter() - t0
         vals.append(g)
     value = float(np.mean(vals))
@@ -240,16 +261,19 @@ def run_reference(args):
 
 
 def workload_config(s, args):
+    kv = getattr(args, "kv", "native")
+    per_layer = kv_bytes_per_layer(s, kv)
+    pages = s.dtype if kv == "native" else "int8 pages (fp32 row scales), %s activations" % s.dtype
     return {"workload": "%s: batch %d, %d layers, %d q / %d kv heads, head_dim %d, page %d, %s, context %d..%d"
-                        % (s.name, s.batch, s.num_layers, s.q_heads, s.kv_heads, s.head_dim, s.page_size, s.dtype,
+                        % (s.name, s.batch, s.num_layers, s.q_heads, s.kv_heads, s.head_dim, s.page_size, pages,
                            int(s.context_lens.min()), int(s.context_lens.max())),
             "batch": s.batch, "layers": s.num_layers, "q_heads": s.q_heads, "kv_heads": s.kv_heads,
-            "head_dim": s.head_dim, "page_size": s.page_size,
-            "kv_bytes_per_layer": s.kv_bytes_read(), "kv_bytes_per_step": s.kv_bytes_read() * s.num_layers,
+            "head_dim": s.head_dim, "page_size": s.page_size, "kv_storage": "int8" if kv == "int8" else s.dtype,
+            "kv_bytes_per_layer": per_layer, "kv_bytes_per_step": per_layer * s.num_layers,
             "parallelism": "replicas" if args.gpus > 1 else "single",
             "l2": "inputs larger than L2: each step streams %d layer caches (%.2f GB of K+V)"
-                  % (s.num_layers, s.kv_bytes_read() * s.num_layers / 1e9)
-                  if s.kv_bytes_read() * s.num_layers > 2 * 126e6
+                  % (s.num_layers, per_layer * s.num_layers / 1e9)
+                  if per_layer * s.num_layers > 2 * 126e6
                   else "L2 flushed (256 MB memset) before every timed step, outside the timed intervals"}
 
 
@@ -269,8 +293,13 @@ def run_ours(args):
 
     s = synth.spec(args.workload, num_layers=args.layers)
     L = s.num_layers
-    kp, vp = synth.pool_values_torch(s, dev)
-    pool = pkv.KVPool(kp, vp)
+    if args.kv == "int8":
+        kc, vc, ksc, vsc = synth.pool_values_i8_torch(s, dev)
+        pool = pkv.KVPool(kc, vc, ksc, vsc, dtype=torch.float16 if s.dtype == "f16" else torch.bfloat16)
+    else:
+        kp, vp = synth.pool_values_torch(s, dev)
+        pool = pkv.KVPool(kp, vp)
+    layer_bytes = kv_bytes_per_layer(s, args.kv)
     qs, ks, vs = synth.step_values_torch(s, INPUT_SETS, dev)
     steps = []
     for j in range(INPUT_SETS):
@@ -281,7 +310,7 @@ def run_ours(args):
         st.v.copy_(vs[j])
         steps.append(st)
     del qs, ks, vs
-    small = s.kv_bytes_read() * L < 2 * 126e6
+    small = layer_bytes * L < 2 * 126e6
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev) if small else None
 
     def sync_all():
@@ -372,7 +401,7 @@ def run_ours(args):
         saved, args.steps = args.steps, n_e2e
         ms_e2e = max_over_ranks(timed(e2e_step), world, dev)
         args.steps = saved
-        e2e = {"value": throughput(world, s.kv_bytes_read() * L, n_e2e, ms_e2e), "unit": UNIT,
+        e2e = {"value": throughput(world, layer_bytes * L, n_e2e, ms_e2e), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e / n_e2e}
 
     err = pkv.kv_get_device_error()
@@ -381,12 +410,12 @@ def run_ours(args):
 
     if rank == 0:
         per_step_ms = ms_total / args.steps
-        value = throughput(world, s.kv_bytes_read() * L, args.steps, ms_total)
+        value = throughput(world, layer_bytes * L, args.steps, ms_total)
         peak, peak_kind = measured_peaks()
-        achieved = s.kv_bytes_read() / (attn_ms_mean * 1e-3) / 1e9
+        achieved = layer_bytes / (attn_ms_mean * 1e-3) / 1e9
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
-            gbs, desc = time_oracle_sample(s, args.cpu_seconds)
+            gbs, desc = time_oracle_sample(s, args.cpu_seconds, kv=args.kv)
             cpu = {"value": gbs, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc}
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -396,7 +425,7 @@ def run_ours(args):
             "attention_us_per_layer": 1000.0 * attn_ms_mean,
             "pct_of_8tbs": 100.0 * value / NOMINAL_HBM_GBS,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": profiled_traffic(args.workload),
+                         "frac": achieved / peak, "traffic": profiled_traffic(args.workload, args.kv),
                          "peak_source": "%s copy bandwidth" % peak_kind,
                          "kernel": "paged_decode_attention (one kernel per call)",
                          "frac_of_8tbs": achieved / NOMINAL_HBM_GBS},

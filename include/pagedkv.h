@@ -56,6 +56,7 @@ extern "C" {
 /* element types */
 #define PKV_F16 0
 #define PKV_BF16 1
+#define PKV_I8 2     /* KV storage only: int8 codes with one fp32 scale per (token, head) row */
 
 /* device error word bits (kv_get_device_error) */
 #define PKV_DEVERR_BAD_PAGE 0x1u     /* block-table entry outside [0, num_pages) */
@@ -87,6 +88,31 @@ const char* pkv_status_string(int status);
 int kv_pool_create(int num_layers, int num_pages, int page_size, int kv_heads, int head_dim,
                    int dtype, void* k_base, void* v_base, pkv_pool** out);
 
+/*
+ * Describe a preallocated int8 paged KV pool ([ENGINE] s3.4: the KV strategy pairs paging
+ * with compression of the cached values).  Each cached (token, kv head) row x of head_dim
+ * values is held as int8 codes c and one fp32 scale s with x ~ c * s:
+ *   s = amax / 127 and c_i = round_half_even(x_i * (127 / amax)) clamped to [-127, 127],
+ *   amax = max_i |x_i|, every step one correctly rounded fp32 operation (amax = 0 gives
+ *   s = 0 and c = 0).  The scale is per row, not per page, because the cache grows one
+ *   token at a time and a page's later tokens may exceed the range of its earlier ones.
+ *   k_codes, v_codes: device int8 [num_layers][num_pages][kv_heads][page_size][head_dim];
+ *   k_scales, v_scales: device fp32 [num_layers][num_pages][kv_heads][page_size];
+ *   all four 16-byte aligned and caller-owned, as for kv_pool_create.
+ *   dtype: PKV_F16 or PKV_BF16, the type of q, k, v and the output of the calls on this pool.
+ * paged_kv_append and rope_append quantise the new rows as they write them;
+ * paged_decode_attention reads k = c * s, v = c * s (every q_heads / kv_heads in {1, 2, 4, 8}
+ * on the CUDA cores); paged_prefill_attention returns UNSUPPORTED on such a pool.
+ * Errors as for kv_pool_create.
+ */
+int kv_pool_create_i8(int num_layers, int num_pages, int page_size, int kv_heads, int head_dim,
+                      int dtype, void* k_codes, void* v_codes, void* k_scales, void* v_scales,
+                      pkv_pool** out);
+
+/* Storage type of the pool's pages: PKV_I8 for kv_pool_create_i8 pools, else the element
+ * type.  INVALID_ARG for a NULL pool or output. */
+int kv_pool_storage(const pkv_pool* pool, int* storage_out);
+
 /* Free the host descriptor (not the caller's device arrays).  NULL is ignored. */
 void kv_pool_destroy(pkv_pool* pool);
 
@@ -112,7 +138,9 @@ int kv_pool_info(const pkv_pool* pool, int* num_layers, int* num_pages, int* pag
 
 /*
  * KV-cache bytes for `tokens` tokens ([ENGINE] s3.4):
- * layers x 2 (K and V) x kv_heads x head_dim x tokens x element bytes.  -1 on bad input.
+ * layers x 2 (K and V) x kv_heads x head_dim x tokens x element bytes; for PKV_I8,
+ * layers x 2 x kv_heads x tokens x (head_dim + 4) (codes and the row's fp32 scale).
+ * -1 on bad input.
  */
 int64_t pkv_kv_cache_bytes(int num_layers, int kv_heads, int head_dim, int64_t tokens, int dtype);
 
@@ -151,6 +179,7 @@ int rope_apply(void* q, void* k, const int32_t* positions, int n_tokens, int q_h
  *   k, v: device [n_tokens][kv_heads][head_dim] (pool's dtype), 16-byte aligned;
  *   slot_mapping: device [n_tokens] int64 (negative = skip the row).
  * A slot >= num_pages * page_size is skipped and sets PKV_DEVERR_BAD_SLOT.
+ * On an int8 pool (kv_pool_create_i8) each written row is quantised instead of copied.
  */
 int paged_kv_append(const pkv_pool* pool, int layer, const void* k, const void* v,
                     const int64_t* slot_mapping, int n_tokens, pkv_stream_t stream);
@@ -162,7 +191,8 @@ int paged_kv_append(const pkv_pool* pool, int layer, const void* k, const void* 
  * and the rotated k and v [n_tokens][kv_heads][head_dim] are copied bit for bit into the
  * pool slots slot_mapping[i] of `layer` (negative = skip; past the pool = skip and set
  * PKV_DEVERR_BAD_SLOT).  kv_heads, head_dim and the element type are the pool's.  Results
- * are identical to the two separate calls.  q, k, v 16-byte aligned.
+ * are identical to the two separate calls (on an int8 pool the rows are quantised as in
+ * paged_kv_append).  q, k, v 16-byte aligned.
  */
 int rope_append(const pkv_pool* pool, int layer, void* q, void* k, const void* v,
                 const int32_t* positions, const int64_t* slot_mapping, int n_tokens, int q_heads,

@@ -19,13 +19,13 @@ import ctypes
 import numpy as np
 
 from . import _lib
-from ._lib import (PKV_BF16, PKV_DEVERR_BAD_PAGE, PKV_DEVERR_BAD_SLOT, PKV_DEVERR_TIMEOUT, PKV_F16,
+from ._lib import (PKV_BF16, PKV_DEVERR_BAD_PAGE, PKV_DEVERR_BAD_SLOT, PKV_DEVERR_TIMEOUT, PKV_F16, PKV_I8,
                    PagedKVError, lib)
 
 __all__ = [
     "KVPool", "rope_apply", "paged_kv_append", "rope_append", "paged_decode_attention", "paged_prefill_attention", "rms_norm", "pkv_slot_mapping",
     "pkv_kv_cache_bytes", "pkv_decode_workspace_size", "pkv_decode_default_splits",
-    "kv_get_device_error", "DecodeWorkspace", "PagedKVError", "PKV_F16", "PKV_BF16",
+    "kv_get_device_error", "DecodeWorkspace", "PagedKVError", "PKV_F16", "PKV_BF16", "PKV_I8",
     "PKV_DEVERR_BAD_PAGE", "PKV_DEVERR_BAD_SLOT", "PKV_DEVERR_TIMEOUT",
 ]
 
@@ -71,23 +71,41 @@ class KVPool:
     """A paged KV pool over caller-owned device tensors.
 
     k_cache, v_cache: [num_layers, num_pages, kv_heads, page_size, head_dim], fp16 or bf16.
+    For int8 pages pass int8 code tensors of that shape, fp32 scales k_scales, v_scales
+    [num_layers, num_pages, kv_heads, page_size] and the activation dtype (fp16 or bf16)
+    of q, k, v and the outputs.
     The host free list hands page ids out with ``alloc`` and takes them back with ``free``.
     """
 
-    def __init__(self, k_cache, v_cache):
+    def __init__(self, k_cache, v_cache, k_scales=None, v_scales=None, dtype=None):
         torch = _torch()
         if k_cache.shape != v_cache.shape or k_cache.dtype != v_cache.dtype or k_cache.dim() != 5:
             raise ValueError("k_cache and v_cache must both be [layers, pages, kv_heads, page, head_dim]")
         _need(k_cache, "k_cache", cuda=False)
         _need(v_cache, "v_cache", cuda=False)
         self.k_cache, self.v_cache = k_cache, v_cache
+        self.k_scales, self.v_scales = k_scales, v_scales
         L, N, H, P, D = k_cache.shape
         self.num_layers, self.num_pages, self.kv_heads, self.page_size, self.head_dim = L, N, H, P, D
-        self.dtype = k_cache.dtype
         h = ctypes.c_void_p()
-        st = lib().kv_pool_create(L, N, P, H, D, dtype_code(k_cache.dtype), _ptr(k_cache), _ptr(v_cache),
-                                  ctypes.byref(h))
-        _lib.check("kv_pool_create", st)
+        if k_cache.dtype == torch.int8:
+            if k_scales is None or v_scales is None or dtype is None:
+                raise ValueError("int8 pages need k_scales, v_scales and the activation dtype")
+            for t, n in ((k_scales, "k_scales"), (v_scales, "v_scales")):
+                _need(t, n, torch.float32, cuda=False)
+                if tuple(t.shape) != (L, N, H, P):
+                    raise ValueError("%s must be [layers, pages, kv_heads, page]" % n)
+            self.dtype = dtype
+            self.storage = PKV_I8
+            st = lib().kv_pool_create_i8(L, N, P, H, D, dtype_code(dtype), _ptr(k_cache), _ptr(v_cache),
+                                         _ptr(k_scales), _ptr(v_scales), ctypes.byref(h))
+            _lib.check("kv_pool_create_i8", st)
+        else:
+            self.dtype = k_cache.dtype
+            self.storage = dtype_code(k_cache.dtype)
+            st = lib().kv_pool_create(L, N, P, H, D, dtype_code(k_cache.dtype), _ptr(k_cache), _ptr(v_cache),
+                                      ctypes.byref(h))
+            _lib.check("kv_pool_create", st)
         self.handle = h
         del torch
 
@@ -232,10 +250,12 @@ class DecodeWorkspace:
     Allocated zero-filled, as the kernel's per-partition counters require; every call
     leaves it ready for the next one."""
 
-    def __init__(self, batch, q_heads, kv_heads, head_dim, page_size, dtype, num_splits=0, device=None):
+    def __init__(self, batch, q_heads, kv_heads, head_dim, page_size, dtype, num_splits=0, device=None,
+                 storage=None):
         torch = _torch()
         if num_splits == 0:
-            num_splits = pkv_decode_default_splits(q_heads, kv_heads, head_dim, page_size, dtype_code(dtype))
+            code = dtype_code(dtype) if storage is None else storage
+            num_splits = pkv_decode_default_splits(q_heads, kv_heads, head_dim, page_size, code)
         self.num_splits = num_splits
         self.nbytes = pkv_decode_workspace_size(batch, q_heads, kv_heads, head_dim, num_splits)
         self.buffer = torch.zeros(self.nbytes, dtype=torch.uint8, device=device or "cuda")
@@ -254,7 +274,7 @@ def paged_decode_attention(pool, layer, out, q, block_tables, context_lens, scal
         kv_heads = pool.kv_heads
     if workspace is None:
         workspace = DecodeWorkspace(B, Hq, kv_heads, pool.head_dim, pool.page_size, pool.dtype, num_splits,
-                                    device=q.device)
+                                    device=q.device, storage=pool.storage)
     if num_splits == 0:
         num_splits = workspace.num_splits
     st = lib().paged_decode_attention(pool.handle, layer, _ptr(out), _ptr(q), _ptr(block_tables),

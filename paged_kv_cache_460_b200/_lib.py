@@ -16,6 +16,7 @@ PKV_ERR_CUDA = 3
 PKV_ERR_NO_SPACE = 4
 PKV_F16 = 0
 PKV_BF16 = 1
+PKV_I8 = 2
 PKV_DEVERR_BAD_PAGE = 0x1
 PKV_DEVERR_BAD_SLOT = 0x2
 PKV_DEVERR_TIMEOUT = 0x4
@@ -28,6 +29,8 @@ _P, _I, _I64, _D, _F, _SZ = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctyp
 SIGNATURES = {
     "pkv_status_string": (ctypes.c_char_p, [_I]),
     "kv_pool_create": (_I, [_I, _I, _I, _I, _I, _I, _P, _P, ctypes.POINTER(_P)]),
+    "kv_pool_create_i8": (_I, [_I, _I, _I, _I, _I, _I, _P, _P, _P, _P, ctypes.POINTER(_P)]),
+    "kv_pool_storage": (_I, [_P, ctypes.POINTER(_I)]),
     "kv_pool_destroy": (None, [_P]),
     "kv_pool_alloc": (_I, [_P, _I, _P]),
     "kv_pool_free": (_I, [_P, _I, _P]),

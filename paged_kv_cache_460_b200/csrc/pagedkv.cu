@@ -67,21 +67,21 @@ struct DecodeOps {
 };
 
 // One query head per kv head: the CUDA-core kernel; 2 to 8 heads sharing a kv head: the
-// tensor-core kernel.
-template <int D, int P, int G, typename T, bool kMma = (G > 1)>
+// tensor-core kernel.  Int8 pages (I8): the CUDA-core kernel for every group size.
+template <int D, int P, int G, typename T, bool I8, bool kMma = (G > 1 && !I8)>
 struct DecodeKernel {
-    static constexpr auto fn = decode_pass1_kernel<D, P, G, T>;
-    static int smem(int batch) { return DecodeShape<D, P, G>::smem_bytes(batch); }
+    static constexpr auto fn = decode_pass1_kernel<D, P, G, T, I8>;
+    static int smem(int batch) { return DecodeShape<D, P, G, I8>::smem_bytes(batch); }
 };
 template <int D, int P, int G, typename T>
-struct DecodeKernel<D, P, G, T, true> {
+struct DecodeKernel<D, P, G, T, false, true> {
     static constexpr auto fn = decode_pass1_mma_kernel<D, P, G, T>;
     static int smem(int batch) { return MmaShape<D, G>::smem_bytes(batch); }
 };
 
-template <int D, int P, int G, typename T>
+template <int D, int P, int G, typename T, bool I8>
 struct DecodeImpl {
-    using K = DecodeKernel<D, P, G, T>;
+    using K = DecodeKernel<D, P, G, T, I8>;
     static int configured[kMaxDevices];
 
     static int launch(const DecodeParams& prm, cudaStream_t st)
@@ -110,35 +110,42 @@ struct DecodeImpl {
     }
 };
 
-template <int D, int P, int G, typename T>
-int DecodeImpl<D, P, G, T>::configured[kMaxDevices] = {0};
+template <int D, int P, int G, typename T, bool I8>
+int DecodeImpl<D, P, G, T, I8>::configured[kMaxDevices] = {0};
 
-template <int D, int P, typename T>
+template <int D, int P, typename T, bool I8>
 bool pick_group(int group, DecodeOps& ops)
 {
     switch (group) {
-    case 1: ops = {DecodeImpl<D, P, 1, T>::launch, DecodeImpl<D, P, 1, T>::splits, 1}; return true;
-    case 2: ops = {DecodeImpl<D, P, 2, T>::launch, DecodeImpl<D, P, 2, T>::splits, 2}; return true;
-    case 4: ops = {DecodeImpl<D, P, 4, T>::launch, DecodeImpl<D, P, 4, T>::splits, 4}; return true;
-    case 8: ops = {DecodeImpl<D, P, 8, T>::launch, DecodeImpl<D, P, 8, T>::splits, 8}; return true;
+    case 1: ops = {DecodeImpl<D, P, 1, T, I8>::launch, DecodeImpl<D, P, 1, T, I8>::splits, 1}; return true;
+    case 2: ops = {DecodeImpl<D, P, 2, T, I8>::launch, DecodeImpl<D, P, 2, T, I8>::splits, 2}; return true;
+    case 4: ops = {DecodeImpl<D, P, 4, T, I8>::launch, DecodeImpl<D, P, 4, T, I8>::splits, 4}; return true;
+    case 8: ops = {DecodeImpl<D, P, 8, T, I8>::launch, DecodeImpl<D, P, 8, T, I8>::splits, 8}; return true;
     default: return false;
     }
 }
 
-template <typename T>
+template <typename T, bool I8>
 bool pick_shape(int head_dim, int page_size, int group, DecodeOps& ops)
 {
-    if (head_dim == 128 && page_size == 16) return pick_group<128, 16, T>(group, ops);
-    if (head_dim == 128 && page_size == 32) return pick_group<128, 32, T>(group, ops);
-    if (head_dim == 64 && page_size == 16) return pick_group<64, 16, T>(group, ops);
-    if (head_dim == 64 && page_size == 32) return pick_group<64, 32, T>(group, ops);
+    if (head_dim == 128 && page_size == 16) return pick_group<128, 16, T, I8>(group, ops);
+    if (head_dim == 128 && page_size == 32) return pick_group<128, 32, T, I8>(group, ops);
+    if (head_dim == 64 && page_size == 16) return pick_group<64, 16, T, I8>(group, ops);
+    if (head_dim == 64 && page_size == 32) return pick_group<64, 32, T, I8>(group, ops);
     return false;
 }
 
-bool pick_decode(int head_dim, int page_size, int group, int dtype, DecodeOps& ops)
+// dtype: the type of q and the output; storage: the pages' type (dtype or PKV_I8)
+bool pick_decode(int head_dim, int page_size, int group, int dtype, int storage, DecodeOps& ops)
 {
-    if (dtype == PKV_F16) return pick_shape<__half>(head_dim, page_size, group, ops);
-    if (dtype == PKV_BF16) return pick_shape<__nv_bfloat16>(head_dim, page_size, group, ops);
+    const bool i8 = storage == PKV_I8;
+    if (!i8 && storage != dtype) return false;
+    if (dtype == PKV_F16)
+        return i8 ? pick_shape<__half, true>(head_dim, page_size, group, ops)
+                  : pick_shape<__half, false>(head_dim, page_size, group, ops);
+    if (dtype == PKV_BF16)
+        return i8 ? pick_shape<__nv_bfloat16, true>(head_dim, page_size, group, ops)
+                  : pick_shape<__nv_bfloat16, false>(head_dim, page_size, group, ops);
     return false;
 }
 
@@ -186,9 +193,14 @@ RopeAppendParams pool_params(const pkv_pool* pool, int layer)
 {
     RopeAppendParams prm;
     std::memset(&prm, 0, sizeof(prm));
-    const size_t off = (size_t)layer * pool->layer_elems * 2;
+    const size_t off = (size_t)layer * pool->layer_bytes();
     prm.k_layer = static_cast<char*>(pool->k_base) + off;
     prm.v_layer = static_cast<char*>(pool->v_base) + off;
+    if (pool->storage == kStorageI8) {
+        prm.ks_layer = static_cast<float*>(pool->k_scale_base) + (size_t)layer * pool->layer_rows();
+        prm.vs_layer = static_cast<float*>(pool->v_scale_base) + (size_t)layer * pool->layer_rows();
+        prm.mode = kRopeQuantI8;
+    }
     prm.kv_heads = pool->kv_heads;
     prm.head_dim = pool->head_dim;
     prm.page_size = pool->page_size;
@@ -237,7 +249,7 @@ extern "C" int paged_kv_append(const pkv_pool* pool, int layer, const void* k, c
     prm.k = const_cast<void*>(k);    // read only: no rotation in this mode
     prm.v = v;
     prm.slots = slot_mapping;
-    prm.mode = kRopeAppend;
+    prm.mode |= kRopeAppend;
     return launch_rope_append(prm, n_tokens, pool->dtype, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -258,7 +270,7 @@ extern "C" int rope_append(const pkv_pool* pool, int layer, void* q, void* k, co
     prm.slots = slot_mapping;
     prm.q_heads = q_heads;
     prm.theta = theta;
-    prm.mode = kRopeRotate | kRopeAppend;
+    prm.mode |= kRopeRotate | kRopeAppend;
     return launch_rope_append(prm, n_tokens, pool->dtype, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -289,7 +301,8 @@ extern "C" int pkv_decode_default_splits(int q_heads, int kv_heads, int head_dim
 {
     if (!num_splits_out || q_heads <= 0 || kv_heads <= 0 || q_heads % kv_heads) return PKV_ERR_INVALID_ARG;
     DecodeOps ops;
-    if (!pick_decode(head_dim, page_size, q_heads / kv_heads, dtype, ops)) return PKV_ERR_UNSUPPORTED;
+    const int act = dtype == PKV_I8 ? PKV_F16 : dtype;     // int8 pages: split count of the f16 kernel
+    if (!pick_decode(head_dim, page_size, q_heads / kv_heads, act, dtype, ops)) return PKV_ERR_UNSUPPORTED;
     return ops.splits(num_splits_out);
 }
 
@@ -313,7 +326,7 @@ extern "C" int paged_decode_attention(const pkv_pool* pool, int layer, void* out
     if ((reinterpret_cast<uintptr_t>(out) | reinterpret_cast<uintptr_t>(q)) & 15u) return PKV_ERR_INVALID_ARG;
     if (reinterpret_cast<uintptr_t>(workspace) & 255u) return PKV_ERR_INVALID_ARG;
     DecodeOps ops;
-    if (!pick_decode(pool->head_dim, pool->page_size, q_heads / kv_heads, pool->dtype, ops))
+    if (!pick_decode(pool->head_dim, pool->page_size, q_heads / kv_heads, pool->dtype, pool->storage, ops))
         return PKV_ERR_UNSUPPORTED;
     if (num_splits == 0) {
         const int st = ops.splits(&num_splits);
@@ -322,9 +335,14 @@ extern "C" int paged_decode_attention(const pkv_pool* pool, int layer, void* out
     const WorkspaceLayout wl = workspace_layout(batch, ops.group, pool->head_dim, num_splits);
     if (workspace_bytes < wl.total) return PKV_ERR_NO_SPACE;
     DecodeParams prm;
-    const size_t elt = 2;
-    prm.k = static_cast<const char*>(pool->k_base) + (size_t)layer * pool->layer_elems * elt;
-    prm.v = static_cast<const char*>(pool->v_base) + (size_t)layer * pool->layer_elems * elt;
+    prm.k = static_cast<const char*>(pool->k_base) + (size_t)layer * pool->layer_bytes();
+    prm.v = static_cast<const char*>(pool->v_base) + (size_t)layer * pool->layer_bytes();
+    prm.k_scale = nullptr;
+    prm.v_scale = nullptr;
+    if (pool->storage == kStorageI8) {
+        prm.k_scale = static_cast<const float*>(pool->k_scale_base) + (size_t)layer * pool->layer_rows();
+        prm.v_scale = static_cast<const float*>(pool->v_scale_base) + (size_t)layer * pool->layer_rows();
+    }
     prm.q = q;
     prm.out = out;
     prm.block_tables = block_tables;
@@ -391,6 +409,7 @@ extern "C" int paged_prefill_attention(const pkv_pool* pool, int layer, void* ou
     if (batch < 0 || total_q < 0 || q_heads <= 0 || kv_heads != pool->kv_heads || q_heads % kv_heads)
         return PKV_ERR_INVALID_ARG;
     if (max_pages_per_seq <= 0 || !(scale == scale)) return PKV_ERR_INVALID_ARG;
+    if (pool->storage != pool->dtype) return PKV_ERR_UNSUPPORTED;    // int8 pages: decode only
     if (batch == 0 || total_q == 0) return PKV_OK;
     if (!out || !q || !cu_q || !block_tables || !context_lens) return PKV_ERR_INVALID_ARG;
     if (misaligned16(out, q)) return PKV_ERR_INVALID_ARG;

@@ -25,14 +25,17 @@ extern "C" const char* pkv_status_string(int status)
     }
 }
 
-extern "C" int kv_pool_create(int num_layers, int num_pages, int page_size, int kv_heads,
-                              int head_dim, int dtype, void* k_base, void* v_base, pkv_pool** out)
+namespace {
+
+int make_pool(int num_layers, int num_pages, int page_size, int kv_heads, int head_dim, int dtype, int storage,
+              void* k_base, void* v_base, void* k_scales, void* v_scales, pkv_pool** out)
 {
     if (!out) return PKV_ERR_INVALID_ARG;
     *out = nullptr;
-    if (num_layers <= 0 || num_pages <= 0 || kv_heads <= 0 || !k_base || !v_base)
-        return PKV_ERR_INVALID_ARG;
-    if ((reinterpret_cast<uintptr_t>(k_base) | reinterpret_cast<uintptr_t>(v_base)) & 15u)
+    if (num_layers <= 0 || num_pages <= 0 || kv_heads <= 0 || !k_base || !v_base) return PKV_ERR_INVALID_ARG;
+    if (storage == PKV_I8 && (!k_scales || !v_scales)) return PKV_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(k_base) | reinterpret_cast<uintptr_t>(v_base) |
+         reinterpret_cast<uintptr_t>(k_scales) | reinterpret_cast<uintptr_t>(v_scales)) & 15u)
         return PKV_ERR_INVALID_ARG;
     if (page_size != 16 && page_size != 32) return PKV_ERR_UNSUPPORTED;
     if (head_dim != 64 && head_dim != 128) return PKV_ERR_UNSUPPORTED;
@@ -45,13 +48,41 @@ extern "C" int kv_pool_create(int num_layers, int num_pages, int page_size, int 
     p->kv_heads = kv_heads;
     p->head_dim = head_dim;
     p->dtype = dtype;
+    p->storage = storage;
     p->k_base = k_base;
     p->v_base = v_base;
+    p->k_scale_base = k_scales;
+    p->v_scale_base = v_scales;
     p->layer_elems = (int64_t)num_pages * kv_heads * page_size * head_dim;
     p->free_stack.resize((size_t)num_pages);
     for (int i = 0; i < num_pages; ++i) p->free_stack[(size_t)i] = num_pages - 1 - i;  // top = 0
     p->allocated.assign((size_t)num_pages, 0);
     *out = p;
+    return PKV_OK;
+}
+
+}  // namespace
+
+extern "C" int kv_pool_create(int num_layers, int num_pages, int page_size, int kv_heads,
+                              int head_dim, int dtype, void* k_base, void* v_base, pkv_pool** out)
+{
+    return make_pool(num_layers, num_pages, page_size, kv_heads, head_dim, dtype, dtype, k_base, v_base, nullptr,
+                     nullptr, out);
+}
+
+// int8 pages ([ENGINE] s3.4 compression): codes plus one fp32 scale per (token, head) row.
+extern "C" int kv_pool_create_i8(int num_layers, int num_pages, int page_size, int kv_heads, int head_dim,
+                                 int dtype, void* k_codes, void* v_codes, void* k_scales, void* v_scales,
+                                 pkv_pool** out)
+{
+    return make_pool(num_layers, num_pages, page_size, kv_heads, head_dim, dtype, PKV_I8, k_codes, v_codes,
+                     k_scales, v_scales, out);
+}
+
+extern "C" int kv_pool_storage(const pkv_pool* pool, int* storage_out)
+{
+    if (!pool || !storage_out) return PKV_ERR_INVALID_ARG;
+    *storage_out = pool->storage;
     return PKV_OK;
 }
 
@@ -111,6 +142,7 @@ extern "C" int64_t pkv_kv_cache_bytes(int num_layers, int kv_heads, int head_dim
                                       int dtype)
 {
     if (num_layers < 0 || kv_heads < 0 || head_dim < 0 || tokens < 0) return -1;
+    if (dtype == PKV_I8) return (int64_t)num_layers * 2 * kv_heads * tokens * (head_dim + 4);
     if (dtype != PKV_F16 && dtype != PKV_BF16) return -1;
     const int64_t elt = 2;
     return (int64_t)num_layers * 2 * kv_heads * head_dim * tokens * elt;

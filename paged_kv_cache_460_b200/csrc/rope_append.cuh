@@ -13,6 +13,7 @@ namespace pkv {
 
 constexpr int kRopeRotate = 1;   // turn q and k in place
 constexpr int kRopeAppend = 2;   // write k and v into their pool slots
+constexpr int kRopeQuantI8 = 4;  // ... as int8 codes plus a per-row fp32 scale
 
 struct RopeAppendParams {
     void* q;                 // [n][q_heads][d]   (rotated in place)
@@ -22,6 +23,8 @@ struct RopeAppendParams {
     const int64_t* slots;
     void* k_layer;           // this layer's K pool [pages][kv_heads][P][d]
     void* v_layer;
+    float* ks_layer;         // int8 pools: this layer's row scales [pages][kv_heads][P]
+    float* vs_layer;
     int q_heads;
     int kv_heads;
     int head_dim;
@@ -39,6 +42,10 @@ struct RopeAppendParams {
 // fp64 (explicit _rn products: no fused rounding) and rounded once to the storage type.
 // Appending copies the rotated k and the v vector bit for bit into row slot % P of page
 // slot / P; a negative slot skips the token, a slot past the pool is skipped and flagged.
+// On an int8 pool the head row is quantised instead ([ENGINE] s3.4 compression):
+// amax = max |x| over the row's head_dim/8 threads (a shuffle reduction; a row's threads
+// are consecutive lanes of one warp), codes round_half_even(x * (127 / amax)) clamped to
+// +-127, scale amax / 127, every step a correctly rounded fp32 operation.
 template <typename T>
 __global__ void __launch_bounds__(256) rope_append_kernel(const RopeAppendParams p)
 {
@@ -107,10 +114,37 @@ __global__ void __launch_bounds__(256) rope_append_kernel(const RopeAppendParams
             }
             *src = u;
         }
-        if (slot >= 0 && idx >= nq) {
-            uint4* dst = static_cast<uint4*>(is_v ? p.v_layer : p.k_layer) +
-                         ((page * p.kv_heads + h) * p.page_size + row) * vph + c;
-            *dst = u;
+        if (slot >= 0 && idx >= nq) {      // uniform over the vph threads of a head row
+            const int64_t row_id = (page * p.kv_heads + h) * p.page_size + row;
+            if (p.mode & kRopeQuantI8) {
+                float x[8];
+                unpack8<T>(u, x);
+                float amax = 0.f;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(x[e]));
+                const unsigned lane = threadIdx.x & 31u;
+                const unsigned gmask = vph == 32 ? 0xffffffffu : ((1u << vph) - 1u) << (lane & ~(unsigned)(vph - 1));
+                for (int m = vph >> 1; m >= 1; m >>= 1) amax = fmaxf(amax, __shfl_xor_sync(gmask, amax, m));
+                uint2 codes = make_uint2(0u, 0u);
+                float sc = 0.f;
+                if (amax > 0.f) {
+                    const float inv = __fdiv_rn(127.f, amax);
+                    uint32_t w[2] = {0u, 0u};
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float r = fminf(fmaxf(rintf(__fmul_rn(x[e], inv)), -127.f), 127.f);
+                        w[e >> 2] |= ((uint32_t)(int)r & 0xffu) << (8 * (e & 3));
+                    }
+                    codes = make_uint2(w[0], w[1]);
+                    sc = __fdiv_rn(amax, 127.f);
+                }
+                *reinterpret_cast<uint2*>(static_cast<int8_t*>(is_v ? p.v_layer : p.k_layer) +
+                                          row_id * p.head_dim + c * 8) = codes;
+                if (c == 0) (is_v ? p.vs_layer : p.ks_layer)[row_id] = sc;
+            } else {
+                uint4* dst = static_cast<uint4*>(is_v ? p.v_layer : p.k_layer) + row_id * vph + c;
+                *dst = u;
+            }
         }
     }
 }

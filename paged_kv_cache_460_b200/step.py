@@ -43,7 +43,8 @@ class DecodeStep:
         self.slot_mapping = torch.full((batch,), -1, dtype=torch.int64, device=dev)
         self.scale = 1.0 / math.sqrt(d) if scale is None else scale
         self.theta = theta
-        self.workspace = DecodeWorkspace(batch, q_heads, Hkv, d, pool.page_size, dt, num_splits, device=dev)
+        self.workspace = DecodeWorkspace(batch, q_heads, Hkv, d, pool.page_size, dt, num_splits, device=dev,
+                                         storage=pool.storage)
         self.graph = None
         self.kernels_per_step = 2 * L
 

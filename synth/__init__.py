@@ -295,3 +295,48 @@ def mini_pool_numpy(s, b, g, seed):
     k = round_f32(rng.standard_normal(shape, dtype=np.float32), s.dtype)
     v = round_f32(rng.standard_normal(shape, dtype=np.float32), s.dtype)
     return k, v
+
+
+# ----------------------------------------------------------------- int8 pages
+# Stored int8 pages are drawn directly: codes uniform in [-127, 127], per-row fp32 scales
+# uniform in [1.5, 2.5] / 127 (values within about +-2, like the fp16 pools' N(0, 1)), the
+# keys of the long-context mix's peaky rows with an 8x scale.
+
+def pool_values_i8_numpy(s, seed=None):
+    """(k_codes, v_codes) int8 [layers, pages, Hkv, P, d] and (k_scales, v_scales) fp32
+    [layers, pages, Hkv, P], numpy PCG64."""
+    rng = _rng((value_seed(s) if seed is None else seed) + 4_000_000)
+    shape = s.pool_shape()
+    kc = rng.integers(-127, 128, size=shape, dtype=np.int8)
+    vc = rng.integers(-127, 128, size=shape, dtype=np.int8)
+    ks = (rng.uniform(1.5, 2.5, size=shape[:-1]) / 127.0).astype(np.float32)
+    vs = (rng.uniform(1.5, 2.5, size=shape[:-1]) / 127.0).astype(np.float32)
+    if s.peaky_keys > 0:
+        for (_, _, page, row) in _peaky_rows(s, rng):
+            ks[:, page, :, row] *= np.float32(8.0)
+    return kc, vc, ks, vs
+
+
+def pool_values_i8_torch(s, device, seed=None):
+    """The same kind of int8 pages as torch tensors on `device`, filled layer by layer from
+    torch's seeded generator: (k_codes, v_codes, k_scales, v_scales)."""
+    import torch
+    base = (value_seed(s) if seed is None else seed) + 5_000_000
+    shape = s.pool_shape()
+    codes = [torch.empty(shape, dtype=torch.int8, device=device) for _ in range(2)]
+    scales = [torch.empty(shape[:-1], dtype=torch.float32, device=device) for _ in range(2)]
+    g = torch.Generator(device=device)
+    for layer in range(shape[0]):
+        for i in range(2):
+            g.manual_seed(base + 4 * layer + 2 * i)
+            codes[i][layer].random_(-127, 128, generator=g)
+            g.manual_seed(base + 4 * layer + 2 * i + 1)
+            scales[i][layer].uniform_(1.5 / 127.0, 2.5 / 127.0, generator=g)
+    if s.peaky_keys > 0:
+        rows = _peaky_rows(s, _rng(base))
+        if rows:
+            pages = torch.tensor([r[2] for r in rows], device=device)
+            prow = torch.tensor([r[3] for r in rows], device=device)
+            for layer in range(shape[0]):
+                scales[0][layer][pages, :, prow] *= 8.0
+    return codes[0], codes[1], scales[0], scales[1]

@@ -226,3 +226,42 @@ def test_prefill_validates(L):
     assert L.paged_prefill_attention(h, 0, None, f(), f(), 4, f(), 4, f(), 1, 2, 2, 0.1, None) == _lib.PKV_ERR_INVALID_ARG
     assert L.paged_prefill_attention(h, 0, f(), f(), f(), 0, f(), 4, f(), 1, 2, 2, 0.1, None) == 0
     L.kv_pool_destroy(h)
+
+
+def _pool_i8(L, num_pages=8, page_size=16, kv_heads=2, head_dim=64, dtype=0, layers=1):
+    h = ctypes.c_void_p()
+    f = _fake_ptr
+    st = L.kv_pool_create_i8(layers, num_pages, page_size, kv_heads, head_dim, dtype, f(), f(0x20000), f(0x30000),
+                             f(0x40000), ctypes.byref(h))
+    assert st == 0
+    return h
+
+
+def test_int8_pool_create_validates_and_reports_its_storage(L):
+    h = ctypes.c_void_p()
+    f = _fake_ptr
+    assert L.kv_pool_create_i8(1, 8, 16, 2, 64, 0, f(), f(), None, f(), ctypes.byref(h)) == _lib.PKV_ERR_INVALID_ARG
+    assert L.kv_pool_create_i8(1, 8, 16, 2, 64, 0, f(), f(), f(), f(0x10004), ctypes.byref(h)) == \
+        _lib.PKV_ERR_INVALID_ARG
+    assert L.kv_pool_create_i8(1, 8, 16, 2, 64, _lib.PKV_I8, f(), f(), f(), f(), ctypes.byref(h)) == \
+        _lib.PKV_ERR_UNSUPPORTED          # the activation type must be fp16 or bf16
+    assert L.kv_pool_create_i8(1, 8, 8, 2, 64, 0, f(), f(), f(), f(), ctypes.byref(h)) == _lib.PKV_ERR_UNSUPPORTED
+    h = _pool_i8(L, dtype=1, layers=2)
+    storage, dt = ctypes.c_int(), ctypes.c_int()
+    assert L.kv_pool_storage(h, ctypes.byref(storage)) == 0 and storage.value == _lib.PKV_I8
+    assert L.kv_pool_info(h, None, None, None, None, None, ctypes.byref(dt)) == 0 and dt.value == 1
+    assert L.kv_pool_storage(None, ctypes.byref(storage)) == _lib.PKV_ERR_INVALID_ARG
+    # chunked prefill reads 16-bit pages only
+    assert L.paged_prefill_attention(h, 0, f(), f(), f(), 4, f(), 4, f(), 1, 2, 2, 0.1, None) == \
+        _lib.PKV_ERR_UNSUPPORTED
+    L.kv_pool_destroy(h)
+    h = _pool(L)
+    assert L.kv_pool_storage(h, ctypes.byref(storage)) == 0 and storage.value == 0
+    L.kv_pool_destroy(h)
+
+
+def test_int8_kv_cache_bytes():
+    # 7B shape, 2048 tokens: each (token, head) row is 128 code bytes plus a 4-byte scale, for K and V
+    assert pkv.pkv_kv_cache_bytes(32, 32, 128, 2048, pkv.PKV_I8) == 32 * 2 * 32 * 2048 * 132
+    assert pkv.pkv_kv_cache_bytes(32, 32, 128, 2048, pkv.PKV_I8) * 2 < \
+        pkv.pkv_kv_cache_bytes(32, 32, 128, 2048, pkv.PKV_F16) * 1.04
