@@ -70,25 +70,18 @@ struct DecodeParams {
 
 __host__ __device__ constexpr int align_up(int x, int a) { return (x + a - 1) / a * a; }
 
-template <int D, int P, int G, bool I8 = false>
+template <int D, int P, int G>
 struct DecodeShape {
-    static constexpr int kChunk = P * D * (I8 ? 1 : 2);      // bytes of one (page, head) of K or V
-    static constexpr int kScaleBytes = I8 ? P * 4 : 0;       // its fp32 row scales (int8 pages)
+    static constexpr int kChunk = P * D * 2;                 // bytes of one (page, head)
     static constexpr int kQBytes = G * D * 2;
-    static constexpr int kQOffset = 2 * kChunk + 2 * kScaleBytes;   // q rows within a slot
-    static constexpr int kSlot = kQOffset + kQBytes;
-    // int8 pages: q as fp32, in registers while a lane's slices fit in 32 of them, else in
-    // a per-warp [G][D] shared buffer
-    static constexpr bool kQReg = G * D / 4 <= 32;
-    static constexpr int kQfBytes = (I8 && !kQReg) ? kDecodeWarps * G * D * 4 : 0;
+    static constexpr int kSlot = 2 * kChunk + kQBytes;
     static constexpr int kDepthRaw = kRingBudgetBytes / (kDecodeWarps * kSlot);
     static constexpr int kDepth = kDepthRaw < 2 ? 2 : (kDepthRaw > 8 ? 8 : kDepthRaw);
     static constexpr int kRingBytes = kDecodeWarps * kDepth * kSlot;
     static constexpr int kCmbOffset = kRingBytes;
     static constexpr int kCmbFloats = kDecodeWarps * G * (D + 2);
     static constexpr int kPbufOffset = kCmbOffset + 2 * kCmbFloats * 4;     // [warps][G][P] floats
-    static constexpr int kQfOffset = kPbufOffset + kDecodeWarps * G * P * 4;
-    static constexpr int kWarpTotOffset = kQfOffset + kQfBytes;
+    static constexpr int kWarpTotOffset = kPbufOffset + kDecodeWarps * G * P * 4;
     static constexpr int kScanOffset = kWarpTotOffset + 64;
     // prefix[batch+1] and lens[batch] follow
     static int smem_bytes(int batch) { return kScanOffset + 4 * (2 * batch + 1); }
@@ -154,20 +147,6 @@ __device__ __forceinline__ void next_unit(int& b, int& g, int& j, int& np, const
         ++b;
         np = b < batch ? prefix[b + 1] - prefix[b] : 1;
     } while (np == 0);
-}
-
-// int8 pages: four codes (two's complement bytes of w) -> four exact floats.  Each byte,
-// offset by 128, becomes the low mantissa bits of 2^23 (a byte permute), and one packed
-// subtraction of 2^23 + 128 leaves the code.
-__device__ __forceinline__ void i8x4_to_float(uint32_t w, float (&f)[4])
-{
-    const uint32_t x = w ^ 0x80808080u;
-    const float2 bias = make_float2(-8388736.f, -8388736.f);
-    const float2 a = __fadd2_rn(make_float2(__uint_as_float(__byte_perm(x, 0x4B000000u, 0x7440)),
-                                            __uint_as_float(__byte_perm(x, 0x4B000000u, 0x7441))), bias);
-    const float2 b = __fadd2_rn(make_float2(__uint_as_float(__byte_perm(x, 0x4B000000u, 0x7442)),
-                                            __uint_as_float(__byte_perm(x, 0x4B000000u, 0x7443))), bias);
-    f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
 }
 
 // End of a segment, after every warp has published its (m, l, o) of it in `buf`
@@ -263,22 +242,15 @@ __device__ __forceinline__ void segment_epilogue(const DecodeParams& p, const fl
     }
 }
 
-// I8: int8 pages with per-row fp32 scales ([ENGINE] s3.4 compression).  The same stream
-// of (page, head) units; a page-head is P*D code bytes of K and of V plus P scales each.
-// q.k: four lanes share a K row (lane (t, h) takes 16-byte chunks h, h + 4, ... of rows t,
-// t + 8, ...), the codes become exact floats (i8x4_to_float) and meet q in fp32; the row's
-// dot times its K scale is the score.  p.V: each p is multiplied by the row's V scale when
-// it is published, and the lane's V codes become floats like the K codes.
-template <int D, int P, int G, typename T, bool I8 = false>
+template <int D, int P, int G, typename T>
 __global__ void __launch_bounds__(kDecodeThreads, G == 1 ? 4 : 1) decode_pass1_kernel(const DecodeParams p)
 {
-    using S = DecodeShape<D, P, G, I8>;
+    using S = DecodeShape<D, P, G>;
     constexpr int NW = kDecodeWarps;
     constexpr int DEPTH = S::kDepth;
-    constexpr int CPR = I8 ? D / 16 : D / 8;   // 16-byte chunks per K/V row
-    constexpr int LPRK = I8 ? 4 : 2;      // lanes sharing one K row in q.k
-    constexpr int ROWSTEP = 32 / LPRK;    // rows t, t + ROWSTEP, ... per lane
-    constexpr int RPL = P / ROWSTEP;      // K rows per lane per page
+    constexpr int CPR = D / 8;            // 16-byte chunks per K/V row
+    constexpr int LPRK = 2;               // lanes sharing one K row in q.k
+    constexpr int RPL = P / 16;           // K rows per lane per page (rows t and t + 16)
     constexpr int CPL = CPR / LPRK;       // K chunks per lane per row
     constexpr int EPL = D / 32;           // output columns owned by each lane in p.V
     constexpr int QV = S::kQBytes / 16;   // 16-byte pieces of the group's q rows
@@ -287,7 +259,6 @@ __global__ void __launch_bounds__(kDecodeThreads, G == 1 ? 4 : 1) decode_pass1_k
     extern __shared__ __align__(128) unsigned char smem[];
     float* cmb = reinterpret_cast<float*>(smem + S::kCmbOffset);
     float* pbuf_all = reinterpret_cast<float*>(smem + S::kPbufOffset);
-    float* qf_all = reinterpret_cast<float*>(smem + S::kQfOffset);
     int* warp_tot = reinterpret_cast<int*>(smem + S::kWarpTotOffset);
     volatile int* last_flag = warp_tot + 8;
     int* prefix = reinterpret_cast<int*>(smem + S::kScanOffset);
@@ -326,9 +297,8 @@ __global__ void __launch_bounds__(kDecodeThreads, G == 1 ? 4 : 1) decode_pass1_k
 
     // ---- issue side: this warp's page k (iterator at unit r0 + warp + k NW).
     // K rows land XOR-swizzled by 16-byte chunk -- chunk c of row t at position
-    // c ^ ((2 t + c / CPL) & 7), int8 rows of 128 codes at c ^ (4 (t & 1)) -- so that the
-    // lanes reading different rows at the same column hit different banks; V rows and the
-    // scales land as they are.
+    // c ^ ((2 t + c / CPL) & 7) -- so that the lanes reading different rows at the same
+    // column hit different banks; V rows land as they are.
     int ib = 0, ig = 0, ij = 0, inp = 1, qb = -1, qg = -1;
     if (n_mine > 0) {
         locate_unit(r0 + warp, prefix, p.batch, Hkv, ib, ig, ij);
@@ -342,25 +312,16 @@ __global__ void __launch_bounds__(kDecodeThreads, G == 1 ? 4 : 1) decode_pass1_k
         const int page = __shfl_sync(0xffffffffu, win, (int)(k - win0));
         unsigned char* slot = smem + ring_off + (int)(k % DEPTH) * S::kSlot;
         if ((unsigned)page < (unsigned)p.num_pages) {
-            const long long row0 = ((long long)page * Hkv + ig) * P;     // first (token, head) row
-            const unsigned char* ks = static_cast<const unsigned char*>(p.k) + row0 * (S::kChunk / P);
-            const unsigned char* vs = static_cast<const unsigned char*>(p.v) + row0 * (S::kChunk / P);
+            const long long off = ((long long)page * Hkv + ig) * (P * D);
+            const unsigned char* ks = reinterpret_cast<const unsigned char*>(static_cast<const T*>(p.k) + off);
+            const unsigned char* vs = reinterpret_cast<const unsigned char*>(static_cast<const T*>(p.v) + off);
 #pragma unroll
             for (int n = 0; n < S::kChunk / 512; ++n) {
                 const int gidx = n * 32 + lane;               // 16-byte chunk of the page
                 const int t = gidx / CPR, c = gidx % CPR;
-                const int pos = I8 ? (D == 128 ? c ^ ((t & 1) << 2) : c) : c ^ ((t * LPRK + c / CPL) & 7);
-                cp_async16(slot + t * (S::kChunk / P) + pos * 16, ks + gidx * 16);
+                const int pos = c ^ ((t * LPRK + c / CPL) & 7);
+                cp_async16(slot + t * (2 * D) + pos * 16, ks + gidx * 16);
                 cp_async16(slot + S::kChunk + gidx * 16, vs + gidx * 16);
-            }
-            if constexpr (I8) {
-                constexpr int SC = S::kScaleBytes / 16;      // 16-byte pieces of P scales
-                if (lane < SC)
-                    cp_async16(slot + 2 * S::kChunk + lane * 16,
-                               reinterpret_cast<const unsigned char*>(p.k_scale + row0) + lane * 16);
-                else if (lane >= 16 && lane < 16 + SC)
-                    cp_async16(slot + 2 * S::kChunk + S::kScaleBytes + (lane - 16) * 16,
-                               reinterpret_cast<const unsigned char*>(p.v_scale + row0) + (lane - 16) * 16);
             }
         } else if (lane == 0) {
             atomicOr(&g_error_word, PKV_DEVERR_BAD_PAGE);   // never dereferenced
@@ -370,7 +331,7 @@ __global__ void __launch_bounds__(kDecodeThreads, G == 1 ? 4 : 1) decode_pass1_k
         unsigned char* slot = smem + ring_off + (int)(k % DEPTH) * S::kSlot;
         const unsigned char* qs = reinterpret_cast<const unsigned char*>(
             static_cast<const T*>(p.q) + ((long long)bq * p.q_heads + (long long)gq * G) * D);
-        for (int n = lane; n < QV; n += 32) cp_async16(slot + S::kQOffset + n * 16, qs + n * 16);
+        for (int n = lane; n < QV; n += 32) cp_async16(slot + 2 * S::kChunk + n * 16, qs + n * 16);
     };
     auto advance = [&]() {
         if (ij + NW < inp) {
@@ -431,11 +392,8 @@ __global__ void __launch_bounds__(kDecodeThreads, G == 1 ? 4 : 1) decode_pass1_k
     // at P = 32) over chunks h*CPL .. h*CPL+CPL-1; p.V: lane owns output columns
     // lane*EPL .. lane*EPL+EPL-1.
     const int t_own = lane / LPRK, h_own = lane % LPRK;
-    const int sw_own = I8 ? (D == 128 ? (t_own & 1) << 2 : 0) : (t_own * LPRK + h_own) & 7;
-    uint4 qraw[I8 ? 1 : G][I8 ? 1 : CPL];
-    constexpr bool kQReg = I8 && S::kQReg;
-    float qreg[kQReg ? G : 1][kQReg ? CPL * 16 : 1];     // int8: q slices of chunks h_own + 4 i
-    float* qf = qf_all + warp * G * D;                  // int8, !kQReg: q [G][D], swizzled
+    const int sw_own = (t_own * LPRK + h_own) & 7;
+    uint4 qraw[G][CPL];
     float o[G][EPL], m_run[G], l_run[G];
 #pragma unroll
     for (int gi = 0; gi < G; ++gi) {
@@ -461,102 +419,33 @@ __global__ void __launch_bounds__(kDecodeThreads, G == 1 ? 4 : 1) decode_pass1_k
             const unsigned char* s = ring + (int)(kc % DEPTH) * S::kSlot;
             if (!have_q) {                      // first page of this segment for this warp
                 have_q = true;
-                if constexpr (!I8) {
 #pragma unroll
-                    for (int gi = 0; gi < G; ++gi)
+                for (int gi = 0; gi < G; ++gi)
 #pragma unroll
-                        for (int i = 0; i < CPL; ++i)
-                            qraw[gi][i] = *reinterpret_cast<const uint4*>(s + S::kQOffset + gi * (2 * D) +
-                                                                          (h_own * CPL + i) * 16);
-                } else if constexpr (kQReg) {
-#pragma unroll
-                    for (int gi = 0; gi < G; ++gi)
-#pragma unroll
-                        for (int i = 0; i < CPL; ++i) {
-                            const uint4* src = reinterpret_cast<const uint4*>(s + S::kQOffset + gi * (2 * D) +
-                                                                              (i * LPRK + h_own) * 32);
-                            float f[8];
-                            unpack8<T>(src[0], f);
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) qreg[gi][i * 16 + e] = f[e];
-                            unpack8<T>(src[1], f);
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) qreg[gi][i * 16 + 8 + e] = f[e];
-                        }
-                } else {
-                    // q [G][D] as fp32 into the warp's buffer; element 16 c + 4 w + e of a row
-                    // at 16 c + 4 ((w ^ c) & 3) + e, so that the four lanes of a K row (chunks
-                    // c = h, h + 4, ...) read distinct banks
-                    for (int n = lane; n < G * D / 8; n += 32) {
-                        const int gi = n / (D / 8), e0 = (n % (D / 8)) * 8;
-                        const int c = e0 / 16, w0 = (e0 % 16) / 4;
-                        float f[8];
-                        unpack8<T>(*reinterpret_cast<const uint4*>(s + S::kQOffset + n * 16), f);
-                        float* row = qf + gi * D + c * 16;
-                        *reinterpret_cast<float4*>(row + 4 * ((w0 ^ c) & 3)) = make_float4(f[0], f[1], f[2], f[3]);
-                        *reinterpret_cast<float4*>(row + 4 * (((w0 + 1) ^ c) & 3)) =
-                            make_float4(f[4], f[5], f[6], f[7]);
-                    }
-                    __syncwarp();
-                }
+                    for (int i = 0; i < CPL; ++i)
+                        qraw[gi][i] = *reinterpret_cast<const uint4*>(s + 2 * S::kChunk + gi * (2 * D) +
+                                                                      (h_own * CPL + i) * 16);
             }
             const int nvalid = min(P, lens[b] - (j + (int)(uu - u)) * P);
-            // ---- scores: lane's partial dots over its chunks of rows t_own, t_own + ROWSTEP, ...
+            // ---- scores: lane's partial dots over its chunks of rows t_own (+ 16)
             float sc[G][RPL];
-            const float* ksc = reinterpret_cast<const float*>(s + 2 * S::kChunk);               // int8
-            const float* vsc = reinterpret_cast<const float*>(s + 2 * S::kChunk + S::kScaleBytes);
 #pragma unroll
             for (int rr = 0; rr < RPL; ++rr) {
                 float acc[G];
 #pragma unroll
                 for (int gi = 0; gi < G; ++gi) acc[gi] = 0.f;
-                const int t = t_own + ROWSTEP * rr;
-                if constexpr (!I8) {
+                const int t = t_own + 16 * rr;
 #pragma unroll
-                    for (int i = 0; i < CPL; ++i) {
-                        const int pos = (h_own * CPL + i) ^ sw_own;
-                        const uint4 ku = *reinterpret_cast<const uint4*>(s + t * (2 * D) + pos * 16);
+                for (int i = 0; i < CPL; ++i) {
+                    const int pos = (h_own * CPL + i) ^ sw_own;
+                    const uint4 ku = *reinterpret_cast<const uint4*>(s + t * (2 * D) + pos * 16);
 #pragma unroll
-                        for (int gi = 0; gi < G; ++gi) acc[gi] += dot8<T>(qraw[gi][i], ku);
-                    }
-                } else {
-                    float2 acc2[G];
-#pragma unroll
-                    for (int gi = 0; gi < G; ++gi) acc2[gi] = make_float2(0.f, 0.f);
-#pragma unroll
-                    for (int i = 0; i < CPL; ++i) {
-                        const int c = i * LPRK + h_own;
-                        const uint4 ku = *reinterpret_cast<const uint4*>(s + t * D + (c ^ sw_own) * 16);
-                        const uint32_t kw[4] = {ku.x, ku.y, ku.z, ku.w};
-#pragma unroll
-                        for (int w = 0; w < 4; ++w) {
-                            float kf[4];
-                            i8x4_to_float(kw[w], kf);
-#pragma unroll
-                            for (int gi = 0; gi < G; ++gi) {
-                                float4 q4;
-                                if constexpr (kQReg) {
-                                    q4 = make_float4(qreg[gi][i * 16 + 4 * w], qreg[gi][i * 16 + 4 * w + 1],
-                                                     qreg[gi][i * 16 + 4 * w + 2], qreg[gi][i * 16 + 4 * w + 3]);
-                                } else {
-                                    q4 = *reinterpret_cast<const float4*>(qf + gi * D + c * 16 + 4 * ((w ^ c) & 3));
-                                }
-                                acc2[gi] = __ffma2_rn(make_float2(q4.x, q4.y), make_float2(kf[0], kf[1]), acc2[gi]);
-                                acc2[gi] = __ffma2_rn(make_float2(q4.z, q4.w), make_float2(kf[2], kf[3]), acc2[gi]);
-                            }
-                        }
-                    }
-#pragma unroll
-                    for (int gi = 0; gi < G; ++gi) acc[gi] = acc2[gi].x + acc2[gi].y;
+                    for (int gi = 0; gi < G; ++gi) acc[gi] += dot8<T>(qraw[gi][i], ku);
                 }
 #pragma unroll
                 for (int gi = 0; gi < G; ++gi) {
-#pragma unroll
-                    for (int m = 1; m < LPRK; m <<= 1) acc[gi] += __shfl_xor_sync(0xffffffffu, acc[gi], m);
-                    if constexpr (I8)
-                        sc[gi][rr] = t < nvalid ? acc[gi] * ksc[t] * p.scale_log2 : -INFINITY;
-                    else
-                        sc[gi][rr] = t < nvalid ? acc[gi] * p.scale_log2 : -INFINITY;
+                    acc[gi] += __shfl_xor_sync(0xffffffffu, acc[gi], 1);
+                    sc[gi][rr] = t < nvalid ? acc[gi] * p.scale_log2 : -INFINITY;
                 }
             }
             // ---- online softmax update; p of every row published to the warp's buffer
@@ -568,7 +457,7 @@ __global__ void __launch_bounds__(kDecodeThreads, G == 1 ? 4 : 1) decode_pass1_k
 #pragma unroll
                 for (int rr = 1; rr < RPL; ++rr) pm = fmaxf(pm, sc[gi][rr]);
 #pragma unroll
-                for (int m = 16; m >= LPRK; m >>= 1) pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, m));
+                for (int m = 16; m >= 2; m >>= 1) pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, m));
                 const float mn = fmaxf(m_run[gi], pm);   // finite: row 0 of a page is always valid
                 alpha[gi] = fast_exp2(m_run[gi] - mn);
                 rescale |= m_run[gi] != mn;
@@ -578,12 +467,7 @@ __global__ void __launch_bounds__(kDecodeThreads, G == 1 ? 4 : 1) decode_pass1_k
                 for (int rr = 0; rr < RPL; ++rr) {
                     const float pr = fast_exp2(sc[gi][rr] - mn);   // 0 for rows past the context
                     ls += pr;
-                    const int t = t_own + ROWSTEP * rr;
-                    if constexpr (I8) {
-                        if (h_own == 0) pbuf[gi * P + t] = t < nvalid ? pr * vsc[t] : 0.f;
-                    } else {
-                        if (h_own == 0) pbuf[gi * P + t] = pr;
-                    }
+                    if (h_own == 0) pbuf[gi * P + t_own + 16 * rr] = pr;
                 }
                 l_run[gi] = l_run[gi] * alpha[gi] + (h_own == 0 ? ls : 0.f);
             }
@@ -599,19 +483,10 @@ __global__ void __launch_bounds__(kDecodeThreads, G == 1 ? 4 : 1) decode_pass1_k
             }
             __syncwarp();                         // p of all rows visible to the warp
             // ---- o += p V: row t's EPL columns of this lane (rows past the context skipped)
-            const unsigned char* vbase = s + S::kChunk + lane * (EPL * (I8 ? 1 : 2));
+            const unsigned char* vbase = s + S::kChunk + lane * (EPL * 2);
             auto pv_row = [&](int t) {
                 float vf[EPL];
-                if constexpr (I8) {
-                    float f4[4];
-                    if constexpr (EPL == 4) {
-                        i8x4_to_float(*reinterpret_cast<const uint32_t*>(vbase + t * D), f4);
-                    } else {
-                        i8x4_to_float(*reinterpret_cast<const uint16_t*>(vbase + t * D), f4);
-                    }
-#pragma unroll
-                    for (int e = 0; e < EPL; ++e) vf[e] = f4[e];
-                } else if constexpr (EPL == 4) {
+                if constexpr (EPL == 4) {
                     const uint2 w = *reinterpret_cast<const uint2*>(vbase + t * (2 * D));
                     const float2 a = Elt<T>::to_float2(w.x), c2 = Elt<T>::to_float2(w.y);
                     vf[0] = a.x; vf[1] = a.y; vf[2] = c2.x; vf[3] = c2.y;

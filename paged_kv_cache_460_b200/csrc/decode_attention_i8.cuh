@@ -1,0 +1,424 @@
+// Paged decode attention over int8 KV pages on the tensor cores.
+//
+// The pages' KV strategy pairs paging with compression of the cached values ("为什么要
+// 自己动手写一个LLM推理引擎" (wzjinhao.cn/news/61427) s3.4).  Here every cached (token, kv
+// head) row of K and V is head_dim int8 codes c with one fp32 scale s, the value being
+// c * s.  The kernel computes the same softmax(scale q.K^T) V as the 16-bit kernels, with
+// the balanced partition, per-warp cp.async rings, PDL prologue and in-kernel merge of
+// decode_attention.cuh, over 16-token units as in decode_attention_mma.cuh:
+//   S^T[16 tokens x 8 heads] = C_K[16 x D] . Q^T[D x 8]          (fp16 MMAs, fp32 sums)
+//   scores = S^T * s_K(token) * scale                             (heads >= G are zero)
+//   O^T[D x 8] += C_V^T[D x 16] . (p * s_V * 2^E)^T[16 x 8]       (fp16 MMAs)
+// Decoding: the codes are read with ldmatrix as 16-bit pairs (non-transposed for K,
+// transposed for V) and each byte becomes an exact fp16 value: the byte offset by 128 is
+// placed under the exponent of 1024 with one byte permute, and one packed fp16
+// subtraction of 1152 leaves the code.  Which bytes of a fragment register feed which
+// MMA operand slot fixes a permutation of the contraction index (head_dim for K, the
+// output column order for V); q's fragments are loaded in the same permuted order and
+// the output columns are written back in place, so no data is moved to undo it.
+// fp16 for both data types: codes are exact in fp16; bf16 q is scaled by a power of two
+// per head row (none unless max |q| >= 2^15) so that it converts exactly; P times the V
+// scale is scaled by 2^E per unit (E from the unit's largest V scale), which keeps it in
+// fp16's normal range, and the accumulated output is rescaled when E changes.  A row whose
+// V scale lies more than 2^14 below the unit's largest one gets a subnormal fp16 weight:
+// its absolute error stays under 2^-25 of the unit's largest possible weight.
+#ifndef PKV_DECODE_ATTENTION_I8_CUH_
+#define PKV_DECODE_ATTENTION_I8_CUH_
+
+#include "decode_attention_mma.cuh"
+
+namespace pkv {
+
+template <int D, int G>
+struct I8Shape {
+    static constexpr int kRows = 16;                          // token rows per unit
+    static constexpr int kChunk = kRows * D;                  // code bytes of one unit's K (or V)
+    static constexpr int kScaleBytes = kRows * 4;             // its fp32 row scales
+    static constexpr int kQOffset = 2 * kChunk + 2 * kScaleBytes;
+    static constexpr int kQBytes = G * D * 2;
+    static constexpr int kSlot = kQOffset + kQBytes;
+    static constexpr int kDepthRaw = kRingBudgetBytes / (kDecodeWarps * kSlot);
+    static constexpr int kDepth = kDepthRaw < 2 ? 2 : (kDepthRaw > 8 ? 8 : kDepthRaw);
+    static constexpr int kRingBytes = kDecodeWarps * kDepth * kSlot;
+    static constexpr int kCmbOffset = kRingBytes;
+    static constexpr int kCmbFloats = kDecodeWarps * G * (D + 2);
+    static constexpr int kWarpTotOffset = kCmbOffset + 2 * kCmbFloats * 4;
+    static constexpr int kScanOffset = kWarpTotOffset + 64;
+    static int smem_bytes(int batch) { return kScanOffset + 4 * (2 * batch + 1); }
+};
+
+// Position of 16-byte chunk c of token row t in shared memory: c ^ swizzle(t), so that the
+// eight rows of one ldmatrix (consecutive tokens, same chunk) fall in distinct banks
+// (rows of 128 bytes: eight chunks; rows of 64 bytes: two rows per 128-byte line).
+template <int D>
+__device__ __forceinline__ int i8_swizzle(int t)
+{
+    return D == 128 ? (t & 7) : ((t >> 1) & 3);
+}
+
+// Two exact fp16 codes from the bytes of x picked by `sel` (a byte-permute selector whose
+// odd nibbles pick 0x64): ((0x64 << 8) | (byte ^ 0x80)) is 1024 + code + 128.
+__device__ __forceinline__ uint32_t i8_pair_to_f16x2(uint32_t x_biased, uint32_t sel)
+{
+    const uint32_t h = __byte_perm(x_biased, 0x64646464u, sel);
+    uint32_t r;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(h), "r"(0x64806480u));   // 1152 = 0x6480
+    return r;
+}
+
+// Bytes 0,1 / 2,3 (K fragments: consecutive head_dim columns of one token)
+__device__ __forceinline__ void i8_lo_hi(uint32_t w, uint32_t& lo, uint32_t& hi)
+{
+    const uint32_t x = w ^ 0x80808080u;
+    lo = i8_pair_to_f16x2(x, 0x5140u);
+    hi = i8_pair_to_f16x2(x, 0x5342u);
+}
+
+// Bytes 0,2 / 1,3 (transposed V fragments: tokens 2i, 2i+1 of an even / odd column)
+__device__ __forceinline__ void i8_even_odd(uint32_t w, uint32_t& ev, uint32_t& od)
+{
+    const uint32_t x = w ^ 0x80808080u;
+    ev = i8_pair_to_f16x2(x, 0x5240u);
+    od = i8_pair_to_f16x2(x, 0x5341u);
+}
+
+template <int D, int P, int G, typename T>
+__global__ void __launch_bounds__(kDecodeThreads, 4) decode_i8_kernel(const DecodeParams p)
+{
+    using S = I8Shape<D, G>;
+    using Mma = MmaOps<__half>;
+    constexpr int NW = kDecodeWarps;
+    constexpr int DEPTH = S::kDepth;
+    constexpr int CPR = D / 16;           // 16-byte chunks per token row
+    constexpr int U = P / 16;             // units per page
+    constexpr int KS = D / 16;            // k-steps of q.k = m-tiles of p.V
+    constexpr int QV = S::kQBytes / 16;
+    static_assert(P == 16 || P == 32, "page size");
+    static_assert(D == 64 || D == 128, "head_dim");
+    static_assert(G >= 1 && G <= 8, "1 to 8 query heads per kv head");
+    extern __shared__ __align__(128) unsigned char smem[];
+    float* cmb = reinterpret_cast<float*>(smem + S::kCmbOffset);
+    int* warp_tot = reinterpret_cast<int*>(smem + S::kWarpTotOffset);
+    volatile int* last_flag = warp_tot + 8;
+    int* prefix = reinterpret_cast<int*>(smem + S::kScanOffset);
+    int* lens = prefix + p.batch + 1;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    // Prologue before the PDL wait, as in the 16-bit kernels.
+    block_page_prefix<16>(p.context_lens, p.batch, prefix, lens, warp_tot);
+    __syncthreads();
+    const int Hkv = p.kv_heads;
+    const long long W = (long long)Hkv * prefix[p.batch];
+    const long long chunk = W > 0 ? (W + p.num_splits - 1) / p.num_splits : 1;
+    const long long r0 = (long long)blockIdx.x * chunk;
+    const long long r1 = min(W, r0 + chunk);
+    const long long n_mine = r1 - r0 > warp ? (r1 - r0 - warp + NW - 1) / NW : 0;
+
+    auto load_window = [&](long long win0) {
+        const long long k = win0 + lane;
+        int id = 0;
+        if (k < n_mine) {
+            int bb, gg, jj;
+            locate_unit(r0 + warp + k * NW, prefix, p.batch, Hkv, bb, gg, jj);
+            const int pg = jj / U;
+            id = pg < p.max_pages ? p.block_tables[(long long)bb * p.max_pages + pg] : -1;
+        }
+        return id;
+    };
+    long long win0 = 0;
+    int win = load_window(0);
+    unsigned char* ring = smem + warp * DEPTH * S::kSlot;
+
+    int ib = 0, ig = 0, ij = 0, inp = 1, qb = -1, qg = -1;
+    if (n_mine > 0) {
+        locate_unit(r0 + warp, prefix, p.batch, Hkv, ib, ig, ij);
+        inp = prefix[ib + 1] - prefix[ib];
+    }
+    // unit k of this warp into ring slot `sl` (= k mod DEPTH)
+    auto issue_kv = [&](long long k, int sl) {
+        if (k >= win0 + 32) {
+            win0 = k;
+            win = load_window(k);
+        }
+        const int page = __shfl_sync(0xffffffffu, win, (int)(k - win0));
+        unsigned char* slot = ring + sl * S::kSlot;
+        if ((unsigned)page < (unsigned)p.num_pages) {
+            const long long row0 = ((long long)page * Hkv + ig) * P + (ij % U) * 16;   // first token row
+            const unsigned char* ks = static_cast<const unsigned char*>(p.k) + row0 * D;
+            const unsigned char* vs = static_cast<const unsigned char*>(p.v) + row0 * D;
+#pragma unroll
+            for (int n = 0; n < S::kChunk / 512; ++n) {
+                const int gidx = n * 32 + lane;
+                const int t = gidx / CPR, c = gidx % CPR;
+                const int dst = t * D + ((c ^ i8_swizzle<D>(t)) * 16);
+                cp_async16(slot + dst, ks + gidx * 16);
+                cp_async16(slot + S::kChunk + dst, vs + gidx * 16);
+            }
+            if (lane < 4)
+                cp_async16(slot + 2 * S::kChunk + lane * 16,
+                           reinterpret_cast<const unsigned char*>(p.k_scale + row0) + lane * 16);
+            else if (lane >= 16 && lane < 20)
+                cp_async16(slot + 2 * S::kChunk + S::kScaleBytes + (lane - 16) * 16,
+                           reinterpret_cast<const unsigned char*>(p.v_scale + row0) + (lane - 16) * 16);
+        } else if (lane == 0) {
+            atomicOr(&g_error_word, PKV_DEVERR_BAD_PAGE);   // never dereferenced
+        }
+    };
+    auto issue_q = [&](int sl, int bq, int gq) {
+        unsigned char* slot = ring + sl * S::kSlot;
+        const unsigned char* qs = reinterpret_cast<const unsigned char*>(
+            static_cast<const T*>(p.q) + ((long long)bq * p.q_heads + (long long)gq * G) * D);
+        for (int n = lane; n < QV; n += 32) cp_async16(slot + S::kQOffset + n * 16, qs + n * 16);
+    };
+    auto advance = [&]() {
+        if (ij + NW < inp) {
+            ij += NW;
+        } else {
+            for (int t = 0; t < NW; ++t) next_unit(ib, ig, ij, inp, prefix, Hkv, p.batch);
+        }
+    };
+    auto issue = [&](long long k, int sl) {
+        issue_kv(k, sl);
+        if (ib != qb || ig != qg) {
+            qb = ib;
+            qg = ig;
+            issue_q(sl, ib, ig);
+        }
+        advance();
+    };
+    int m_pre = 0, pre_qb[DEPTH], pre_qg[DEPTH];
+    for (; m_pre < DEPTH && m_pre < n_mine; ++m_pre) {
+        if (ij == inp - 1) break;
+        issue_kv(m_pre, m_pre);
+        pre_qb[m_pre] = -1;
+        if (ib != qb || ig != qg) {
+            qb = ib;
+            qg = ig;
+            pre_qb[m_pre] = ib;
+            pre_qg[m_pre] = ig;
+        }
+        advance();
+        cp_async_commit();
+    }
+
+    pdl_wait();
+    pdl_launch_dependents();
+    for (int b = blockIdx.x; b < p.batch; b += gridDim.x) {
+        if (prefix[b + 1] != prefix[b]) continue;
+        T* row = static_cast<T*>(p.out) + (long long)b * p.q_heads * D;
+        for (int idx = tid; idx < p.q_heads * D; idx += blockDim.x) row[idx] = Elt<T>::from_float(0.f);
+    }
+    if (r0 >= r1) return;
+
+    for (int k = 0; k < m_pre; ++k)
+        if (pre_qb[k] >= 0) issue_q(k, pre_qb[k], pre_qg[k]);
+    if (m_pre == DEPTH) cp_async_commit();
+    for (int k = m_pre; k < DEPTH; ++k) {
+        if (k < n_mine) issue(k, k);
+        cp_async_commit();
+    }
+    cp_async_wait<0>();
+
+    // ---- compute side (fragments of m16n8k16: g4 = lane / 4, t4 = lane % 4).  ldmatrix
+    // x4 rows: lane l supplies token ((l >> 3) & 1) * 8 + (l & 7) of chunk 2x + (l >> 4).
+    const int g4 = lane >> 2, t4 = lane & 3;
+    const int lm_tok = ((lane >> 3) & 1) * 8 + (lane & 7);
+    const int lm_off = lm_tok * D;
+    const int lm_chunk = lane >> 4, lm_swz = i8_swizzle<D>(lm_tok);
+    uint32_t bq[KS][2];                       // Q^T fragments: head g4, columns 16kk + 4t4 + {0,1 | 2,3}
+    float qscale[2];                          // 2^s(head) * scale * log2(e) for heads 2 t4 + j
+    float oacc[KS][4], m_run[2], l_run[2];    // O^T * 2^E: rows 16 mt + 2 g4 (+1), heads 2 t4 + j
+#pragma unroll
+    for (int mt = 0; mt < KS; ++mt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) oacc[mt][e] = 0.f;
+    m_run[0] = m_run[1] = -INFINITY;
+    l_run[0] = l_run[1] = 0.f;
+    int e_cur = 127;                          // biased exponent of 2^-E (the unit scale in use)
+    long long kc = 0;
+    int cs = 0;                               // ring slot of unit kc
+    int b, g, j;
+    locate_unit(r0, prefix, p.batch, Hkv, b, g, j);
+    int np = prefix[b + 1] - prefix[b];
+    int seg = 0;
+    for (long long u = r0; u < r1; ++seg) {
+        const long long u_end = min(r1, u + (np - j));
+        const long long first = u + ((warp - (int)((u - r0) % NW)) + NW) % NW;
+        bool have_q = false;
+        for (long long uu = first; uu < u_end; uu += NW) {
+            cp_async_wait<DEPTH - 1>();
+            __syncwarp();
+            const unsigned char* s = ring + cs * S::kSlot;
+            if (!have_q) {
+                have_q = true;
+                const T* qa = reinterpret_cast<const T*>(s + S::kQOffset);
+                int shift = 0;                // power of two that brings the head row's max under 2^15
+                if constexpr (std::is_same<T, __half>::value) {
+#pragma unroll
+                    for (int kk = 0; kk < KS; ++kk) {
+                        const uint2 w = g4 < G ? *reinterpret_cast<const uint2*>(qa + g4 * D + kk * 16 + 4 * t4)
+                                               : make_uint2(0u, 0u);
+                        bq[kk][0] = w.x;
+                        bq[kk][1] = w.y;
+                    }
+                } else {
+                    float qf[KS][4];
+                    float mx = 0.f;
+#pragma unroll
+                    for (int kk = 0; kk < KS; ++kk) {
+                        const uint2 w = g4 < G ? *reinterpret_cast<const uint2*>(qa + g4 * D + kk * 16 + 4 * t4)
+                                               : make_uint2(0u, 0u);
+                        const float2 a = Elt<T>::to_float2(w.x), c2 = Elt<T>::to_float2(w.y);
+                        qf[kk][0] = a.x; qf[kk][1] = a.y; qf[kk][2] = c2.x; qf[kk][3] = c2.y;
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) mx = fmaxf(mx, fabsf(qf[kk][e]));
+                    }
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+                    shift = max(0, (int)((__float_as_uint(mx) >> 23) & 0xff) - 141);   // 141 = 127 + 14
+                    const float down = __uint_as_float((uint32_t)(127 - shift) << 23);   // 2^-shift
+#pragma unroll
+                    for (int kk = 0; kk < KS; ++kk) {
+                        bq[kk][0] = Mma::pack(qf[kk][0] * down, qf[kk][1] * down);
+                        bq[kk][1] = Mma::pack(qf[kk][2] * down, qf[kk][3] * down);
+                    }
+                }
+#pragma unroll
+                for (int jh = 0; jh < 2; ++jh) {
+                    const int sh = __shfl_sync(0xffffffffu, shift, (2 * t4 + jh) * 4);
+                    qscale[jh] = __uint_as_float((uint32_t)(127 + sh) << 23) * p.scale_log2;
+                }
+            }
+            const int nvalid = min(16, lens[b] - (j + (int)(uu - u)) * 16);
+            const unsigned char* kb = s;
+            const unsigned char* vb = s + S::kChunk;
+            const float* ksc = reinterpret_cast<const float*>(s + 2 * S::kChunk);
+            const float* vsc = reinterpret_cast<const float*>(s + 2 * S::kChunk + S::kScaleBytes);
+            // ---- S^T = C_K . Q^T
+            float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int x = 0; x < KS / 2; ++x) {
+                uint32_t r[4];
+                ldmatrix_x4(r, kb + lm_off + (((2 * x + lm_chunk) ^ lm_swz) * 16));
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {             // k-step 2x + h: r[2h] tokens 0-7, r[2h+1] 8-15
+                    uint32_t a[4];
+                    i8_lo_hi(r[2 * h], a[0], a[2]);
+                    i8_lo_hi(r[2 * h + 1], a[1], a[3]);
+                    Mma::mma(sacc, a, bq[2 * x + h][0], bq[2 * x + h][1]);
+                }
+            }
+            // ---- scores: (token g4, heads 2t4, 2t4+1), (token g4 + 8, same heads)
+            const bool v0 = g4 < nvalid, v1 = g4 + 8 < nvalid;
+            const float k0 = ksc[g4], k1 = ksc[g4 + 8];
+            float sc[4];
+            sc[0] = v0 ? sacc[0] * k0 * qscale[0] : -INFINITY;
+            sc[1] = v0 ? sacc[1] * k0 * qscale[1] : -INFINITY;
+            sc[2] = v1 ? sacc[2] * k1 * qscale[0] : -INFINITY;
+            sc[3] = v1 ? sacc[3] * k1 * qscale[1] : -INFINITY;
+            // ---- this unit's power-of-two scale 2^E: the largest valid V scale times 2^E is in [1, 2)
+            const float s0 = v0 ? vsc[g4] : 0.f, s1 = v1 ? vsc[g4 + 8] : 0.f;
+            float smax = fmaxf(s0, s1);
+#pragma unroll
+            for (int m = 4; m < 32; m <<= 1) smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, m));
+            const int e_unit = (int)(__float_as_uint(smax) >> 23);        // 0 for an all-zero unit
+            const int e_new = e_unit > 0 ? e_unit : e_cur;
+            const float up = __uint_as_float((uint32_t)(254 - e_new) << 23);            // 2^E
+            // O' = O * 2^E: rescale by 2^(E_new - E_old) = 2^(e_cur - e_new) (clamped to
+            // fp32's normal range)
+            const float ratio = __uint_as_float((uint32_t)min(254, max(1, 127 + e_cur - e_new)) << 23);
+            float alpha[2], pr[4];
+#pragma unroll
+            for (int jh = 0; jh < 2; ++jh) {
+                float pm = fmaxf(sc[jh], sc[jh + 2]);
+#pragma unroll
+                for (int m = 4; m < 32; m <<= 1) pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, m));
+                const float mn = fmaxf(m_run[jh], pm);         // finite: row 0 is always valid
+                alpha[jh] = fast_exp2(m_run[jh] - mn);
+                m_run[jh] = mn;
+                pr[jh] = fast_exp2(sc[jh] - mn);
+                pr[jh + 2] = fast_exp2(sc[jh + 2] - mn);
+                l_run[jh] = l_run[jh] * alpha[jh] + pr[jh] + pr[jh + 2];
+            }
+            if (__any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f || e_new != e_cur)) {
+                const float f0 = alpha[0] * ratio, f1 = alpha[1] * ratio;
+#pragma unroll
+                for (int mt = 0; mt < KS; ++mt) {
+                    oacc[mt][0] *= f0;
+                    oacc[mt][1] *= f1;
+                    oacc[mt][2] *= f0;
+                    oacc[mt][3] *= f1;
+                }
+            }
+            e_cur = e_new;
+            // ---- (p * s_V * 2^E)^T as the B operand (fp16), via movmatrix.trans of the
+            //      8x8 blocks of tokens 0-7 and 8-15
+            const float w0 = s0 * up, w1 = s1 * up;
+            const uint32_t pb0 = movmatrix_trans(Mma::pack(pr[0] * w0, pr[1] * w0));
+            const uint32_t pb1 = movmatrix_trans(Mma::pack(pr[2] * w1, pr[3] * w1));
+            // ---- O^T += C_V^T . P'^T; m-tile mt holds columns 16 mt + 2 g4 (row g4) and
+            //      16 mt + 2 g4 + 1 (row g4 + 8)
+#pragma unroll
+            for (int x = 0; x < KS / 2; ++x) {
+                uint32_t r[4];
+                ldmatrix_x4_trans(r, vb + lm_off + (((2 * x + lm_chunk) ^ lm_swz) * 16));
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {             // m-tile 2x + h: r[2h] tokens 0-7, r[2h+1] 8-15
+                    uint32_t a[4];
+                    i8_even_odd(r[2 * h], a[0], a[1]);
+                    i8_even_odd(r[2 * h + 1], a[2], a[3]);
+                    Mma::mma(oacc[2 * x + h], a, pb0, pb1);
+                }
+            }
+            __syncwarp();
+            if (kc + DEPTH < n_mine) issue(kc + DEPTH, cs);
+            cp_async_commit();
+            ++kc;
+            cs = cs + 1 == DEPTH ? 0 : cs + 1;
+        }
+        // ---- publish this warp's state: o[head][d] (2^-E applied), m, l of the real heads
+        float* buf = cmb + (seg & 1) * S::kCmbFloats;
+        const float down = __uint_as_float((uint32_t)e_cur << 23);                 // 2^-E
+#pragma unroll
+        for (int jh = 0; jh < 2; ++jh) {
+            float lt = l_run[jh];
+#pragma unroll
+            for (int m = 4; m < 32; m <<= 1) lt += __shfl_xor_sync(0xffffffffu, lt, m);
+            const int head = 2 * t4 + jh;
+            if (head < G) {
+                float* row = buf + (warp * G + head) * (D + 2);
+#pragma unroll
+                for (int mt = 0; mt < KS; ++mt) {
+                    row[mt * 16 + 2 * g4] = oacc[mt][jh] * down;
+                    row[mt * 16 + 2 * g4 + 1] = oacc[mt][2 + jh] * down;
+                }
+                if (g4 == 0) {
+                    row[D] = m_run[jh];
+                    row[D + 1] = lt;
+                }
+            }
+            m_run[jh] = -INFINITY;
+            l_run[jh] = 0.f;
+        }
+#pragma unroll
+        for (int mt = 0; mt < KS; ++mt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) oacc[mt][e] = 0.f;
+        e_cur = 127;
+        segment_epilogue<D, G, T>(p, buf, b, g, np, prefix, r0, r1, chunk, last_flag);
+        u = u_end;
+        j = 0;
+        if (++g == Hkv) {
+            g = 0;
+            do {
+                ++b;
+                np = b < p.batch ? prefix[b + 1] - prefix[b] : 1;
+            } while (np == 0);
+        }
+    }
+    cp_async_wait<0>();
+}
+
+}  // namespace pkv
+
+#endif  // PKV_DECODE_ATTENTION_I8_CUH_

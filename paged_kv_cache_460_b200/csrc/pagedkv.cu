@@ -13,6 +13,7 @@
 #include <mutex>
 
 #include "decode_attention.cuh"
+#include "decode_attention_i8.cuh"
 #include "decode_attention_mma.cuh"
 #include "prefill_attention.cuh"
 #include "pagedkv.h"
@@ -67,11 +68,16 @@ struct DecodeOps {
 };
 
 // One query head per kv head: the CUDA-core kernel; 2 to 8 heads sharing a kv head: the
-// tensor-core kernel.  Int8 pages (I8): the CUDA-core kernel for every group size.
-template <int D, int P, int G, typename T, bool I8, bool kMma = (G > 1 && !I8)>
+// tensor-core kernel.  Int8 pages (I8): the int8 tensor-core kernel for every group size.
+template <int D, int P, int G, typename T, bool I8, bool kMma = (G > 1)>
 struct DecodeKernel {
-    static constexpr auto fn = decode_pass1_kernel<D, P, G, T, I8>;
-    static int smem(int batch) { return DecodeShape<D, P, G, I8>::smem_bytes(batch); }
+    static constexpr auto fn = decode_pass1_kernel<D, P, G, T>;
+    static int smem(int batch) { return DecodeShape<D, P, G>::smem_bytes(batch); }
+};
+template <int D, int P, int G, typename T, bool kMma>
+struct DecodeKernel<D, P, G, T, true, kMma> {
+    static constexpr auto fn = decode_i8_kernel<D, P, G, T>;
+    static int smem(int batch) { return I8Shape<D, G>::smem_bytes(batch); }
 };
 template <int D, int P, int G, typename T>
 struct DecodeKernel<D, P, G, T, false, true> {

@@ -126,6 +126,25 @@ def test_int8_step_matches_oracle_on_workload(name):
     assert pkv.kv_get_device_error() == 0
 
 
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_int8_row_scales_spanning_many_binades(dtype):
+    """Row scales drawn log-uniformly over 2^-10 .. 2^2 (and a few all-zero V rows), so that
+    the largest V scale of consecutive 16-token units changes binade all the time.  (The
+    kernel keeps each unit's P * s_V in fp16 relative to the unit's largest V scale: rows
+    more than 2^14 below it lose relative precision; 12 binades stay inside that range.)"""
+    s = synth.random_spec(650, 4, 16, 4, 128, 16, [700, 33, 129, 2047], dtype=dtype)
+    c = I8Case(s)
+    r = np.random.Generator(np.random.PCG64(651))
+    for arr, t in ((c.ks, c.t[2]), (c.vs, c.t[3])):
+        arr[...] = (2.0 ** r.uniform(-10, 2, size=arr.shape) / 127.0).astype(np.float32)
+        t.copy_(torch.from_numpy(arr))
+    zero = r.random(c.vs.shape) < 0.02
+    c.vs[zero] = 0
+    c.t[3].copy_(torch.from_numpy(c.vs))
+    _expect_close(c.gpu_layer(0), c.oracle_layer(0), dtype, "int8 wide scales")
+    assert pkv.kv_get_device_error() == 0
+
+
 def test_int8_split_count_sweep():
     s = synth.random_spec(700, 5, 8, 8, 128, 16, [1000, 17, 300, 0, 2000])
     ref = None
