@@ -5,14 +5,19 @@
 // head) row of K and V is head_dim int8 codes c with one fp32 scale s, the value being
 // c * s.  The kernel computes the same softmax(scale q.K^T) V as the 16-bit kernels, with
 // the balanced partition, per-warp cp.async rings, PDL prologue and in-kernel merge of
-// decode_attention.cuh, over 16-token units as in decode_attention_mma.cuh:
-//   S^T[16 tokens x 8 heads] = C_K[16 x D] . Q^T[D x 8]          (fp16 MMAs, fp32 sums)
+// decode_attention.cuh, over 32-token units (a 32-token page or two 16-token pages),
+// each two 16-token tiles:
+//   S^T[32 tokens x 8 heads] = C_K[32 x D] . Q^T[D x 8]          (fp16 MMAs, fp32 sums)
 //   scores = S^T * s_K(token) * scale                             (heads >= G are zero)
-//   O^T[D x 8] += C_V^T[D x 16] . (p * s_V * 2^E)^T[16 x 8]       (fp16 MMAs)
+//   O^T[D x 8] += C_V^T[D x 32] . (p * s_V * 2^E)^T[32 x 8]       (fp16 MMAs)
+// A 32-token unit halves, per token, the fixed cost of a unit (softmax reductions, ring
+// and page-table bookkeeping) next to the 16-token tiles of the 16-bit MMA kernel.
 // Decoding: the codes are read with ldmatrix as 16-bit pairs (non-transposed for K,
 // transposed for V) and each byte becomes an exact fp16 value: the byte offset by 128 is
-// placed under the exponent of 1024 with one byte permute, and one packed fp16
-// subtraction of 1152 leaves the code.  Which bytes of a fragment register feed which
+// placed under the exponent of 1024 with one byte permute (1152 + code); for V one packed
+// fp16 subtraction of 1152 leaves the code, for K the constant stays in the MMA operand and
+// 1152 * sum_d q_d is subtracted from each score (q is fixed for the whole segment, and the
+// offset sum spans only head_dim terms, unlike the output sums over the whole context).  Which bytes of a fragment register feed which
 // MMA operand slot fixes a permutation of the contraction index (head_dim for K, the
 // output column order for V); q's fragments are loaded in the same permuted order and
 // the output columns are written back in place, so no data is moved to undo it.
@@ -31,7 +36,7 @@ namespace pkv {
 
 template <int D, int G>
 struct I8Shape {
-    static constexpr int kRows = 16;                          // token rows per unit
+    static constexpr int kRows = 32;                          // token rows per unit
     static constexpr int kChunk = kRows * D;                  // code bytes of one unit's K (or V)
     static constexpr int kScaleBytes = kRows * 4;             // its fp32 row scales
     static constexpr int kQOffset = 2 * kChunk + 2 * kScaleBytes;
@@ -66,12 +71,13 @@ __device__ __forceinline__ uint32_t i8_pair_to_f16x2(uint32_t x_biased, uint32_t
     return r;
 }
 
-// Bytes 0,1 / 2,3 (K fragments: consecutive head_dim columns of one token)
-__device__ __forceinline__ void i8_lo_hi(uint32_t w, uint32_t& lo, uint32_t& hi)
+// Bytes 0,1 / 2,3 (K fragments: consecutive head_dim columns of one token) as fp16
+// 1152 + code: the constant is removed after the MMA (1152 * sum(q) per head).
+__device__ __forceinline__ void i8_lo_hi_biased(uint32_t w, uint32_t& lo, uint32_t& hi)
 {
     const uint32_t x = w ^ 0x80808080u;
-    lo = i8_pair_to_f16x2(x, 0x5140u);
-    hi = i8_pair_to_f16x2(x, 0x5342u);
+    lo = __byte_perm(x, 0x64646464u, 0x5140u);
+    hi = __byte_perm(x, 0x64646464u, 0x5342u);
 }
 
 // Bytes 0,2 / 1,3 (transposed V fragments: tokens 2i, 2i+1 of an even / odd column)
@@ -83,14 +89,15 @@ __device__ __forceinline__ void i8_even_odd(uint32_t w, uint32_t& ev, uint32_t& 
 }
 
 template <int D, int P, int G, typename T>
-__global__ void __launch_bounds__(kDecodeThreads, 4) decode_i8_kernel(const DecodeParams p)
+__global__ void __launch_bounds__(kDecodeThreads, 3) decode_i8_kernel(const DecodeParams p)
 {
     using S = I8Shape<D, G>;
     using Mma = MmaOps<__half>;
     constexpr int NW = kDecodeWarps;
     constexpr int DEPTH = S::kDepth;
     constexpr int CPR = D / 16;           // 16-byte chunks per token row
-    constexpr int U = P / 16;             // units per page
+    constexpr int PPU = 32 / P;           // pages per 32-token unit
+    constexpr int WIN = 32 / PPU;         // units whose page ids one window holds
     constexpr int KS = D / 16;            // k-steps of q.k = m-tiles of p.V
     constexpr int QV = S::kQBytes / 16;
     static_assert(P == 16 || P == 32, "page size");
@@ -104,28 +111,30 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_i8_kernel(const Deco
     int* lens = prefix + p.batch + 1;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-    // Prologue before the PDL wait, as in the 16-bit kernels.
-    block_page_prefix<16>(p.context_lens, p.batch, prefix, lens, warp_tot);
+    // Prologue before the PDL wait, as in the 16-bit kernels; units are 32 tokens.
+    block_page_prefix<32>(p.context_lens, p.batch, prefix, lens, warp_tot);
     __syncthreads();
     const int Hkv = p.kv_heads;
     const long long W = (long long)Hkv * prefix[p.batch];
     const long long chunk = W > 0 ? (W + p.num_splits - 1) / p.num_splits : 1;
     const long long r0 = (long long)blockIdx.x * chunk;
     const long long r1 = min(W, r0 + chunk);
-    const long long n_mine = r1 - r0 > warp ? (r1 - r0 - warp + NW - 1) / NW : 0;
+    const int n_mine = r1 - r0 > warp ? (int)((r1 - r0 - warp + NW - 1) / NW) : 0;
 
-    auto load_window = [&](long long win0) {
-        const long long k = win0 + lane;
-        int id = 0;
+    // lane l holds the id of page l % PPU of this warp's unit win0 + l / PPU: -1 when the
+    // page table has no such entry, -2 when the unit's tokens end before that page
+    auto load_window = [&](int win0) {
+        const int k = win0 + lane / PPU;
+        int id = -2;
         if (k < n_mine) {
             int bb, gg, jj;
-            locate_unit(r0 + warp + k * NW, prefix, p.batch, Hkv, bb, gg, jj);
-            const int pg = jj / U;
-            id = pg < p.max_pages ? p.block_tables[(long long)bb * p.max_pages + pg] : -1;
+            locate_unit(r0 + warp + (long long)k * NW, prefix, p.batch, Hkv, bb, gg, jj);
+            const int pg = jj * PPU + lane % PPU;
+            if (pg * P < lens[bb]) id = pg < p.max_pages ? p.block_tables[(long long)bb * p.max_pages + pg] : -1;
         }
         return id;
     };
-    long long win0 = 0;
+    int win0 = 0;
     int win = load_window(0);
     unsigned char* ring = smem + warp * DEPTH * S::kSlot;
 
@@ -134,34 +143,40 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_i8_kernel(const Deco
         locate_unit(r0 + warp, prefix, p.batch, Hkv, ib, ig, ij);
         inp = prefix[ib + 1] - prefix[ib];
     }
-    // unit k of this warp into ring slot `sl` (= k mod DEPTH)
-    auto issue_kv = [&](long long k, int sl) {
-        if (k >= win0 + 32) {
+    // unit k of this warp into ring slot `sl` (= k mod DEPTH): its P-token pages land at
+    // unit rows pp * P ..
+    auto issue_kv = [&](int k, int sl) {
+        if (k >= win0 + WIN) {
             win0 = k;
             win = load_window(k);
         }
-        const int page = __shfl_sync(0xffffffffu, win, (int)(k - win0));
         unsigned char* slot = ring + sl * S::kSlot;
-        if ((unsigned)page < (unsigned)p.num_pages) {
-            const long long row0 = ((long long)page * Hkv + ig) * P + (ij % U) * 16;   // first token row
-            const unsigned char* ks = static_cast<const unsigned char*>(p.k) + row0 * D;
-            const unsigned char* vs = static_cast<const unsigned char*>(p.v) + row0 * D;
 #pragma unroll
-            for (int n = 0; n < S::kChunk / 512; ++n) {
-                const int gidx = n * 32 + lane;
-                const int t = gidx / CPR, c = gidx % CPR;
-                const int dst = t * D + ((c ^ i8_swizzle<D>(t)) * 16);
-                cp_async16(slot + dst, ks + gidx * 16);
-                cp_async16(slot + S::kChunk + dst, vs + gidx * 16);
+        for (int pp = 0; pp < PPU; ++pp) {
+            const int page = __shfl_sync(0xffffffffu, win, (k - win0) * PPU + pp);
+            if (page == -2) continue;                        // past the sequence's last token
+            if ((unsigned)page < (unsigned)p.num_pages) {
+                const long long row0 = ((long long)page * Hkv + ig) * P;       // first token row
+                const unsigned char* ks = static_cast<const unsigned char*>(p.k) + row0 * D;
+                const unsigned char* vs = static_cast<const unsigned char*>(p.v) + row0 * D;
+#pragma unroll
+                for (int n = 0; n < P * D / 512; ++n) {
+                    const int gidx = n * 32 + lane;
+                    const int t = pp * P + gidx / CPR, c = gidx % CPR;
+                    const int dst = t * D + ((c ^ i8_swizzle<D>(t)) * 16);
+                    cp_async16(slot + dst, ks + gidx * 16);
+                    cp_async16(slot + S::kChunk + dst, vs + gidx * 16);
+                }
+                constexpr int SC = P / 4;                    // 16-byte pieces of P scales
+                if (lane < SC)
+                    cp_async16(slot + 2 * S::kChunk + pp * P * 4 + lane * 16,
+                               reinterpret_cast<const unsigned char*>(p.k_scale + row0) + lane * 16);
+                else if (lane >= 16 && lane < 16 + SC)
+                    cp_async16(slot + 2 * S::kChunk + S::kScaleBytes + pp * P * 4 + (lane - 16) * 16,
+                               reinterpret_cast<const unsigned char*>(p.v_scale + row0) + (lane - 16) * 16);
+            } else if (lane == 0) {
+                atomicOr(&g_error_word, PKV_DEVERR_BAD_PAGE);   // never dereferenced
             }
-            if (lane < 4)
-                cp_async16(slot + 2 * S::kChunk + lane * 16,
-                           reinterpret_cast<const unsigned char*>(p.k_scale + row0) + lane * 16);
-            else if (lane >= 16 && lane < 20)
-                cp_async16(slot + 2 * S::kChunk + S::kScaleBytes + (lane - 16) * 16,
-                           reinterpret_cast<const unsigned char*>(p.v_scale + row0) + (lane - 16) * 16);
-        } else if (lane == 0) {
-            atomicOr(&g_error_word, PKV_DEVERR_BAD_PAGE);   // never dereferenced
         }
     };
     auto issue_q = [&](int sl, int bq, int gq) {
@@ -177,7 +192,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_i8_kernel(const Deco
             for (int t = 0; t < NW; ++t) next_unit(ib, ig, ij, inp, prefix, Hkv, p.batch);
         }
     };
-    auto issue = [&](long long k, int sl) {
+    auto issue = [&](int k, int sl) {
         issue_kv(k, sl);
         if (ib != qb || ig != qg) {
             qb = ib;
@@ -219,14 +234,16 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_i8_kernel(const Deco
     }
     cp_async_wait<0>();
 
-    // ---- compute side (fragments of m16n8k16: g4 = lane / 4, t4 = lane % 4).  ldmatrix
-    // x4 rows: lane l supplies token ((l >> 3) & 1) * 8 + (l & 7) of chunk 2x + (l >> 4).
+    // ---- compute side (fragments of m16n8k16: g4 = lane / 4, t4 = lane % 4).  A unit is
+    // two 16-token tiles; ldmatrix x4 rows: lane l supplies token ((l >> 3) & 1) * 8 + (l & 7)
+    // of the tile, chunk 2x + (l >> 4).
     const int g4 = lane >> 2, t4 = lane & 3;
     const int lm_tok = ((lane >> 3) & 1) * 8 + (lane & 7);
     const int lm_off = lm_tok * D;
-    const int lm_chunk = lane >> 4, lm_swz = i8_swizzle<D>(lm_tok);
+    const int lm_chunk = lane >> 4, lm_swz = i8_swizzle<D>(lm_tok);   // same for tile 1 (rows + 16)
     uint32_t bq[KS][2];                       // Q^T fragments: head g4, columns 16kk + 4t4 + {0,1 | 2,3}
     float qscale[2];                          // 2^s(head) * scale * log2(e) for heads 2 t4 + j
+    float qbias[2];                           // 1152 * sum_d q_d (fp16 operand) of heads 2 t4 + j
     float oacc[KS][4], m_run[2], l_run[2];    // O^T * 2^E: rows 16 mt + 2 g4 (+1), heads 2 t4 + j
 #pragma unroll
     for (int mt = 0; mt < KS; ++mt)
@@ -235,7 +252,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_i8_kernel(const Deco
     m_run[0] = m_run[1] = -INFINITY;
     l_run[0] = l_run[1] = 0.f;
     int e_cur = 127;                          // biased exponent of 2^-E (the unit scale in use)
-    long long kc = 0;
+    int kc = 0;
     int cs = 0;                               // ring slot of unit kc
     int b, g, j;
     locate_unit(r0, prefix, p.batch, Hkv, b, g, j);
@@ -253,6 +270,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_i8_kernel(const Deco
                 have_q = true;
                 const T* qa = reinterpret_cast<const T*>(s + S::kQOffset);
                 int shift = 0;                // power of two that brings the head row's max under 2^15
+                float qs = 0.f;               // this lane's part of sum_d q_d (of the fp16 operand)
                 if constexpr (std::is_same<T, __half>::value) {
 #pragma unroll
                     for (int kk = 0; kk < KS; ++kk) {
@@ -260,6 +278,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_i8_kernel(const Deco
                                                : make_uint2(0u, 0u);
                         bq[kk][0] = w.x;
                         bq[kk][1] = w.y;
+                        const float2 a = Elt<__half>::to_float2(w.x), c2 = Elt<__half>::to_float2(w.y);
+                        qs += (a.x + a.y) + (c2.x + c2.y);
                     }
                 } else {
                     float qf[KS][4];
@@ -281,44 +301,59 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_i8_kernel(const Deco
                     for (int kk = 0; kk < KS; ++kk) {
                         bq[kk][0] = Mma::pack(qf[kk][0] * down, qf[kk][1] * down);
                         bq[kk][1] = Mma::pack(qf[kk][2] * down, qf[kk][3] * down);
+                        const float2 a = Elt<__half>::to_float2(bq[kk][0]), c2 = Elt<__half>::to_float2(bq[kk][1]);
+                        qs += (a.x + a.y) + (c2.x + c2.y);
                     }
                 }
+                qs += __shfl_xor_sync(0xffffffffu, qs, 1);
+                qs += __shfl_xor_sync(0xffffffffu, qs, 2);
 #pragma unroll
                 for (int jh = 0; jh < 2; ++jh) {
-                    const int sh = __shfl_sync(0xffffffffu, shift, (2 * t4 + jh) * 4);
+                    const int src = (2 * t4 + jh) * 4;
+                    const int sh = __shfl_sync(0xffffffffu, shift, src);
                     qscale[jh] = __uint_as_float((uint32_t)(127 + sh) << 23) * p.scale_log2;
+                    qbias[jh] = 1152.f * __shfl_sync(0xffffffffu, qs, src);
                 }
             }
-            const int nvalid = min(16, lens[b] - (j + (int)(uu - u)) * 16);
+            const int nvalid = (int)min(32LL, (long long)lens[b] - (j + (uu - u)) * 32);
             const unsigned char* kb = s;
             const unsigned char* vb = s + S::kChunk;
             const float* ksc = reinterpret_cast<const float*>(s + 2 * S::kChunk);
             const float* vsc = reinterpret_cast<const float*>(s + 2 * S::kChunk + S::kScaleBytes);
-            // ---- S^T = C_K . Q^T
-            float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+            // ---- S^T = C_K . Q^T for the two 16-token tiles
+            float sacc[2][4];
 #pragma unroll
-            for (int x = 0; x < KS / 2; ++x) {
-                uint32_t r[4];
-                ldmatrix_x4(r, kb + lm_off + (((2 * x + lm_chunk) ^ lm_swz) * 16));
+            for (int tau = 0; tau < 2; ++tau) {
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {             // k-step 2x + h: r[2h] tokens 0-7, r[2h+1] 8-15
-                    uint32_t a[4];
-                    i8_lo_hi(r[2 * h], a[0], a[2]);
-                    i8_lo_hi(r[2 * h + 1], a[1], a[3]);
-                    Mma::mma(sacc, a, bq[2 * x + h][0], bq[2 * x + h][1]);
+                for (int e = 0; e < 4; ++e) sacc[tau][e] = 0.f;
+#pragma unroll
+                for (int x = 0; x < KS / 2; ++x) {
+                    uint32_t r[4];
+                    ldmatrix_x4(r, kb + tau * 16 * D + lm_off + (((2 * x + lm_chunk) ^ lm_swz) * 16));
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {         // k-step 2x + h: r[2h] tokens 0-7, r[2h+1] 8-15
+                        uint32_t a[4];
+                        i8_lo_hi_biased(r[2 * h], a[0], a[2]);
+                        i8_lo_hi_biased(r[2 * h + 1], a[1], a[3]);
+                        Mma::mma(sacc[tau], a, bq[2 * x + h][0], bq[2 * x + h][1]);
+                    }
                 }
             }
-            // ---- scores: (token g4, heads 2t4, 2t4+1), (token g4 + 8, same heads)
-            const bool v0 = g4 < nvalid, v1 = g4 + 8 < nvalid;
-            const float k0 = ksc[g4], k1 = ksc[g4 + 8];
-            float sc[4];
-            sc[0] = v0 ? sacc[0] * k0 * qscale[0] : -INFINITY;
-            sc[1] = v0 ? sacc[1] * k0 * qscale[1] : -INFINITY;
-            sc[2] = v1 ? sacc[2] * k1 * qscale[0] : -INFINITY;
-            sc[3] = v1 ? sacc[3] * k1 * qscale[1] : -INFINITY;
-            // ---- this unit's power-of-two scale 2^E: the largest valid V scale times 2^E is in [1, 2)
-            const float s0 = v0 ? vsc[g4] : 0.f, s1 = v1 ? vsc[g4 + 8] : 0.f;
-            float smax = fmaxf(s0, s1);
+            // ---- scores of tokens 16 tau + g4 (+8), heads 2t4, 2t4+1; the unit's 2^E
+            float sc[2][4], w[2][2];
+            float smax = 0.f;
+#pragma unroll
+            for (int tau = 0; tau < 2; ++tau)
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int tok = 16 * tau + 8 * hh + g4;
+                    const bool ok = tok < nvalid;
+                    const float kscale = ksc[tok];
+                    sc[tau][2 * hh] = ok ? (sacc[tau][2 * hh] - qbias[0]) * kscale * qscale[0] : -INFINITY;
+                    sc[tau][2 * hh + 1] = ok ? (sacc[tau][2 * hh + 1] - qbias[1]) * kscale * qscale[1] : -INFINITY;
+                    w[tau][hh] = ok ? vsc[tok] : 0.f;
+                    smax = fmaxf(smax, w[tau][hh]);
+                }
 #pragma unroll
             for (int m = 4; m < 32; m <<= 1) smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, m));
             const int e_unit = (int)(__float_as_uint(smax) >> 23);        // 0 for an all-zero unit
@@ -327,18 +362,23 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_i8_kernel(const Deco
             // O' = O * 2^E: rescale by 2^(E_new - E_old) = 2^(e_cur - e_new) (clamped to
             // fp32's normal range)
             const float ratio = __uint_as_float((uint32_t)min(254, max(1, 127 + e_cur - e_new)) << 23);
-            float alpha[2], pr[4];
+            float alpha[2], pr[2][4];
 #pragma unroll
             for (int jh = 0; jh < 2; ++jh) {
-                float pm = fmaxf(sc[jh], sc[jh + 2]);
+                float pm = fmaxf(fmaxf(sc[0][jh], sc[0][jh + 2]), fmaxf(sc[1][jh], sc[1][jh + 2]));
 #pragma unroll
                 for (int m = 4; m < 32; m <<= 1) pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, m));
                 const float mn = fmaxf(m_run[jh], pm);         // finite: row 0 is always valid
                 alpha[jh] = fast_exp2(m_run[jh] - mn);
                 m_run[jh] = mn;
-                pr[jh] = fast_exp2(sc[jh] - mn);
-                pr[jh + 2] = fast_exp2(sc[jh + 2] - mn);
-                l_run[jh] = l_run[jh] * alpha[jh] + pr[jh] + pr[jh + 2];
+                float ls = 0.f;
+#pragma unroll
+                for (int tau = 0; tau < 2; ++tau) {
+                    pr[tau][jh] = fast_exp2(sc[tau][jh] - mn);
+                    pr[tau][jh + 2] = fast_exp2(sc[tau][jh + 2] - mn);
+                    ls += pr[tau][jh] + pr[tau][jh + 2];
+                }
+                l_run[jh] = l_run[jh] * alpha[jh] + ls;
             }
             if (__any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f || e_new != e_cur)) {
                 const float f0 = alpha[0] * ratio, f1 = alpha[1] * ratio;
@@ -351,23 +391,30 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_i8_kernel(const Deco
                 }
             }
             e_cur = e_new;
-            // ---- (p * s_V * 2^E)^T as the B operand (fp16), via movmatrix.trans of the
-            //      8x8 blocks of tokens 0-7 and 8-15
-            const float w0 = s0 * up, w1 = s1 * up;
-            const uint32_t pb0 = movmatrix_trans(Mma::pack(pr[0] * w0, pr[1] * w0));
-            const uint32_t pb1 = movmatrix_trans(Mma::pack(pr[2] * w1, pr[3] * w1));
-            // ---- O^T += C_V^T . P'^T; m-tile mt holds columns 16 mt + 2 g4 (row g4) and
-            //      16 mt + 2 g4 + 1 (row g4 + 8)
+            // ---- (p * s_V * 2^E)^T as B operands (fp16): movmatrix.trans of the 8x8 blocks
+            //      of tokens 16 tau + 0-7 and 16 tau + 8-15
+            uint32_t pb[2][2];
+#pragma unroll
+            for (int tau = 0; tau < 2; ++tau) {
+                const float w0 = w[tau][0] * up, w1 = w[tau][1] * up;
+                pb[tau][0] = movmatrix_trans(Mma::pack(pr[tau][0] * w0, pr[tau][1] * w0));
+                pb[tau][1] = movmatrix_trans(Mma::pack(pr[tau][2] * w1, pr[tau][3] * w1));
+            }
+            // ---- O^T += C_V^T . P'^T over both tiles; m-tile mt holds columns 16 mt + 2 g4
+            //      (row g4) and 16 mt + 2 g4 + 1 (row g4 + 8)
 #pragma unroll
             for (int x = 0; x < KS / 2; ++x) {
-                uint32_t r[4];
-                ldmatrix_x4_trans(r, vb + lm_off + (((2 * x + lm_chunk) ^ lm_swz) * 16));
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {             // m-tile 2x + h: r[2h] tokens 0-7, r[2h+1] 8-15
-                    uint32_t a[4];
-                    i8_even_odd(r[2 * h], a[0], a[1]);
-                    i8_even_odd(r[2 * h + 1], a[2], a[3]);
-                    Mma::mma(oacc[2 * x + h], a, pb0, pb1);
+                for (int tau = 0; tau < 2; ++tau) {
+                    uint32_t r[4];
+                    ldmatrix_x4_trans(r, vb + tau * 16 * D + lm_off + (((2 * x + lm_chunk) ^ lm_swz) * 16));
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {         // m-tile 2x + h: r[2h] tokens 0-7, r[2h+1] 8-15
+                        uint32_t a[4];
+                        i8_even_odd(r[2 * h], a[0], a[1]);
+                        i8_even_odd(r[2 * h + 1], a[2], a[3]);
+                        Mma::mma(oacc[2 * x + h], a, pb[tau][0], pb[tau][1]);
+                    }
                 }
             }
             __syncwarp();

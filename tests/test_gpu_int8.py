@@ -145,6 +145,19 @@ def test_int8_row_scales_spanning_many_binades(dtype):
     assert pkv.kv_get_device_error() == 0
 
 
+@pytest.mark.parametrize("dtype,mean,mag", [("f16", 4.0, 1.0), ("bf16", 0.0, 2.0 ** 17), ("bf16", 3.0, 1.0)])
+def test_int8_biased_and_large_queries(dtype, mean, mag):
+    """q with a large common offset (sum_d q_d far from 0, which the K side subtracts after
+    the MMA) and bf16 q beyond fp16's range (scaled by a power of two per head row)."""
+    s = synth.random_spec(660, 3, 8, 2, 128, 16, [300, 47, 1500], dtype=dtype)
+    c = I8Case(s)
+    r = np.random.Generator(np.random.PCG64(661))
+    q = (r.standard_normal(c.q.shape, dtype=np.float32) + np.float32(mean)) * np.float32(mag / 8.0)
+    c.q = synth.round_f32(q, dtype)
+    _expect_close(c.gpu_layer(0), c.oracle_layer(0), dtype, "int8 q mean %g mag %g" % (mean, mag))
+    assert pkv.kv_get_device_error() == 0
+
+
 def test_int8_split_count_sweep():
     s = synth.random_spec(700, 5, 8, 8, 128, 16, [1000, 17, 300, 0, 2000])
     ref = None
