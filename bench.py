@@ -75,7 +75,7 @@ def measured_peaks():
 
 def kernel_source_digest():
     h = hashlib.sha256()
-    for name in ("decode_attention.cuh", "pkv_device.cuh"):
+    for name in ("decode_attention.cuh", "decode_attention_mma.cuh", "decode_attention_i8.cuh", "pkv_device.cuh"):
         with open(os.path.join(ROOT, "paged_kv_cache_460_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
