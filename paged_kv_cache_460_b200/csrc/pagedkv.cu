@@ -435,9 +435,10 @@ extern "C" int paged_prefill_attention(const pkv_pool* pool, int layer, void* ou
     prm.kv_heads = kv_heads;
     prm.num_pages = pool->num_pages;
     prm.scale_log2 = scale * 1.4426950408889634f;
-    // work items: kv_heads * sum_b ceil(n_b * group / 16) <= kv_heads * ((total_q * group + 15 * batch) / 16 + 1)
-    const long long bound = (long long)kv_heads * (((long long)total_q * group + 15LL * batch) / 16 + 1);
-    const long long grid = (bound + kPrefillWarps - 1) / kPrefillWarps;
+    // work items (one CTA each): kv_heads * sum_b ceil(n_b * group / R), R = kPrefillRows,
+    // at most kv_heads * ((total_q * group + (R - 1) * batch) / R + 1)
+    const long long grid = (long long)kv_heads *
+                           (((long long)total_q * group + (long long)(kPrefillRows - 1) * batch) / kPrefillRows + 1);
     if (grid > 0x7fffffffLL) return PKV_ERR_UNSUPPORTED;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (pool->dtype == PKV_F16)

@@ -6,17 +6,18 @@
 // sees keys 0 .. start_pos + i.  With a chunk of rows the contraction is dense (16 query
 // rows per MMA), unlike the single-row decode step.
 //
-// Work: one warp per (sequence, kv head, tile of 16 MMA rows), a row being one (query
-// token, query head of the group) pair, so a tile holds 16 / G tokens x G heads.  The
-// warp streams the key units (16 rows of K and V) that the tile's last token can see,
-// 0 .. pos_max, through its own cp.async ring (chunks XOR-swizzled as in the decode
-// tensor-core kernel), and per unit computes
-//   S[16 rows x 16 keys] = Q . K^T      (2 x D/16 mma.sync m16n8k16)
+// Work: one CTA per (sequence, kv head, tile of 64 MMA rows), a row being one (query
+// token, query head of the group) pair; warp w owns rows 16w .. 16w + 15.  The CTA streams
+// the blocks of 64 keys that its last token can see through a two-stage shared-memory ring
+// that all 128 threads fill with 16-byte cp.async copies (keys past the cache are
+// zero-filled by the copy itself) and all four warps read, so a K/V block crosses the
+// memory system once per 64 rows instead of once per 16.  Per block each warp computes
+//   S[16 rows x 64 keys] = Q . K^T      (8 x D/16 mma.sync m16n8k16)
 //   causal mask, fp32 online softmax per row (log2 domain)
-//   O[16 x D] += P . V                 (D/8 MMAs; P from the S accumulators in registers,
-//                                        bf16 P as hi + lo)
+//   O[16 x D] += P . V                 (4 x D/8 MMAs; P from the S accumulators in
+//                                        registers, bf16 P as hi + lo)
 // and finally writes O / l.  Rows past the chunk and keys past a row's position are
-// masked; V rows past the cached length are zeroed before they meet a zero weight.
+// masked; a warp whose rows all end before a block skips it (it still joins the barriers).
 #ifndef PKV_PREFILL_ATTENTION_CUH_
 #define PKV_PREFILL_ATTENTION_CUH_
 
@@ -28,7 +29,8 @@ namespace pkv {
 
 constexpr int kPrefillWarps = 4;
 constexpr int kPrefillThreads = kPrefillWarps * 32;
-constexpr int kPrefillDepth = 2;
+constexpr int kPrefillRows = kPrefillWarps * 16;   // MMA rows per CTA
+constexpr int kPrefillKeys = 64;                    // keys per ring stage
 
 struct PrefillParams {
     const void* k;                 // this layer's K pool [pages][kv_heads][P][D]
@@ -48,45 +50,51 @@ struct PrefillParams {
 
 template <int D>
 struct PrefillShape {
-    static constexpr int kUnit = 16 * D * 2;                 // bytes of 16 K (or V) rows
-    static constexpr int kSlot = 2 * kUnit;
-    static constexpr int kRingBytes = kPrefillWarps * kPrefillDepth * kSlot;
+    static constexpr int kBlock = kPrefillKeys * D * 2;      // bytes of 64 K (or V) rows
+    static constexpr int kStage = 2 * kBlock;
+    static constexpr int kRingBytes = 2 * kStage;
     static constexpr int kScanOffset = kRingBytes;            // item prefix [batch + 1]
     static int smem_bytes(int batch) { return kScanOffset + 4 * (batch + 1); }
 };
 
+// 16-byte cp.async that writes zeros instead when `valid` is false (src-size 0: nothing is
+// read from `src`, which must still be a mapped address).
+__device__ __forceinline__ void cp_async16_zfill(void* dst, const void* src, bool valid)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(dst)), "l"(src),
+                 "r"(valid ? 16u : 0u)
+                 : "memory");
+}
+
 template <int D, int P, int G, typename T>
-__global__ void __launch_bounds__(kPrefillThreads) prefill_attention_kernel(const PrefillParams p)
+__global__ void __launch_bounds__(kPrefillThreads, 3) prefill_attention_kernel(const PrefillParams p)
 {
     using S = PrefillShape<D>;
-    constexpr int DEPTH = kPrefillDepth;
-    constexpr int CPR = D / 8;
-    constexpr int U = P / 16;              // key units per page
+    constexpr int CPR = D / 8;             // 16-byte chunks per row
     constexpr int KS = D / 16;             // k-steps of Q.K^T
     constexpr int ND = D / 8;              // n-tiles of O
-    constexpr int TT = 16 / G;             // query tokens per tile
+    constexpr int CT = kPrefillRows / G;   // query tokens per CTA tile
+    constexpr int NKC = kPrefillKeys * CPR / kPrefillThreads;   // chunks per thread per block (K or V)
     static_assert(G >= 1 && G <= 16 && 16 % G == 0, "group size");
     extern __shared__ __align__(128) unsigned char smem[];
     int* items = reinterpret_cast<int*>(smem + S::kScanOffset);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int Hkv = p.kv_heads;
 
-    // prefix of work items over the sequences: Hkv * ceil(n_b * G / 16) per sequence
-    for (int b = threadIdx.x; b <= p.batch; b += blockDim.x) items[b] = 0;
-    __syncthreads();
-    if (threadIdx.x == 0) {
+    // prefix of work items over the sequences: Hkv * ceil(n_b * G / 64) per sequence
+    if (tid == 0) {
         int run = 0;
         for (int b = 0; b < p.batch; ++b) {
             items[b] = run;
             const int n = p.cu_q[b + 1] - p.cu_q[b];
-            run += n > 0 ? Hkv * ((n * G + 15) / 16) : 0;
+            run += n > 0 ? Hkv * ((n * G + kPrefillRows - 1) / kPrefillRows) : 0;
         }
         items[p.batch] = run;
     }
     __syncthreads();
     pdl_wait();
     pdl_launch_dependents();
-    const int item = blockIdx.x * kPrefillWarps + warp;
+    const int item = blockIdx.x;
     if (item >= items[p.batch]) return;
     int lo = 0, hi = p.batch - 1;         // sequence of the item: largest b with items[b] <= item
     while (lo < hi) {
@@ -96,24 +104,26 @@ __global__ void __launch_bounds__(kPrefillThreads) prefill_attention_kernel(cons
     }
     const int b = lo;
     const int q0 = p.cu_q[b], n_b = p.cu_q[b + 1] - q0;
-    const int tiles = (n_b * G + 15) / 16;
+    const int tiles = (n_b * G + kPrefillRows - 1) / kPrefillRows;
     const int g = (item - items[b]) / tiles, tile = (item - items[b]) % tiles;
     const int L = p.context_lens[b];
     const int start = L - n_b;
-    const int last_tok = min(n_b - 1, tile * TT + TT - 1);
-    const int n_units = (start + last_tok) / 16 + 1;   // keys 0 .. position of the tile's last token
+    const int cta_last = min(n_b - 1, tile * CT + CT - 1);
+    const int n_blocks = (start + cta_last) / kPrefillKeys + 1;   // keys 0 .. position of the CTA's last token
 
     const int g4 = lane >> 2, t4 = lane & 3;
-    // rows of this thread: r = g4 and g4 + 8 -> token tile * TT + r / G, head r % G
+    // rows of this thread: r = 16 warp + g4 (+ 8) -> token tile * CT + r / G, head r % G
     int tok[2], pos[2];
     bool rvalid[2];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-        const int r = g4 + 8 * h;
-        tok[h] = tile * TT + r / G;
+        const int r = 16 * warp + g4 + 8 * h;
+        tok[h] = tile * CT + r / G;
         rvalid[h] = tok[h] < n_b;
         pos[h] = rvalid[h] ? start + tok[h] : -1;
     }
+    const int warp_first = tile * CT + (16 * warp) / G;
+    const int warp_maxpos = warp_first < n_b ? start + min(n_b - 1, tile * CT + (16 * warp + 15) / G) : -1;
     // Q as A fragments (rows x d)
     uint32_t qa[KS][4];
 #pragma unroll
@@ -128,38 +138,36 @@ __global__ void __launch_bounds__(kPrefillThreads) prefill_attention_kernel(cons
         }
     }
 
-    // ---- per-warp ring of key units
-    unsigned char* ring = smem + warp * DEPTH * S::kSlot;
-    int win = 0, win0 = -1;
-    auto issue = [&](int u) {
-        if (win0 < 0 || u >= win0 + 32) {
-            win0 = u;
-            const int pg = (u + lane) / U;
-            win = (u + lane < n_units && pg < p.max_pages) ? p.block_tables[(long long)b * p.max_pages + pg] : -1;
-        }
-        const int page = __shfl_sync(0xffffffffu, win, u - win0);
-        unsigned char* slot = ring + (u % DEPTH) * S::kSlot;
-        if ((unsigned)page < (unsigned)p.num_pages) {
-            const long long off = (((long long)page * Hkv + g) * P + (u % U) * 16) * D;
-            const unsigned char* ks = reinterpret_cast<const unsigned char*>(static_cast<const T*>(p.k) + off);
-            const unsigned char* vs = reinterpret_cast<const unsigned char*>(static_cast<const T*>(p.v) + off);
+    // ---- the CTA's two-stage ring of 64-key blocks (K then V, rows XOR-swizzled by chunk)
+    const int32_t* table = p.block_tables + (long long)b * p.max_pages;
+    auto issue = [&](int blk, int st) {
+        unsigned char* kd = smem + st * S::kStage;
 #pragma unroll
-            for (int n = 0; n < S::kUnit / 512; ++n) {
-                const int gidx = n * 32 + lane;
-                const int t = gidx / CPR, c = gidx % CPR;
-                const int dst = t * (2 * D) + ((c ^ (t & 7)) * 16);
-                cp_async16(slot + dst, ks + gidx * 16);
-                cp_async16(slot + S::kUnit + dst, vs + gidx * 16);
+        for (int n = 0; n < NKC; ++n) {
+            const int idx = n * kPrefillThreads + tid;
+            const int t = idx / CPR, c = idx % CPR;
+            const int key = blk * kPrefillKeys + t;
+            bool valid = key < L;
+            long long off = 0;
+            if (valid) {
+                const int pg = key / P;
+                const int page = pg < p.max_pages ? table[pg] : -1;
+                if ((unsigned)page < (unsigned)p.num_pages) {
+                    off = (((long long)page * Hkv + g) * P + key % P) * D + c * 8;
+                } else {
+                    valid = false;
+                    if (c == 0) atomicOr(&g_error_word, PKV_DEVERR_BAD_PAGE);   // never dereferenced
+                }
             }
-        } else if (lane == 0) {
-            atomicOr(&g_error_word, PKV_DEVERR_BAD_PAGE);   // never dereferenced
+            const int dst = t * (2 * D) + ((c ^ (t & 7)) * 16);
+            cp_async16_zfill(kd + dst, static_cast<const T*>(p.k) + off, valid);
+            cp_async16_zfill(kd + S::kBlock + dst, static_cast<const T*>(p.v) + off, valid);
         }
     };
-#pragma unroll
-    for (int u = 0; u < DEPTH; ++u) {
-        if (u < n_units) issue(u);
-        cp_async_commit();
-    }
+    issue(0, 0);
+    cp_async_commit();
+    if (n_blocks > 1) issue(1, 1);
+    cp_async_commit();
 
     float oacc[ND][4], m_run[2], l_run[2];
 #pragma unroll
@@ -172,96 +180,99 @@ __global__ void __launch_bounds__(kPrefillThreads) prefill_attention_kernel(cons
     const int vb_row = (lane & 7) + 8 * ((lane >> 3) & 1), vb_hi = lane >> 4;      // V as B^T (keys x d)
     constexpr bool kSplitP = std::is_same<T, __nv_bfloat16>::value;
 
-    for (int u = 0; u < n_units; ++u) {
-        cp_async_wait<DEPTH - 1>();
-        __syncwarp();
-        unsigned char* s = ring + (u % DEPTH) * S::kSlot;
-        const int kvalid = min(16, L - u * 16);
-        if (kvalid < 16) {                    // rows past the cache: zero V (weights are 0 there)
-            for (int x = lane; x < (16 - kvalid) * CPR; x += 32)
-                reinterpret_cast<uint4*>(s + S::kUnit + kvalid * (2 * D))[x] = make_uint4(0, 0, 0, 0);
-            __syncwarp();
-        }
-        // ---- S = Q . K^T for the unit's 16 keys (two n-tiles of 8 keys)
-        float sacc[2][4];
+    for (int blk = 0; blk < n_blocks; ++blk) {
+        cp_async_wait<1>();
+        __syncthreads();                      // block blk visible to every warp
+        const unsigned char* ks = smem + (blk & 1) * S::kStage;
+        const unsigned char* vs = ks + S::kBlock;
+        if (blk * kPrefillKeys <= warp_maxpos) {
+            // ---- S = Q . K^T for the block's 64 keys (eight n-tiles of 8 keys)
+            float sacc[8][4];
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
+            for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
+                for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
 #pragma unroll
-        for (int kk = 0; kk < KS; ++kk) {
-            uint32_t kb[4];
-            const int ch = 2 * kk + kb_hi;
-            ldmatrix_x4(kb, s + kb_row * (2 * D) + ((ch ^ (kb_row & 7)) * 16));
-            MmaOps<T>::mma(sacc[0], qa[kk], kb[0], kb[1]);
-            MmaOps<T>::mma(sacc[1], qa[kk], kb[2], kb[3]);
-        }
-        // ---- causal mask and online softmax per row (rows g4: e = 0,1; g4 + 8: e = 2,3)
-        float alpha[2];
+            for (int j = 0; j < 4; ++j) {
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            float mx = -INFINITY;
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    const int key = u * 16 + nt * 8 + 2 * t4 + c;
-                    float& sv = sacc[nt][2 * h + c];
-                    sv = key <= pos[h] ? sv * p.scale_log2 : -INFINITY;
-                    mx = fmaxf(mx, sv);
+                for (int kk = 0; kk < KS; ++kk) {
+                    uint32_t kb[4];
+                    const int ch = 2 * kk + kb_hi;
+                    ldmatrix_x4(kb, ks + (16 * j + kb_row) * (2 * D) + ((ch ^ (kb_row & 7)) * 16));
+                    MmaOps<T>::mma(sacc[2 * j], qa[kk], kb[0], kb[1]);
+                    MmaOps<T>::mma(sacc[2 * j + 1], qa[kk], kb[2], kb[3]);
                 }
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-            const float mn = fmaxf(m_run[h], mx);
-            const bool none = mn == -INFINITY;       // row past the chunk: keep it empty
-            alpha[h] = none ? 1.f : fast_exp2(m_run[h] - mn);
-            m_run[h] = mn;
-            float ls = 0.f;
+            }
+            // ---- causal mask and online softmax per row (rows g4: e = 0,1; g4 + 8: e = 2,3)
+            float alpha[2];
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
+            for (int h = 0; h < 2; ++h) {
+                float mx = -INFINITY;
 #pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    float& sv = sacc[nt][2 * h + c];
-                    sv = none ? 0.f : fast_exp2(sv - mn);
-                    ls += sv;
+                for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        const int key = blk * kPrefillKeys + nt * 8 + 2 * t4 + c;
+                        float& sv = sacc[nt][2 * h + c];
+                        sv = key <= pos[h] ? sv * p.scale_log2 : -INFINITY;
+                        mx = fmaxf(mx, sv);
+                    }
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+                const float mn = fmaxf(m_run[h], mx);
+                const bool none = mn == -INFINITY;       // row past the chunk: keep it empty
+                alpha[h] = none ? 1.f : fast_exp2(m_run[h] - mn);
+                m_run[h] = mn;
+                float ls = 0.f;
+#pragma unroll
+                for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        float& sv = sacc[nt][2 * h + c];
+                        sv = none ? 0.f : fast_exp2(sv - mn);
+                        ls += sv;
+                    }
+                l_run[h] = l_run[h] * alpha[h] + ls;
+            }
+#pragma unroll
+            for (int n = 0; n < ND; ++n) {
+                oacc[n][0] *= alpha[0];
+                oacc[n][1] *= alpha[0];
+                oacc[n][2] *= alpha[1];
+                oacc[n][3] *= alpha[1];
+            }
+            // ---- O += P . V, 16 keys at a time (P as A fragments; bf16 P as hi + lo)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                uint32_t pa[4], pl[4];
+                pa[0] = MmaOps<T>::pack(sacc[2 * j][0], sacc[2 * j][1]);
+                pa[1] = MmaOps<T>::pack(sacc[2 * j][2], sacc[2 * j][3]);
+                pa[2] = MmaOps<T>::pack(sacc[2 * j + 1][0], sacc[2 * j + 1][1]);
+                pa[3] = MmaOps<T>::pack(sacc[2 * j + 1][2], sacc[2 * j + 1][3]);
+                if constexpr (kSplitP) {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float* sv = &sacc[2 * j + (i >> 1)][2 * (i & 1)];
+                        pl[i] = MmaOps<T>::pack(sv[0] - __uint_as_float(pa[i] << 16),
+                                                sv[1] - __uint_as_float(pa[i] & 0xffff0000u));
+                    }
                 }
-            l_run[h] = l_run[h] * alpha[h] + ls;
-        }
 #pragma unroll
-        for (int n = 0; n < ND; ++n) {
-            oacc[n][0] *= alpha[0];
-            oacc[n][1] *= alpha[0];
-            oacc[n][2] *= alpha[1];
-            oacc[n][3] *= alpha[1];
-        }
-        // ---- P as A fragments (rows x 16 keys); bf16 P as hi + lo
-        uint32_t pa[4], pl[4];
-        pa[0] = MmaOps<T>::pack(sacc[0][0], sacc[0][1]);
-        pa[1] = MmaOps<T>::pack(sacc[0][2], sacc[0][3]);
-        pa[2] = MmaOps<T>::pack(sacc[1][0], sacc[1][1]);
-        pa[3] = MmaOps<T>::pack(sacc[1][2], sacc[1][3]);
-        if constexpr (kSplitP) {
-            const float* sv = &sacc[0][0];
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                pl[i] = MmaOps<T>::pack(sv[2 * i] - __uint_as_float(pa[i] << 16),
-                                        sv[2 * i + 1] - __uint_as_float(pa[i] & 0xffff0000u));
-        }
-        // ---- O += P . V (two n-tiles of 8 columns per ldmatrix)
-#pragma unroll
-        for (int jt = 0; jt < ND / 2; ++jt) {
-            uint32_t vb[4];
-            const int ch = 2 * jt + vb_hi;
-            ldmatrix_x4_trans(vb, s + S::kUnit + vb_row * (2 * D) + ((ch ^ (vb_row & 7)) * 16));
-            MmaOps<T>::mma(oacc[2 * jt], pa, vb[0], vb[1]);
-            MmaOps<T>::mma(oacc[2 * jt + 1], pa, vb[2], vb[3]);
-            if constexpr (kSplitP) {
-                MmaOps<T>::mma(oacc[2 * jt], pl, vb[0], vb[1]);
-                MmaOps<T>::mma(oacc[2 * jt + 1], pl, vb[2], vb[3]);
+                for (int jt = 0; jt < ND / 2; ++jt) {
+                    uint32_t vb[4];
+                    const int ch = 2 * jt + vb_hi;
+                    ldmatrix_x4_trans(vb, vs + (16 * j + vb_row) * (2 * D) + ((ch ^ (vb_row & 7)) * 16));
+                    MmaOps<T>::mma(oacc[2 * jt], pa, vb[0], vb[1]);
+                    MmaOps<T>::mma(oacc[2 * jt + 1], pa, vb[2], vb[3]);
+                    if constexpr (kSplitP) {
+                        MmaOps<T>::mma(oacc[2 * jt], pl, vb[0], vb[1]);
+                        MmaOps<T>::mma(oacc[2 * jt + 1], pl, vb[2], vb[3]);
+                    }
+                }
             }
         }
-        __syncwarp();
-        if (u + DEPTH < n_units) issue(u + DEPTH);
+        __syncthreads();                      // every warp is done with this stage
+        if (blk + 2 < n_blocks) issue(blk + 2, blk & 1);
         cp_async_commit();
     }
     cp_async_wait<0>();
