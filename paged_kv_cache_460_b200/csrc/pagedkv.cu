@@ -15,7 +15,7 @@
 #include "decode_attention.cuh"
 #include "decode_attention_i8.cuh"
 #include "decode_attention_mma.cuh"
-#include "prefill_attention.cuh"
+#include "prefill_attention_tc.cuh"
 #include "pagedkv.h"
 #include "pkv_internal.h"
 #include "rms_norm.cuh"
@@ -374,11 +374,11 @@ template <int D, int P, int G, typename T>
 int launch_prefill(const PrefillParams& prm, int grid, cudaStream_t st)
 {
     static int configured[kMaxDevices] = {0};
-    const int smem = PrefillShape<D>::smem_bytes(prm.batch);
+    using S = TcShape<D, std::is_same<T, __nv_bfloat16>::value>;
+    const int smem = S::kBytes + 4 * (prm.batch + 1);
     if (smem > kMaxSmemPerCta) return PKV_ERR_UNSUPPORTED;
-    if (ensure_smem(prefill_attention_kernel<D, P, G, T>, smem, configured) != cudaSuccess) return PKV_ERR_CUDA;
-    return status_of(launch_pdl(prefill_attention_kernel<D, P, G, T>, dim3(grid), dim3(kPrefillThreads), smem, st,
-                                prm));
+    if (ensure_smem(prefill_tc_kernel<D, P, G, T>, smem, configured) != cudaSuccess) return PKV_ERR_CUDA;
+    return status_of(launch_pdl(prefill_tc_kernel<D, P, G, T>, dim3(grid), dim3(kTcRows), smem, st, prm));
 }
 
 template <int D, int P, typename T>
@@ -435,10 +435,10 @@ extern "C" int paged_prefill_attention(const pkv_pool* pool, int layer, void* ou
     prm.kv_heads = kv_heads;
     prm.num_pages = pool->num_pages;
     prm.scale_log2 = scale * 1.4426950408889634f;
-    // work items (one CTA each): kv_heads * sum_b ceil(n_b * group / R), R = kPrefillRows,
+    // work items (one CTA each): kv_heads * sum_b ceil(n_b * group / R), R = kTcRows,
     // at most kv_heads * ((total_q * group + (R - 1) * batch) / R + 1)
     const long long grid = (long long)kv_heads *
-                           (((long long)total_q * group + (long long)(kPrefillRows - 1) * batch) / kPrefillRows + 1);
+                           (((long long)total_q * group + (long long)(kTcRows - 1) * batch) / kTcRows + 1);
     if (grid > 0x7fffffffLL) return PKV_ERR_UNSUPPORTED;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (pool->dtype == PKV_F16)

@@ -1,0 +1,379 @@
+// Chunked prefill attention over the paged KV cache on the fifth-generation tensor cores.
+//
+// "为什么要自己动手写一个LLM推理引擎" (wzjinhao.cn/news/61427) s4.3: the forward of a chunk
+// of seq_len new tokens at start_pos appends their k, v to the cache and applies the
+// causal mask slice [start_pos : start_pos + seq_len, : start_pos + seq_len] -- query row i
+// sees keys 0 .. start_pos + i.  A chunk makes the contraction dense, so it runs on
+// tcgen05: one elected thread issues the MMAs, operands come from shared memory, the
+// accumulators live in tensor memory (TMEM).
+//
+// Work: one CTA of 128 threads per (sequence, kv head, tile of 128 rows), a row being one
+// (query token, query head of the group) pair; thread t owns row t (TMEM lane t).  Per
+// block of NK keys (64 for fp16; 32 for bf16, whose P takes two buffers):
+//   S[128 x NK] = Q . K^T          tcgen05.mma kind::f16, M 128, N NK, D/16 k-steps -> TMEM
+//   each thread: its S row from TMEM, causal mask, fp32 online softmax (log2 domain), its
+//                O row rescaled in TMEM when its warp's running max moved, its P row
+//                written to shared memory
+//   O[128 x D] += P . V            M 128, N D, NK/16 k-steps (bf16: P as hi + lo, twice)
+// Shared memory uses the 128-byte-swizzle canonical layouts: Q, K and P K-major (rows of
+// 128 bytes, 16-byte chunk c of row r at c ^ (r & 7), 8-row atoms 1024 bytes apart, a
+// region per 64 columns), V MN-major -- which is the same bytes as K's layout read with
+// the other major-ness, so K and V blocks are staged identically by cp.async from the
+// pages (keys past the cache zero-filled by the copy).  K and V blocks go through rings of
+// their own (two stages each): K(b) is refilled as soon as S(b) is done, V(b) as soon as
+// P.V(b) is, so each load has an iteration to land; and the elected thread issues S of the
+// next block before P.V of the current one (each with its own commit), so the next softmax
+// can start while P.V is still on the tensor cores.  Every wait on
+// an MMA is bounded: on timeout the kernel sets PKV_DEVERR_TIMEOUT, skips its output and
+// still frees its TMEM.
+#ifndef PKV_PREFILL_ATTENTION_TC_CUH_
+#define PKV_PREFILL_ATTENTION_TC_CUH_
+
+#include <cuda/ptx>
+#include <type_traits>
+
+#include "prefill_attention.cuh"
+
+namespace pkv {
+
+constexpr int kTcRows = 128;          // query rows per CTA (= threads = TMEM lanes)
+template <int D, bool kSplitP>
+struct TcShape {
+    static constexpr int kKeys = kSplitP ? 32 : 64;             // keys per block
+    static constexpr int kQBytes = kTcRows * D * 2;             // Q, D/64 regions of 128 rows x 128 B
+    static constexpr int kRegion = kKeys * 128;                 // one 64-column region of a K (or V) block
+    static constexpr int kKvBytes = (D / 64) * kRegion;         // one K (or V) block
+    static constexpr int kPBytes = kTcRows * 128;               // one P buffer: 128 rows of 128 B
+    static constexpr int kQOff = 0;
+    static constexpr int kKOff = kQOff + kQBytes;               // K ring, 2 stages
+    static constexpr int kVOff = kKOff + 2 * kKvBytes;          // V ring, 2 stages
+    static constexpr int kPOff = kVOff + 2 * kKvBytes;
+    static constexpr int kBarOff = kPOff + (kSplitP ? 2 : 1) * kPBytes;
+    static constexpr int kBytes = kBarOff + 64;                 // 2 mbarriers, TMEM base, abort flag
+    static constexpr uint32_t kTmemCols = D + kKeys <= 128 ? 128u : 256u;   // O at 0, S at D
+};
+
+// UMMA shared-memory descriptor, 128-byte swizzle (start, leading and stride byte offsets)
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo)
+{
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// kind::f16 instruction descriptor: fp32 accumulator, A and B of the element type,
+// A K-major, B K-major or MN-major, M x N
+template <typename T>
+__host__ __device__ constexpr uint32_t umma_idesc(int m, int n, bool b_mn_major)
+{
+    constexpr uint32_t fmt = std::is_same<T, __nv_bfloat16>::value ? 1u : 0u;
+    return (1u << 4) | (fmt << 7) | (fmt << 10) | ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(n >> 3) << 17) |
+           ((uint32_t)(m >> 4) << 24);
+}
+
+__device__ __forceinline__ bool mbar_wait_parity_bounded(uint64_t* bar, uint32_t parity)
+{
+    const long long t0 = clock64();
+    for (;;) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (clock64() - t0 > kWaitLimitCycles) return false;
+    }
+}
+
+template <int D, int P, int G, typename T>
+__global__ void __launch_bounds__(kTcRows, 1) prefill_tc_kernel(const PrefillParams p)
+{
+    namespace ptx = cuda::ptx;
+    constexpr bool kSplitP = std::is_same<T, __nv_bfloat16>::value;
+    using S = TcShape<D, kSplitP>;
+    constexpr int CPR = D / 8;                 // 16-byte chunks per row
+    constexpr int KS = D / 16;                 // k-steps of Q.K^T
+    constexpr int CT = kTcRows / G;            // query tokens per CTA tile
+    constexpr int NK = S::kKeys;               // keys per block
+    constexpr int NKC = NK * CPR / kTcRows;    // chunks per thread per K (or V) block
+    static_assert(G >= 1 && G <= 16 && 16 % G == 0, "group size");
+    static_assert(D == 64 || D == 128, "head_dim");
+    extern __shared__ __align__(1024) unsigned char smem[];
+    const int tid = threadIdx.x, warp = tid >> 5;
+    uint64_t* bar_s = reinterpret_cast<uint64_t*>(smem + S::kBarOff);
+    uint64_t* bar_o = bar_s + 1;
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + S::kBarOff + 16);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S::kBarOff + 20);
+    int* items = reinterpret_cast<int*>(smem + S::kBytes);   // [batch + 1] after the fixed part
+    const int Hkv = p.kv_heads;
+
+    if (tid == 0) {
+        int run = 0;
+        for (int b = 0; b < p.batch; ++b) {
+            items[b] = run;
+            const int n = p.cu_q[b + 1] - p.cu_q[b];
+            run += n > 0 ? Hkv * ((n * G + kTcRows - 1) / kTcRows) : 0;
+        }
+        items[p.batch] = run;
+        *abort_flag = (smem_addr(smem) & 1023u) != 0;     // the swizzle atoms need 1024-byte alignment
+    }
+    __syncthreads();
+    pdl_wait();
+    pdl_launch_dependents();
+    const int item = blockIdx.x;
+    if (item >= items[p.batch] || *abort_flag) {
+        if (tid == 0 && *abort_flag) atomicOr(&g_error_word, PKV_DEVERR_TIMEOUT);
+        return;
+    }
+    int lo = 0, hi = p.batch - 1;               // sequence of the item
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (items[mid] <= item) lo = mid;
+        else hi = mid - 1;
+    }
+    const int b = lo;
+    const int q0 = p.cu_q[b], n_b = p.cu_q[b + 1] - q0;
+    const int tiles = (n_b * G + kTcRows - 1) / kTcRows;
+    const int g = (item - items[b]) / tiles;
+    const int tile = tiles - 1 - (item - items[b]) % tiles;     // later (longer) tiles first
+    const int L = p.context_lens[b];
+    const int start = L - n_b;
+    const int cta_last = min(n_b - 1, tile * CT + CT - 1);
+    const int n_blocks = (start + cta_last) / NK + 1;
+
+    // this thread's row
+    const int tok = tile * CT + tid / G;
+    const bool rvalid = tok < n_b;
+    const int pos = rvalid ? start + tok : -1;
+
+    unsigned char* qs = smem + S::kQOff;
+    unsigned char* kring = smem + S::kKOff;
+    unsigned char* vring = smem + S::kVOff;
+    unsigned char* ps = smem + S::kPOff;
+    // ---- Q row -> shared memory (K-major, swizzled); rows past the chunk are zero
+    {
+        const uint4* src = reinterpret_cast<const uint4*>(
+            static_cast<const T*>(p.q) + ((long long)(q0 + (rvalid ? tok : 0)) * p.q_heads + g * G + tid % G) * D);
+#pragma unroll
+        for (int c = 0; c < CPR; ++c) {
+            const uint4 v = rvalid ? src[c] : make_uint4(0u, 0u, 0u, 0u);
+            *reinterpret_cast<uint4*>(qs + (c / 8) * (kTcRows * 128) + tid * 128 + (((c % 8) ^ (tid & 7)) * 16)) = v;
+        }
+    }
+    // ---- K or V block loads (the same swizzled layout for both; keys past the cache are zero)
+    const int32_t* table = p.block_tables + (long long)b * p.max_pages;
+    auto load_block = [&](const void* pool, unsigned char* dst_block, int blk) {
+#pragma unroll
+        for (int n = 0; n < NKC; ++n) {
+            const int idx = n * kTcRows + tid;
+            const int t = idx / CPR, c = idx % CPR;
+            const int key = blk * NK + t;
+            bool valid = key < L;
+            long long off = 0;
+            if (valid) {
+                const int pg = key / P;
+                const int page = pg < p.max_pages ? table[pg] : -1;
+                if ((unsigned)page < (unsigned)p.num_pages) {
+                    off = (((long long)page * Hkv + g) * P + key % P) * D + c * 8;
+                } else {
+                    valid = false;
+                    if (c == 0) atomicOr(&g_error_word, PKV_DEVERR_BAD_PAGE);   // never dereferenced
+                }
+            }
+            const int dst = (c / 8) * S::kRegion + t * 128 + (((c % 8) ^ (t & 7)) * 16);
+            cp_async16_zfill(dst_block + dst, static_cast<const T*>(pool) + off, valid);
+        }
+    };
+    auto load_k = [&](int blk) { if (blk < n_blocks) load_block(p.k, kring + (blk & 1) * S::kKvBytes, blk); };
+    auto load_v = [&](int blk) { if (blk < n_blocks) load_block(p.v, vring + (blk & 1) * S::kKvBytes, blk); };
+    // cp.async groups, in commit order: K0, V0, K1, then per iteration blk: K(blk+2), V(blk+1)
+    load_k(0);
+    cp_async_commit();
+    load_v(0);
+    cp_async_commit();
+    load_k(1);
+    cp_async_commit();
+
+    // ---- TMEM and barriers
+    const uint32_t tmem_cols = S::kTmemCols;
+    if (warp == 0) {
+        ptx::tcgen05_alloc(ptx::cta_group_1, tslot, tmem_cols);
+        ptx::tcgen05_relinquish_alloc_permit(ptx::cta_group_1);
+    }
+    if (tid == 0) {
+        mbar_init(bar_s, 1);
+        mbar_init(bar_o, 1);
+        fence_barrier_init();
+    }
+    const uint32_t idesc_s = umma_idesc<T>(kTcRows, NK, false);
+    const uint32_t idesc_o = umma_idesc<T>(kTcRows, D, true);
+    // S = Q . K^T of block blk into the S columns
+    auto issue_s = [&](int blk, uint32_t tm) {
+        const unsigned char* ks = kring + (blk & 1) * S::kKvBytes;
+#pragma unroll
+        for (int kk = 0; kk < KS; ++kk) {
+            const uint64_t ad = umma_desc_sw128(smem_addr(qs) + (kk / 4) * (kTcRows * 128) + (kk % 4) * 32, 16, 1024);
+            const uint64_t bd = umma_desc_sw128(smem_addr(ks) + (kk / 4) * S::kRegion + (kk % 4) * 32, 16, 1024);
+            ptx::tcgen05_mma(ptx::kind_f16, ptx::cta_group_1, tm + D, ad, bd, idesc_s, kk > 0);
+        }
+        ptx::tcgen05_commit(ptx::cta_group_1, bar_s);
+    };
+    cp_async_wait<2>();                          // K0 landed (V0, K1 may be in flight)
+    fence_proxy_async_smem();
+    ptx::tcgen05_fence_before_thread_sync();
+    __syncthreads();                             // Q, block 0, TMEM base and barriers ready
+    ptx::tcgen05_fence_after_thread_sync();
+    const uint32_t tmem = *tslot;
+    const uint32_t t_row = tmem + ((uint32_t)(32 * warp) << 16);     // this warp's lane quarter
+    if (tid == 0) issue_s(0, tmem);
+
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    int timed_out = 0;                           // this thread gave up on a wait; every exit is decided
+                                                 // by a barrier over all threads, so it is uniform
+    for (int blk = 0; blk < n_blocks; ++blk) {
+        // ---- S of this block from TMEM
+        if (!mbar_wait_parity_bounded(bar_s, blk & 1)) {
+            timed_out = 1;
+            atomicOr(&g_error_word, PKV_DEVERR_TIMEOUT);
+        }
+        ptx::tcgen05_fence_after_thread_sync();
+        float sv[NK];
+#pragma unroll
+        for (int j = 0; j < NK / 32; ++j) {
+            uint32_t r[32];
+            ptx::tcgen05_ld_32x32b(r, t_row + D + 32 * j);
+            ptx::tcgen05_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) sv[32 * j + i] = __uint_as_float(r[i]);
+        }
+        // K stage blk & 1 is free again (S(blk) is done): fetch K(blk + 2) into it
+        load_k(blk + 2);
+        cp_async_commit();
+        // ---- causal mask and online softmax of this thread's row.  The running max is
+        //      taken over the raw scores (max of s * c is max(s) * c for c > 0, min(s) * c
+        //      otherwise) and each p is exp2(s * c - m) with one packed FMA per pair.
+        const float sc = p.scale_log2 != 0.f ? p.scale_log2 : 1e-30f;   // zero: uniform weights, no 0 * inf
+        const float sgn_inf = sc >= 0.f ? -INFINITY : INFINITY;   // a masked score's raw value
+        if (__any_sync(0xffffffffu, blk * NK + NK - 1 > pos)) {   // some key of the block is past a row
+#pragma unroll
+            for (int i = 0; i < NK; ++i) sv[i] = blk * NK + i <= pos ? sv[i] : sgn_inf;
+        }
+        float ext = sgn_inf;
+        if (sc >= 0.f) {
+#pragma unroll
+            for (int i = 0; i < NK; ++i) ext = fmaxf(ext, sv[i]);
+        } else {
+#pragma unroll
+            for (int i = 0; i < NK; ++i) ext = fminf(ext, sv[i]);
+        }
+        const float mx = ext * sc;                 // -inf when every key of the block is masked
+        const float mn = fmaxf(m_run, mx);
+        const bool none = mn == -INFINITY;       // no visible key yet (or a row past the chunk)
+        const float alpha = none ? 1.f : fast_exp2(m_run - mn);
+        m_run = mn;
+        float2 ls2 = make_float2(0.f, 0.f);
+        if (none) {
+#pragma unroll
+            for (int i = 0; i < NK; ++i) sv[i] = 0.f;
+        } else {
+            const float2 c2 = make_float2(sc, sc), nm2 = make_float2(-mn, -mn);
+#pragma unroll
+            for (int i = 0; i < NK; i += 2) {
+                const float2 t = __ffma2_rn(make_float2(sv[i], sv[i + 1]), c2, nm2);
+                sv[i] = fast_exp2(t.x);
+                sv[i + 1] = fast_exp2(t.y);
+                ls2 = __fadd2_rn(ls2, make_float2(sv[i], sv[i + 1]));
+            }
+        }
+        l_run = l_run * alpha + (ls2.x + ls2.y);
+        // ---- the previous P.V must be done before O is rescaled, P rewritten and its stage refilled
+        if (blk > 0) {
+            if (!mbar_wait_parity_bounded(bar_o, (blk - 1) & 1)) {
+                timed_out = 1;
+                atomicOr(&g_error_word, PKV_DEVERR_TIMEOUT);
+            }
+            ptx::tcgen05_fence_after_thread_sync();
+            if (__any_sync(0xffffffffu, alpha != 1.f)) {        // rescale this warp's O rows
+#pragma unroll
+                for (int c0 = 0; c0 < D; c0 += 32) {
+                    uint32_t r[32];
+                    ptx::tcgen05_ld_32x32b(r, t_row + c0);
+                    ptx::tcgen05_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+                    ptx::tcgen05_st_32x32b(t_row + c0, r);
+                }
+                ptx::tcgen05_wait_st();
+            }
+        }
+        // V stage (blk + 1) & 1 last held V(blk - 1), whose P.V is complete
+        load_v(blk + 1);
+        cp_async_commit();
+        // ---- this row of P (and of its low part) -> shared memory, K-major swizzled
+#pragma unroll
+        for (int c = 0; c < NK / 8; ++c) {
+            uint32_t w[4], wl[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float a = sv[8 * c + 2 * e], bb = sv[8 * c + 2 * e + 1];
+                w[e] = MmaOps<T>::pack(a, bb);
+                if constexpr (kSplitP)
+                    wl[e] = MmaOps<T>::pack(a - __uint_as_float(w[e] << 16), bb - __uint_as_float(w[e] & 0xffff0000u));
+            }
+            const int off = tid * 128 + ((c ^ (tid & 7)) * 16);
+            *reinterpret_cast<uint4*>(ps + off) = make_uint4(w[0], w[1], w[2], w[3]);
+            if constexpr (kSplitP)
+                *reinterpret_cast<uint4*>(ps + S::kPBytes + off) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+        }
+        cp_async_wait<2>();                      // K(blk + 1) and V(blk) landed (K(blk + 2), V(blk + 1) may not)
+        fence_proxy_async_smem();
+        ptx::tcgen05_fence_before_thread_sync();
+        const int stop = __syncthreads_or(timed_out);   // P, rescaled O, S reads and block blk + 1 ready
+        ptx::tcgen05_fence_after_thread_sync();
+        if (stop) { ok = false; break; }
+        if (tid == 0) {
+            // S of the next block first (it needs neither P nor O), then O += P . V
+            if (blk + 1 < n_blocks) issue_s(blk + 1, tmem);
+            const unsigned char* vs = vring + (blk & 1) * S::kKvBytes;
+#pragma unroll
+            for (int part = 0; part < (kSplitP ? 2 : 1); ++part) {
+#pragma unroll
+                for (int kk = 0; kk < NK / 16; ++kk) {
+                    const uint64_t ad = umma_desc_sw128(smem_addr(ps) + part * S::kPBytes + kk * 32, 16, 1024);
+                    const uint64_t bd = umma_desc_sw128(smem_addr(vs) + kk * 2048, S::kRegion, 1024);
+                    ptx::tcgen05_mma(ptx::kind_f16, ptx::cta_group_1, tmem, ad, bd, idesc_o, blk > 0 || kk > 0 || part > 0);
+                }
+            }
+            ptx::tcgen05_commit(ptx::cta_group_1, bar_o);
+        }
+    }
+    // ---- out = O / l
+    if (ok) {
+        if (!mbar_wait_parity_bounded(bar_o, (n_blocks - 1) & 1)) timed_out = 1;
+        ok = !__syncthreads_or(timed_out);
+        if (!ok && tid == 0) atomicOr(&g_error_word, PKV_DEVERR_TIMEOUT);
+        ptx::tcgen05_fence_after_thread_sync();
+        const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+        T* orow = static_cast<T*>(p.out) + ((long long)(q0 + (rvalid ? tok : 0)) * p.q_heads + g * G + tid % G) * D;
+#pragma unroll
+        for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t r[32];
+            ptx::tcgen05_ld_32x32b(r, t_row + c0);
+            ptx::tcgen05_wait_ld();
+            if (ok && rvalid) {
+#pragma unroll
+                for (int e = 0; e < 32; e += 8) {
+                    uint4 u;
+                    uint32_t* uw = reinterpret_cast<uint32_t*>(&u);
+#pragma unroll
+                    for (int h = 0; h < 4; ++h)
+                        uw[h] = MmaOps<T>::pack(__uint_as_float(r[e + 2 * h]) * inv, __uint_as_float(r[e + 2 * h + 1]) * inv);
+                    *reinterpret_cast<uint4*>(orow + c0 + e) = u;
+                }
+            }
+        }
+    }
+    cp_async_wait<0>();
+    ptx::tcgen05_fence_before_thread_sync();
+    __syncthreads();
+    if (warp == 0) ptx::tcgen05_dealloc(ptx::cta_group_1, tmem, tmem_cols);
+}
+
+}  // namespace pkv
+
+#endif  // PKV_PREFILL_ATTENTION_TC_CUH_

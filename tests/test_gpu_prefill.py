@@ -62,6 +62,29 @@ def test_prefill_chunk_matches_oracle(d, P, Hq, Hkv, dtype, cached, chunk):
     assert pkv.kv_get_device_error() == 0
 
 
+@pytest.mark.parametrize("scale", [-0.2, 0.0])
+def test_prefill_with_negative_and_zero_scale(scale):
+    """A negative scale puts the softmax weight on the smallest scores; zero gives every visible
+    key the same weight."""
+    d, P, Hq, Hkv, dtype, cached, chunk = 128, 16, 8, 2, "bf16", [40, 3], [70, 9]
+    L = [c + n for c, n in zip(cached, chunk)]
+    s = synth.random_spec(1200, len(L), Hq, Hkv, d, P, [x - 1 for x in L], dtype=dtype)
+    kp, vp = synth.pool_values_numpy(s)
+    r = np.random.Generator(np.random.PCG64(1201))
+    q = synth.round_f32(r.standard_normal((sum(chunk), Hq, d), dtype=np.float32), dtype)
+    cu_q = np.concatenate([[0], np.cumsum(chunk)]).astype(np.int32)
+    ctx = np.array(L, np.int32)
+    pool = pkv.KVPool(to_dev(kp, dtype), to_dev(vp, dtype))
+    q_t = to_dev(q, dtype)
+    out = torch.full_like(q_t, float("nan"))
+    pkv.paged_prefill_attention(pool, 0, out, q_t, torch.from_numpy(cu_q).cuda(),
+                                torch.from_numpy(s.block_tables).cuda(), torch.from_numpy(ctx).cuda(), scale)
+    ref = oracle.prefill_attention(q, kp[0], vp[0], s.block_tables, cu_q, ctx, scale, dtype)
+    ok, maxerr, ratio = tolerance_report(to_bits(out), ref, dtype)
+    assert ok, "scale %g: max |err| %.3g, err/bound %.3g" % (scale, maxerr, ratio)
+    assert pkv.kv_get_device_error() == 0
+
+
 def test_prefill_of_single_tokens_equals_decode():
     """A chunk of one token per sequence is the decode step; both kernels agree within the
     tolerance (their reduction orders differ)."""
