@@ -56,6 +56,9 @@ def parse_args(argv=None):
     ap.add_argument("--op", choices=("decode", "rms_norm", "prefill"), default="decode",
                     help="decode: the decode step (default); rms_norm / prefill: that kernel alone")
     ap.add_argument("--chunk", type=int, default=512, help="prefill: new tokens per sequence")
+    ap.add_argument("--no-fused", action="store_true",
+                    help="decode: RoPE + append and attention as two launches per layer even where the fused "
+                         "layer kernel applies (16-bit pages, one query head per kv head)")
     ap.add_argument("--kv", choices=("native", "int8"), default="native",
                     help="decode: page storage -- the workload's 16-bit type, or int8 codes with a fp32 "
                          "scale per (token, head) row")
@@ -301,9 +304,11 @@ def run_ours(args):
         pool = pkv.KVPool(kp, vp)
     layer_bytes = kv_bytes_per_layer(s, args.kv)
     qs, ks, vs = synth.step_values_torch(s, INPUT_SETS, dev)
+    fused = not args.no_fused and args.kv == "native" and s.q_heads == s.kv_heads
     steps = []
     for j in range(INPUT_SETS):
-        st = DecodeStep(pool, s.batch, s.q_heads, s.max_pages, theta=s.theta, num_splits=args.splits, device=dev)
+        st = DecodeStep(pool, s.batch, s.q_heads, s.max_pages, theta=s.theta, num_splits=args.splits, device=dev,
+                        fused=fused)
         st.set_metadata(s.block_tables, s.context_lens, s.positions, non_blocking=False)
         st.q.copy_(qs[j])
         st.k.copy_(ks[j])
@@ -324,15 +329,20 @@ def run_ours(args):
         steps[i % INPUT_SETS].eager()
     for st in steps:
         st.capture()
-    attn = torch.cuda.CUDAGraph()                 # the 32 attention calls of one step alone
+    attn = torch.cuda.CUDAGraph()                 # the 32 attention (fused: layer) calls of one step alone
     cs = torch.cuda.Stream()
     cs.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(cs), torch.cuda.graph(attn, stream=cs):
         st0 = steps[0]
         for layer in range(L):
-            pkv.paged_decode_attention(pool, layer, st0.out[layer], st0.q[layer], st0.block_tables,
-                                       st0.context_lens, st0.scale, num_splits=st0.workspace.num_splits,
-                                       workspace=st0.workspace)
+            if fused:                               # the angle table of st0 is current
+                pkv.paged_decode_layer(pool, layer, st0.out[layer], st0.q[layer], st0.k[layer], st0.v[layer],
+                                       st0.rope, st0.block_tables, st0.context_lens, st0.scale,
+                                       num_splits=st0.workspace.num_splits, workspace=st0.workspace)
+            else:
+                pkv.paged_decode_attention(pool, layer, st0.out[layer], st0.q[layer], st0.block_tables,
+                                           st0.context_lens, st0.scale, num_splits=st0.workspace.num_splits,
+                                           workspace=st0.workspace)
     torch.cuda.current_stream().wait_stream(cs)
     for i in range(args.warmup):
         steps[i % INPUT_SETS].replay()
@@ -427,13 +437,15 @@ def run_ours(args):
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": profiled_traffic(args.workload, args.kv),
                          "peak_source": "%s copy bandwidth" % peak_kind,
-                         "kernel": "paged_decode_attention (one kernel per call)",
+                         "kernel": ("paged_decode_layer (RoPE + append + attention, one kernel per layer)"
+                                    if fused else "paged_decode_attention (one kernel per call)"),
                          "frac_of_8tbs": achieved / NOMINAL_HBM_GBS},
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": args.steps * steps[0].kernels_per_step * world,
             "num_splits": steps[0].workspace.num_splits,
-            "launch": "one CUDA graph per step (%d kernels)" % steps[0].kernels_per_step,
+            "launch": "one CUDA graph per step (%d kernels%s)" % (
+                steps[0].kernels_per_step, ": an angle table, then one fused kernel per layer" if fused else ""),
             "clocks": clk,
         }
         print(json.dumps(line), flush=True)

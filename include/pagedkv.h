@@ -311,6 +311,34 @@ int paged_prefill_attention(const pkv_pool* pool, int layer, void* out, const vo
                             pkv_stream_t stream);
 
 /*
+ * Angles of a decode step's new tokens, shared by all layers of the step ([ENGINE] s4.2):
+ * table[b][i] = (cos, sin)(pos_b * theta^(-2i/head_dim)) in fp64 for pos_b = context_lens[b] - 1
+ * (the new token's position; zeros when context_lens[b] <= 0), evaluated exactly as
+ * rope_apply does.
+ *   context_lens: device [batch] int32; table: device [batch][head_dim / 2][2] double,
+ *   16-byte aligned, written by the call.  head_dim 64 or 128.
+ */
+int rope_table(const int32_t* context_lens, int batch, int head_dim, double theta, double* table,
+               pkv_stream_t stream);
+
+/*
+ * One whole decode layer in one launch ([ENGINE] s4.3 rotate, append, attend; s5.3 fuse small
+ * kernels): for each sequence b with L = context_lens[b] > 0 the new token sits at position
+ * L - 1 of its page table; its k is turned by RoPE and written with v into that slot of
+ * `layer` (the append, bit for bit as rope_append would), q is turned likewise, and `out`
+ * receives the same attention as paged_decode_attention over the L tokens.
+ *   q: device [batch][q_heads][head_dim] and k, v: device [batch][kv_heads][head_dim], not yet
+ *      turned and left unchanged; rope: the step's rope_table; every other argument as for
+ *      paged_decode_attention (workspace sized by pkv_decode_workspace_size).
+ * Supported: 16-bit pools with q_heads == kv_heads (UNSUPPORTED otherwise).  A page id out of
+ * range is skipped and flagged as in paged_decode_attention.
+ */
+int paged_decode_layer(const pkv_pool* pool, int layer, void* out, const void* q, const void* k,
+                       const void* v, const double* rope, const int32_t* block_tables, int max_pages_per_seq,
+                       const int32_t* context_lens, int batch, int q_heads, int kv_heads, float scale,
+                       int num_splits, void* workspace, size_t workspace_bytes, pkv_stream_t stream);
+
+/*
  * Zero-fill a decode workspace (cudaMemsetAsync on `stream`) before its first use with
  * paged_decode_attention.  INVALID_ARG for a NULL workspace with a non-zero size.
  */

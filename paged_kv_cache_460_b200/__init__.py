@@ -23,7 +23,8 @@ from ._lib import (PKV_BF16, PKV_DEVERR_BAD_PAGE, PKV_DEVERR_BAD_SLOT, PKV_DEVER
                    PagedKVError, lib)
 
 __all__ = [
-    "KVPool", "rope_apply", "paged_kv_append", "rope_append", "paged_decode_attention", "paged_prefill_attention", "rms_norm", "pkv_slot_mapping",
+    "KVPool", "rope_apply", "paged_kv_append", "rope_append", "paged_decode_attention", "rope_table",
+    "paged_decode_layer", "paged_prefill_attention", "rms_norm", "pkv_slot_mapping",
     "pkv_kv_cache_bytes", "pkv_decode_workspace_size", "pkv_decode_default_splits",
     "kv_get_device_error", "DecodeWorkspace", "PagedKVError", "PKV_F16", "PKV_BF16", "PKV_I8",
     "PKV_DEVERR_BAD_PAGE", "PKV_DEVERR_BAD_SLOT", "PKV_DEVERR_TIMEOUT",
@@ -281,4 +282,42 @@ def paged_decode_attention(pool, layer, out, q, block_tables, context_lens, scal
                                       block_tables.shape[1], _ptr(context_lens), B, Hq, kv_heads, float(scale),
                                       num_splits, _ptr(workspace.buffer), workspace.nbytes, _stream(stream))
     _lib.check("paged_decode_attention", st)
+    return out
+
+
+def rope_table(context_lens, head_dim, theta=10000.0, table=None, stream=None):
+    """(cos, sin) of each sequence's new-token angles, float64 [batch, head_dim / 2, 2] on the
+    device, for paged_decode_layer (position = context_lens[b] - 1)."""
+    torch = _torch()
+    _need(context_lens, "context_lens", torch.int32)
+    B = context_lens.shape[0]
+    if table is None:
+        table = torch.empty((B, head_dim // 2, 2), dtype=torch.float64, device=context_lens.device)
+    _need(table, "table", torch.float64)
+    _lib.check("rope_table", lib().rope_table(_ptr(context_lens), B, head_dim, float(theta), _ptr(table),
+                                              _stream(stream)))
+    return table
+
+
+def paged_decode_layer(pool, layer, out, q, k, v, rope, block_tables, context_lens, scale, num_splits=0,
+                       workspace=None, stream=None):
+    """One decode layer in one launch: RoPE on q [B, Hq, d] and k [B, Hkv, d] (inputs left
+    unchanged), k and v appended at position context_lens[b] - 1, and out = attention over the
+    context_lens[b] tokens.  rope: the step's rope_table."""
+    torch = _torch()
+    for t, n in ((out, "out"), (q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, pool.dtype)
+    _need(rope, "rope", torch.float64)
+    _need(block_tables, "block_tables", torch.int32)
+    _need(context_lens, "context_lens", torch.int32)
+    B, Hq, _ = q.shape
+    if workspace is None:
+        workspace = DecodeWorkspace(B, Hq, pool.kv_heads, pool.head_dim, pool.page_size, pool.dtype, num_splits,
+                                    device=q.device, storage=pool.storage)
+    if num_splits == 0:
+        num_splits = workspace.num_splits
+    st = lib().paged_decode_layer(pool.handle, layer, _ptr(out), _ptr(q), _ptr(k), _ptr(v), _ptr(rope),
+                                  _ptr(block_tables), block_tables.shape[1], _ptr(context_lens), B, Hq, pool.kv_heads,
+                                  float(scale), num_splits, _ptr(workspace.buffer), workspace.nbytes, _stream(stream))
+    _lib.check("paged_decode_layer", st)
     return out

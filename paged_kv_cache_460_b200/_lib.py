@@ -46,6 +46,8 @@ SIGNATURES = {
     "pkv_decode_default_splits": (_I, [_I, _I, _I, _I, _I, ctypes.POINTER(_I)]),
     "pkv_decode_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
     "pkv_decode_workspace_clear": (_I, [_P, _SZ, _P]),
+    "rope_table": (_I, [_P, _I, _I, _D, _P, _P]),
+    "paged_decode_layer": (_I, [_P, _I, _P, _P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _F, _I, _P, _SZ, _P]),
     "paged_decode_attention": (_I, [_P, _I, _P, _P, _P, _I, _P, _I, _I, _I, _F, _I, _P, _SZ, _P]),
     "paged_decode_attention_noalloc": (_I, [_P, _I, _P, _P, _P, _I, _P, _I, _I, _I, _F, _I, _P]),
     "kv_get_device_error": (_I, [ctypes.POINTER(ctypes.c_uint32)]),

@@ -36,6 +36,7 @@
 #define PKV_DECODE_ATTENTION_CUH_
 
 #include "pkv_device.cuh"
+#include "rope_append.cuh"
 
 namespace pkv {
 
@@ -56,6 +57,9 @@ struct DecodeParams {
     const int32_t* context_lens;
     const float* k_scale;       // int8 pools: this layer's row scales [pages][kv_heads][P]
     const float* v_scale;
+    const void* k_new;          // fused layer: the new token's k (not yet turned) and v,
+    const void* v_new;          //   [batch][kv_heads][D]
+    const double* rope;         // fused layer: (cos, sin) of the new token's angles, [batch][D/2][2]
     float* part_o;              // [2 * num_splits][G][D]
     float* part_ml;             // [2 * num_splits][G][2]
     int* counters;              // [num_splits]: partials delivered per cut segment (zero between calls)
@@ -242,7 +246,14 @@ __device__ __forceinline__ void segment_epilogue(const DecodeParams& p, const fl
     }
 }
 
-template <int D, int P, int G, typename T>
+// kFused: the whole decode layer in one kernel ("为什么要自己动手写一个LLM推理引擎"
+// (wzjinhao.cn/news/61427) s4.3 rotate q and k, append k and v, attend; s5.3 fuse small
+// kernels).  q arrives unturned and each warp turns its segment's q rows in shared memory
+// from the step's angle table; the warp that owns a sequence's last page (which holds the
+// new token at position L - 1) turns the new k, writes k and v into the pool (the append)
+// and into its staged copy of the page.  No other kernel writes the pool meanwhile, so every
+// page may be prefetched before the PDL wait.
+template <int D, int P, int G, typename T, bool kFused = false>
 __global__ void __launch_bounds__(kDecodeThreads, G == 1 ? 4 : 1) decode_pass1_kernel(const DecodeParams p)
 {
     using S = DecodeShape<D, P, G>;
@@ -354,7 +365,7 @@ __global__ void __launch_bounds__(kDecodeThreads, G == 1 ? 4 : 1) decode_pass1_k
     // writing it) and the q rows (the kernel before may still be producing them).
     int m_pre = 0, pre_qb[DEPTH], pre_qg[DEPTH];
     for (; m_pre < DEPTH && m_pre < n_mine; ++m_pre) {
-        if (ij == inp - 1) break;
+        if (!kFused && ij == inp - 1) break;
         issue_kv(m_pre);
         pre_qb[m_pre] = -1;
         if (ib != qb || ig != qg) {
@@ -416,9 +427,40 @@ __global__ void __launch_bounds__(kDecodeThreads, G == 1 ? 4 : 1) decode_pass1_k
         for (long long uu = first; uu < u_end; uu += NW) {
             cp_async_wait<DEPTH - 1>();         // page kc has landed (this lane's copies)
             __syncwarp();                       // ... and every lane's
-            const unsigned char* s = ring + (int)(kc % DEPTH) * S::kSlot;
+            unsigned char* s = ring + (int)(kc % DEPTH) * S::kSlot;
+            if constexpr (kFused) {
+                if (j + (int)(uu - u) == np - 1) {
+                    // the new token: row L - 1 of the sequence, in this (its last) page
+                    const int tn = lens[b] - 1 - (np - 1) * P;
+                    const int page = p.block_tables[(long long)b * p.max_pages + np - 1];
+                    if (lane < 2 * CPR) {
+                        const bool is_v = lane >= CPR;
+                        const int c = is_v ? lane - CPR : lane;
+                        uint4 w = reinterpret_cast<const uint4*>(static_cast<const T*>(is_v ? p.v_new : p.k_new) +
+                                                                 ((long long)b * Hkv + g) * D)[c];
+                        if (!is_v) rope_rotate8<T>(w, p.rope + (long long)b * D, 4 * c);
+                        if (is_v)
+                            *reinterpret_cast<uint4*>(s + S::kChunk + tn * (2 * D) + c * 16) = w;
+                        else
+                            *reinterpret_cast<uint4*>(s + tn * (2 * D) + ((c ^ ((tn * LPRK + c / CPL) & 7)) * 16)) = w;
+                        if ((unsigned)page < (unsigned)p.num_pages)      // the append
+                            reinterpret_cast<uint4*>(const_cast<T*>(static_cast<const T*>(is_v ? p.v : p.k)) +
+                                                     (((long long)page * Hkv + g) * P + tn) * D)[c] = w;
+                    }
+                    __syncwarp();
+                }
+            }
             if (!have_q) {                      // first page of this segment for this warp
                 have_q = true;
+                if constexpr (kFused) {         // turn the group's q rows in place
+                    for (int n = lane; n < G * CPR; n += 32) {
+                        uint4* qv = reinterpret_cast<uint4*>(s + 2 * S::kChunk) + n;
+                        uint4 w = *qv;
+                        rope_rotate8<T>(w, p.rope + (long long)b * D, 4 * (n % CPR));
+                        *qv = w;
+                    }
+                    __syncwarp();
+                }
 #pragma unroll
                 for (int gi = 0; gi < G; ++gi)
 #pragma unroll

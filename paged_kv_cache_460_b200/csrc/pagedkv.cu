@@ -370,6 +370,94 @@ extern "C" int paged_decode_attention(const pkv_pool* pool, int layer, void* out
 namespace pkv {
 namespace {
 
+// The fused decode layer: the CUDA-core kernel with RoPE and the append folded in
+// (16-bit pages, one query head per kv head).
+template <int D, int P, typename T>
+int launch_fused(const DecodeParams& prm, cudaStream_t st)
+{
+    static int configured[kMaxDevices] = {0};
+    const int smem = DecodeShape<D, P, 1>::smem_bytes(prm.batch);
+    if (smem > kMaxSmemPerCta) return PKV_ERR_UNSUPPORTED;
+    if (ensure_smem(decode_pass1_kernel<D, P, 1, T, true>, smem, configured) != cudaSuccess) return PKV_ERR_CUDA;
+    return status_of(launch_pdl(decode_pass1_kernel<D, P, 1, T, true>, dim3(prm.num_splits), dim3(kDecodeThreads),
+                                smem, st, prm));
+}
+
+template <typename T>
+int fused_shape(int head_dim, int page_size, const DecodeParams& prm, cudaStream_t st)
+{
+    if (head_dim == 128 && page_size == 16) return launch_fused<128, 16, T>(prm, st);
+    if (head_dim == 128 && page_size == 32) return launch_fused<128, 32, T>(prm, st);
+    if (head_dim == 64 && page_size == 16) return launch_fused<64, 16, T>(prm, st);
+    if (head_dim == 64 && page_size == 32) return launch_fused<64, 32, T>(prm, st);
+    return PKV_ERR_UNSUPPORTED;
+}
+
+}  // namespace
+}  // namespace pkv
+
+extern "C" int rope_table(const int32_t* context_lens, int batch, int head_dim, double theta, double* table,
+                          pkv_stream_t stream)
+{
+    if (batch < 0 || !(theta > 0.0)) return PKV_ERR_INVALID_ARG;
+    if (head_dim != 64 && head_dim != 128) return PKV_ERR_UNSUPPORTED;
+    if (batch == 0) return PKV_OK;
+    if (!context_lens || !table || (reinterpret_cast<uintptr_t>(table) & 15u)) return PKV_ERR_INVALID_ARG;
+    return status_of(launch_pdl(rope_table_kernel, dim3(batch), dim3(64), 0, reinterpret_cast<cudaStream_t>(stream),
+                                context_lens, head_dim, theta, table));
+}
+
+extern "C" int paged_decode_layer(const pkv_pool* pool, int layer, void* out, const void* q, const void* k,
+                                  const void* v, const double* rope, const int32_t* block_tables, int max_pages_per_seq,
+                                  const int32_t* context_lens, int batch, int q_heads, int kv_heads, float scale,
+                                  int num_splits, void* workspace, size_t workspace_bytes, pkv_stream_t stream)
+{
+    if (!pool || layer < 0 || layer >= pool->num_layers) return PKV_ERR_INVALID_ARG;
+    if (batch < 0 || q_heads <= 0 || kv_heads != pool->kv_heads || q_heads % kv_heads) return PKV_ERR_INVALID_ARG;
+    if (num_splits < 0 || max_pages_per_seq <= 0 || !(scale == scale)) return PKV_ERR_INVALID_ARG;
+    if (q_heads != kv_heads || pool->storage != pool->dtype) return PKV_ERR_UNSUPPORTED;
+    if (batch == 0) return PKV_OK;
+    if (!out || !q || !k || !v || !rope || !block_tables || !context_lens || !workspace) return PKV_ERR_INVALID_ARG;
+    if (misaligned16(out, q, k) || misaligned16(v, rope)) return PKV_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return PKV_ERR_INVALID_ARG;
+    DecodeOps ops;
+    if (!pick_decode(pool->head_dim, pool->page_size, 1, pool->dtype, pool->storage, ops)) return PKV_ERR_UNSUPPORTED;
+    if (num_splits == 0) {
+        const int st = ops.splits(&num_splits);
+        if (st != PKV_OK) return st;
+    }
+    const WorkspaceLayout wl = workspace_layout(batch, 1, pool->head_dim, num_splits);
+    if (workspace_bytes < wl.total) return PKV_ERR_NO_SPACE;
+    DecodeParams prm;
+    std::memset(&prm, 0, sizeof(prm));
+    prm.k = static_cast<const char*>(pool->k_base) + (size_t)layer * pool->layer_bytes();
+    prm.v = static_cast<const char*>(pool->v_base) + (size_t)layer * pool->layer_bytes();
+    prm.q = q;
+    prm.out = out;
+    prm.k_new = k;
+    prm.v_new = v;
+    prm.rope = rope;
+    prm.block_tables = block_tables;
+    prm.context_lens = context_lens;
+    unsigned char* ws = static_cast<unsigned char*>(workspace);
+    prm.counters = reinterpret_cast<int*>(ws + wl.counters);
+    prm.part_o = reinterpret_cast<float*>(ws + wl.part_o);
+    prm.part_ml = reinterpret_cast<float*>(ws + wl.part_ml);
+    prm.batch = batch;
+    prm.max_pages = max_pages_per_seq;
+    prm.q_heads = q_heads;
+    prm.kv_heads = kv_heads;
+    prm.num_pages = pool->num_pages;
+    prm.num_splits = num_splits;
+    prm.scale_log2 = scale * 1.4426950408889634f;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (pool->dtype == PKV_F16) return fused_shape<__half>(pool->head_dim, pool->page_size, prm, st);
+    return fused_shape<__nv_bfloat16>(pool->head_dim, pool->page_size, prm, st);
+}
+
+namespace pkv {
+namespace {
+
 template <int D, int P, int G, typename T>
 int launch_prefill(const PrefillParams& prm, int grid, cudaStream_t st)
 {

@@ -34,6 +34,45 @@ struct RopeAppendParams {
     int mode;
 };
 
+// Turn the four pairs of a 16-byte vector of T in place: pair k of the vector is pair
+// i0 + k of the head, cs[2 i] = cos and cs[2 i + 1] = sin of its angle.  Each pair is turned
+// in fp64 with explicit _rn products (no fused rounding) and rounded once to T.
+template <typename T>
+__device__ __forceinline__ void rope_rotate8(uint4& u, const double* cs, int i0)
+{
+    T* e = reinterpret_cast<T*>(&u);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const double x0 = Elt<T>::to_double(e[2 * k]);
+        const double x1 = Elt<T>::to_double(e[2 * k + 1]);
+        const double cn = cs[2 * (i0 + k)], sn = cs[2 * (i0 + k) + 1];
+        e[2 * k] = Elt<T>::from_double(__dsub_rn(__dmul_rn(x0, cn), __dmul_rn(x1, sn)));
+        e[2 * k + 1] = Elt<T>::from_double(__dadd_rn(__dmul_rn(x0, sn), __dmul_rn(x1, cn)));
+    }
+}
+
+// Angles of the decode step's new tokens, shared by every layer of the step: for sequence b
+// with L = context_lens[b] cached tokens (the new one included), position L - 1, and pair i,
+// table[b][i] = (cos, sin)(pos * theta^(-2i/d)), evaluated in fp64 exactly as the RoPE
+// kernel does.  Sequences with no token get zeros.
+__global__ void __launch_bounds__(64) rope_table_kernel(const int32_t* __restrict__ context_lens, int head_dim,
+                                                        double theta, double* __restrict__ table)
+{
+    pdl_wait();
+    pdl_launch_dependents();
+    const int b = blockIdx.x, half = head_dim >> 1;
+    const int pos = context_lens[b] - 1;
+    for (int i = threadIdx.x; i < half; i += blockDim.x) {
+        double sn = 0.0, cn = 0.0;
+        if (pos >= 0) {
+            const double freq = pow(theta, -2.0 * (double)i / (double)head_dim);
+            sincos((double)pos * freq, &sn, &cn);
+        }
+        table[((long long)b * half + i) * 2] = cn;
+        table[((long long)b * half + i) * 2 + 1] = sn;
+    }
+}
+
 // Grid: (token, part).  Each thread handles one 16-byte vector (8 elements, 4 pairs)
 // of the token's q, k or v rows.  The head_dim/2 angles pos * theta^(-2i/d) and their
 // cosines and sines are evaluated once per CTA in fp64 before griddepcontrol.wait, so
@@ -102,16 +141,7 @@ __global__ void __launch_bounds__(256) rope_append_kernel(const RopeAppendParams
         }
         uint4 u = *src;
         if (!is_v && pos >= 0) {
-            T* e = reinterpret_cast<T*>(&u);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int i = c * 4 + k;                    // pair index within the head
-                const double x0 = Elt<T>::to_double(e[2 * k]);
-                const double x1 = Elt<T>::to_double(e[2 * k + 1]);
-                const double cn = cs[i][0], sn = cs[i][1];
-                e[2 * k] = Elt<T>::from_double(__dsub_rn(__dmul_rn(x0, cn), __dmul_rn(x1, sn)));
-                e[2 * k + 1] = Elt<T>::from_double(__dadd_rn(__dmul_rn(x0, sn), __dmul_rn(x1, cn)));
-            }
+            rope_rotate8<T>(u, &cs[0][0], c * 4);
             *src = u;
         }
         if (slot >= 0 && idx >= nq) {      // uniform over the vph threads of a head row

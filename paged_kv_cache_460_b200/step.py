@@ -13,7 +13,8 @@ import math
 
 import torch
 
-from . import DecodeWorkspace, KVPool, paged_decode_attention, pkv_slot_mapping, rope_append
+from . import (DecodeWorkspace, KVPool, paged_decode_attention, paged_decode_layer, pkv_slot_mapping, rope_append,
+               rope_table)
 
 
 class DecodeStep:
@@ -28,7 +29,7 @@ class DecodeStep:
     """
 
     def __init__(self, pool: KVPool, batch, q_heads, max_pages, scale=None, theta=10000.0, num_splits=0,
-                 device=None):
+                 device=None, fused=False):
         self.pool = pool
         dev = torch.device(device) if device is not None else pool.k_cache.device
         L, d, Hkv = pool.num_layers, pool.head_dim, pool.kv_heads
@@ -46,11 +47,21 @@ class DecodeStep:
         self.workspace = DecodeWorkspace(batch, q_heads, Hkv, d, pool.page_size, dt, num_splits, device=dev,
                                          storage=pool.storage)
         self.graph = None
-        self.kernels_per_step = 2 * L
+        # fused: one angle-table launch per step, then one launch per layer (RoPE, append and
+        # attention together); otherwise RoPE + append and attention, two launches per layer
+        self.fused = fused
+        self.rope = torch.zeros((batch, d // 2, 2), dtype=torch.float64, device=dev) if fused else None
+        self.kernels_per_step = (1 + L) if fused else 2 * L
 
     def layer(self, i, stream=None):
         """Enqueue layer i of the step on the current stream: RoPE + KV append (one
-        kernel), then attention (one kernel)."""
+        kernel), then attention (one kernel); fused: the whole layer in one kernel (the
+        step's angle table must be current)."""
+        if self.fused:
+            paged_decode_layer(self.pool, i, self.out[i], self.q[i], self.k[i], self.v[i], self.rope,
+                               self.block_tables, self.context_lens, self.scale,
+                               num_splits=self.workspace.num_splits, workspace=self.workspace, stream=stream)
+            return
         rope_append(self.pool, i, self.q[i], self.k[i], self.v[i], self.positions, self.slot_mapping, self.theta,
                     stream)
         paged_decode_attention(self.pool, i, self.out[i], self.q[i], self.block_tables, self.context_lens,
@@ -58,6 +69,8 @@ class DecodeStep:
                                stream=stream)
 
     def eager(self):
+        if self.fused:
+            rope_table(self.context_lens, self.pool.head_dim, self.theta, table=self.rope)
         for i in range(self.pool.num_layers):
             self.layer(i)
 
