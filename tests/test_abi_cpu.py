@@ -265,3 +265,26 @@ def test_int8_kv_cache_bytes():
     assert pkv.pkv_kv_cache_bytes(32, 32, 128, 2048, pkv.PKV_I8) == 32 * 2 * 32 * 2048 * 132
     assert pkv.pkv_kv_cache_bytes(32, 32, 128, 2048, pkv.PKV_I8) * 2 < \
         pkv.pkv_kv_cache_bytes(32, 32, 128, 2048, pkv.PKV_F16) * 1.04
+
+
+def test_fused_layer_and_rope_table_validate(L):
+    f = _fake_ptr
+    assert L.rope_table(f(), 4, 96, 10000.0, f(), None) == _lib.PKV_ERR_UNSUPPORTED
+    assert L.rope_table(f(), 4, 128, 0.0, f(), None) == _lib.PKV_ERR_INVALID_ARG
+    assert L.rope_table(f(), 4, 128, 10000.0, f(0x10008), None) == _lib.PKV_ERR_INVALID_ARG
+    assert L.rope_table(None, 0, 128, 10000.0, None, None) == 0
+    h = _pool(L, num_pages=8, page_size=16, kv_heads=2, head_dim=64)
+    args = lambda hq, hkv: (h, 0, f(), f(), f(), f(), f(), f(), 4, f(), 1, hq, hkv, 0.1, 0, f(0x20000), 1 << 20, None)
+    assert L.paged_decode_layer(*args(4, 2)) == _lib.PKV_ERR_UNSUPPORTED        # grouped heads: not fused
+    assert L.paged_decode_layer(*args(3, 2)) == _lib.PKV_ERR_INVALID_ARG
+    a = list(args(2, 2))
+    a[5] = None                                                                  # no v
+    assert L.paged_decode_layer(*a) == _lib.PKV_ERR_INVALID_ARG
+    a = list(args(2, 2))
+    a[1] = 1                                                                     # layer out of range
+    assert L.paged_decode_layer(*a) == _lib.PKV_ERR_INVALID_ARG
+    L.kv_pool_destroy(h)
+    h = _pool_i8(L)
+    assert L.paged_decode_layer(h, 0, f(), f(), f(), f(), f(), f(), 4, f(), 1, 2, 2, 0.1, 0, f(0x20000), 1 << 20,
+                                None) == _lib.PKV_ERR_UNSUPPORTED                 # int8 pages: not fused
+    L.kv_pool_destroy(h)
