@@ -330,8 +330,10 @@ int rope_table(const int32_t* context_lens, int batch, int head_dim, double thet
  *   q: device [batch][q_heads][head_dim] and k, v: device [batch][kv_heads][head_dim], not yet
  *      turned and left unchanged; rope: the step's rope_table; every other argument as for
  *      paged_decode_attention (workspace sized by pkv_decode_workspace_size).
- * Supported: 16-bit pools with q_heads == kv_heads (UNSUPPORTED otherwise).  A page id out of
- * range is skipped and flagged as in paged_decode_attention.
+ * Supported: 16-bit pools with q_heads == kv_heads, and int8 pools (kv_pool_create_i8) with
+ * q_heads / kv_heads in {1, 2, 4, 8}, whose new rows are quantised as paged_kv_append does
+ * (UNSUPPORTED otherwise).  A page id out of range is skipped and flagged as in
+ * paged_decode_attention.
  */
 int paged_decode_layer(const pkv_pool* pool, int layer, void* out, const void* q, const void* k,
                        const void* v, const double* rope, const int32_t* block_tables, int max_pages_per_seq,

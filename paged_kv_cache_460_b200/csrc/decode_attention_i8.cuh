@@ -88,7 +88,41 @@ __device__ __forceinline__ void i8_even_odd(uint32_t w, uint32_t& ev, uint32_t& 
     od = i8_pair_to_f16x2(x, 0x5341u);
 }
 
-template <int D, int P, int G, typename T>
+// Quantise one head row held as 16-byte vectors of T by `vpr` consecutive lanes (vector c of
+// the row in lane c of the group): the row's amax by a shuffle reduction within the group,
+// codes round_half_even(x * (127 / amax)) clamped to +-127, scale amax / 127 -- every step the
+// correctly rounded fp32 operation of the append kernel, so the results are identical.
+// Lanes outside any group take part in the shuffles with amax 0.
+template <typename T>
+__device__ __forceinline__ uint2 i8_quantise_vec(const uint4& u, int vpr, bool active, float& scale)
+{
+    float x[8];
+    unpack8<T>(u, x);
+    float amax = 0.f;
+    if (active) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(x[e]));
+    }
+    for (int m = vpr >> 1; m >= 1; m >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, m));
+    uint32_t w[2] = {0u, 0u};
+    scale = 0.f;
+    if (amax > 0.f) {
+        const float inv = __fdiv_rn(127.f, amax);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const float r = fminf(fmaxf(rintf(__fmul_rn(x[e], inv)), -127.f), 127.f);
+            w[e >> 2] |= ((uint32_t)(int)r & 0xffu) << (8 * (e & 3));
+        }
+        scale = __fdiv_rn(amax, 127.f);
+    }
+    return make_uint2(w[0], w[1]);
+}
+
+// kFused: the whole decode layer in one kernel, as for the 16-bit CUDA-core kernel: q turned
+// in shared memory from the step's angle table at each segment's first unit; the warp that
+// owns a sequence's last unit turns the new k, quantises k and v, appends codes and scales to
+// the pool and patches its staged copy; every unit may be prefetched before the PDL wait.
+template <int D, int P, int G, typename T, bool kFused = false>
 __global__ void __launch_bounds__(kDecodeThreads, 3) decode_i8_kernel(const DecodeParams p)
 {
     using S = I8Shape<D, G>;
@@ -203,7 +237,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_i8_kernel(const Deco
     };
     int m_pre = 0, pre_qb[DEPTH], pre_qg[DEPTH];
     for (; m_pre < DEPTH && m_pre < n_mine; ++m_pre) {
-        if (ij == inp - 1) break;
+        if (!kFused && ij == inp - 1) break;
         issue_kv(m_pre, m_pre);
         pre_qb[m_pre] = -1;
         if (ib != qb || ig != qg) {
@@ -265,9 +299,51 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_i8_kernel(const Deco
         for (long long uu = first; uu < u_end; uu += NW) {
             cp_async_wait<DEPTH - 1>();
             __syncwarp();
-            const unsigned char* s = ring + cs * S::kSlot;
+            unsigned char* s = ring + cs * S::kSlot;
+            if constexpr (kFused) {
+                if (j + (int)(uu - u) == np - 1) {
+                    // the new token: position L - 1 of the sequence, row tn of this (its last) unit
+                    const int last = lens[b] - 1;
+                    const int tn = last - (np - 1) * 32;
+                    const int page = p.block_tables[(long long)b * p.max_pages + last / P];
+                    constexpr int VPR = D / 8;                  // 16-byte vectors of T per row
+                    const bool active = lane < 2 * VPR;
+                    const bool is_v = lane >= VPR;
+                    const int c = lane % VPR;
+                    uint4 w = make_uint4(0u, 0u, 0u, 0u);
+                    if (active) {
+                        w = reinterpret_cast<const uint4*>(static_cast<const T*>(is_v ? p.v_new : p.k_new) +
+                                                           ((long long)b * Hkv + g) * D)[c];
+                        if (!is_v) rope_rotate8<T>(w, p.rope + (long long)b * D, 4 * c);
+                    }
+                    float sc;
+                    const uint2 codes = i8_quantise_vec<T>(w, VPR, active, sc);
+                    if (active) {
+                        unsigned char* row = s + (is_v ? S::kChunk : 0) + tn * D;
+                        *reinterpret_cast<uint2*>(row + (((c >> 1) ^ i8_swizzle<D>(tn)) * 16) + 8 * (c & 1)) = codes;
+                        if (c == 0)
+                            reinterpret_cast<float*>(s + 2 * S::kChunk + (is_v ? S::kScaleBytes : 0))[tn] = sc;
+                        if ((unsigned)page < (unsigned)p.num_pages) {           // the append
+                            const long long rid = ((long long)page * Hkv + g) * P + last % P;
+                            *reinterpret_cast<uint2*>(const_cast<unsigned char*>(
+                                static_cast<const unsigned char*>(is_v ? p.v : p.k)) + rid * D + 8 * c) = codes;
+                            if (c == 0) const_cast<float*>(is_v ? p.v_scale : p.k_scale)[rid] = sc;
+                        }
+                    }
+                    __syncwarp();
+                }
+            }
             if (!have_q) {
                 have_q = true;
+                if constexpr (kFused) {         // turn the group's q rows in place
+                    for (int n = lane; n < G * (D / 8); n += 32) {
+                        uint4* qv = reinterpret_cast<uint4*>(s + S::kQOffset) + n;
+                        uint4 w = *qv;
+                        rope_rotate8<T>(w, p.rope + (long long)b * D, 4 * (n % (D / 8)));
+                        *qv = w;
+                    }
+                    __syncwarp();
+                }
                 const T* qa = reinterpret_cast<const T*>(s + S::kQOffset);
                 int shift = 0;                // power of two that brings the head row's max under 2^15
                 float qs = 0.f;               // this lane's part of sum_d q_d (of the fp16 operand)

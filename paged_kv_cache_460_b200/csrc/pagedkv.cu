@@ -370,26 +370,40 @@ extern "C" int paged_decode_attention(const pkv_pool* pool, int layer, void* out
 namespace pkv {
 namespace {
 
-// The fused decode layer: the CUDA-core kernel with RoPE and the append folded in
-// (16-bit pages, one query head per kv head).
-template <int D, int P, typename T>
+// The fused decode layer: the attention kernels with RoPE and the append folded in --
+// the CUDA-core kernel for 16-bit pages with one query head per kv head, the int8 kernel
+// for int8 pages with any group size.
+template <int D, int P, int G, typename T, bool I8>
 int launch_fused(const DecodeParams& prm, cudaStream_t st)
 {
     static int configured[kMaxDevices] = {0};
-    const int smem = DecodeShape<D, P, 1>::smem_bytes(prm.batch);
+    constexpr auto fn = I8 ? decode_i8_kernel<D, P, G, T, true> : decode_pass1_kernel<D, P, G, T, true>;
+    const int smem = I8 ? I8Shape<D, G>::smem_bytes(prm.batch) : DecodeShape<D, P, G>::smem_bytes(prm.batch);
     if (smem > kMaxSmemPerCta) return PKV_ERR_UNSUPPORTED;
-    if (ensure_smem(decode_pass1_kernel<D, P, 1, T, true>, smem, configured) != cudaSuccess) return PKV_ERR_CUDA;
-    return status_of(launch_pdl(decode_pass1_kernel<D, P, 1, T, true>, dim3(prm.num_splits), dim3(kDecodeThreads),
-                                smem, st, prm));
+    if (ensure_smem(fn, smem, configured) != cudaSuccess) return PKV_ERR_CUDA;
+    return status_of(launch_pdl(fn, dim3(prm.num_splits), dim3(kDecodeThreads), smem, st, prm));
+}
+
+template <int D, int P, typename T>
+int fused_group(int group, bool i8, const DecodeParams& prm, cudaStream_t st)
+{
+    if (!i8) return group == 1 ? launch_fused<D, P, 1, T, false>(prm, st) : PKV_ERR_UNSUPPORTED;
+    switch (group) {
+    case 1: return launch_fused<D, P, 1, T, true>(prm, st);
+    case 2: return launch_fused<D, P, 2, T, true>(prm, st);
+    case 4: return launch_fused<D, P, 4, T, true>(prm, st);
+    case 8: return launch_fused<D, P, 8, T, true>(prm, st);
+    default: return PKV_ERR_UNSUPPORTED;
+    }
 }
 
 template <typename T>
-int fused_shape(int head_dim, int page_size, const DecodeParams& prm, cudaStream_t st)
+int fused_shape(int head_dim, int page_size, int group, bool i8, const DecodeParams& prm, cudaStream_t st)
 {
-    if (head_dim == 128 && page_size == 16) return launch_fused<128, 16, T>(prm, st);
-    if (head_dim == 128 && page_size == 32) return launch_fused<128, 32, T>(prm, st);
-    if (head_dim == 64 && page_size == 16) return launch_fused<64, 16, T>(prm, st);
-    if (head_dim == 64 && page_size == 32) return launch_fused<64, 32, T>(prm, st);
+    if (head_dim == 128 && page_size == 16) return fused_group<128, 16, T>(group, i8, prm, st);
+    if (head_dim == 128 && page_size == 32) return fused_group<128, 32, T>(group, i8, prm, st);
+    if (head_dim == 64 && page_size == 16) return fused_group<64, 16, T>(group, i8, prm, st);
+    if (head_dim == 64 && page_size == 32) return fused_group<64, 32, T>(group, i8, prm, st);
     return PKV_ERR_UNSUPPORTED;
 }
 
@@ -415,18 +429,21 @@ extern "C" int paged_decode_layer(const pkv_pool* pool, int layer, void* out, co
     if (!pool || layer < 0 || layer >= pool->num_layers) return PKV_ERR_INVALID_ARG;
     if (batch < 0 || q_heads <= 0 || kv_heads != pool->kv_heads || q_heads % kv_heads) return PKV_ERR_INVALID_ARG;
     if (num_splits < 0 || max_pages_per_seq <= 0 || !(scale == scale)) return PKV_ERR_INVALID_ARG;
-    if (q_heads != kv_heads || pool->storage != pool->dtype) return PKV_ERR_UNSUPPORTED;
+    const bool i8 = pool->storage == kStorageI8;
+    const int group = q_heads / kv_heads;
+    if (!i8 && group != 1) return PKV_ERR_UNSUPPORTED;
     if (batch == 0) return PKV_OK;
     if (!out || !q || !k || !v || !rope || !block_tables || !context_lens || !workspace) return PKV_ERR_INVALID_ARG;
     if (misaligned16(out, q, k) || misaligned16(v, rope)) return PKV_ERR_INVALID_ARG;
     if (reinterpret_cast<uintptr_t>(workspace) & 255u) return PKV_ERR_INVALID_ARG;
     DecodeOps ops;
-    if (!pick_decode(pool->head_dim, pool->page_size, 1, pool->dtype, pool->storage, ops)) return PKV_ERR_UNSUPPORTED;
+    if (!pick_decode(pool->head_dim, pool->page_size, group, pool->dtype, pool->storage, ops))
+        return PKV_ERR_UNSUPPORTED;
     if (num_splits == 0) {
         const int st = ops.splits(&num_splits);
         if (st != PKV_OK) return st;
     }
-    const WorkspaceLayout wl = workspace_layout(batch, 1, pool->head_dim, num_splits);
+    const WorkspaceLayout wl = workspace_layout(batch, group, pool->head_dim, num_splits);
     if (workspace_bytes < wl.total) return PKV_ERR_NO_SPACE;
     DecodeParams prm;
     std::memset(&prm, 0, sizeof(prm));
@@ -437,6 +454,10 @@ extern "C" int paged_decode_layer(const pkv_pool* pool, int layer, void* out, co
     prm.k_new = k;
     prm.v_new = v;
     prm.rope = rope;
+    if (i8) {
+        prm.k_scale = static_cast<const float*>(pool->k_scale_base) + (size_t)layer * pool->layer_rows();
+        prm.v_scale = static_cast<const float*>(pool->v_scale_base) + (size_t)layer * pool->layer_rows();
+    }
     prm.block_tables = block_tables;
     prm.context_lens = context_lens;
     unsigned char* ws = static_cast<unsigned char*>(workspace);
@@ -451,8 +472,8 @@ extern "C" int paged_decode_layer(const pkv_pool* pool, int layer, void* out, co
     prm.num_splits = num_splits;
     prm.scale_log2 = scale * 1.4426950408889634f;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (pool->dtype == PKV_F16) return fused_shape<__half>(pool->head_dim, pool->page_size, prm, st);
-    return fused_shape<__nv_bfloat16>(pool->head_dim, pool->page_size, prm, st);
+    if (pool->dtype == PKV_F16) return fused_shape<__half>(pool->head_dim, pool->page_size, group, i8, prm, st);
+    return fused_shape<__nv_bfloat16>(pool->head_dim, pool->page_size, group, i8, prm, st);
 }
 
 namespace pkv {

@@ -285,6 +285,6 @@ def test_fused_layer_and_rope_table_validate(L):
     assert L.paged_decode_layer(*a) == _lib.PKV_ERR_INVALID_ARG
     L.kv_pool_destroy(h)
     h = _pool_i8(L)
-    assert L.paged_decode_layer(h, 0, f(), f(), f(), f(), f(), f(), 4, f(), 1, 2, 2, 0.1, 0, f(0x20000), 1 << 20,
-                                None) == _lib.PKV_ERR_UNSUPPORTED                 # int8 pages: not fused
+    assert L.paged_decode_layer(h, 0, f(), f(), f(), f(), f(), f(), 4, f(), 1, 32, 2, 0.1, 0, f(0x20000), 1 << 20,
+                                None) == _lib.PKV_ERR_UNSUPPORTED                 # group 16: no kernel
     L.kv_pool_destroy(h)

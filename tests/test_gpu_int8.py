@@ -217,3 +217,21 @@ def test_int8_full_size_workload_sampled(name, layers, check_layers):
             gots.append(outs[L][b, g * G:(g + 1) * G])
         _expect_close(np.stack(gots), np.stack(refs), s.dtype, "int8 %s layer %d" % (name, L))
     assert pkv.kv_get_device_error() == 0
+
+
+@pytest.mark.parametrize("d,P,Hq,Hkv,dtype,cached", [SHAPES[0], SHAPES[1], SHAPES[3], SHAPES[4], SHAPES[7]])
+def test_int8_fused_layer_matches_two_launch_path(d, P, Hq, Hkv, dtype, cached):
+    """paged_decode_layer on an int8 pool: the new rows quantised in-kernel exactly as the
+    append kernel does; output, codes and scales bit-identical to rope_append + attention."""
+    s = synth.random_spec(1700 + d + P + Hq, len(cached), Hq, Hkv, d, P, cached, dtype=dtype)
+    fused, split = I8Case(s), I8Case(s)
+    ref_out = split.gpu_layer(0)
+    q_t, k_t, v_t = (to_dev(x[0], s.dtype) for x in (fused.q, fused.k, fused.v))
+    rope = pkv.rope_table(fused.cl_t, s.head_dim, s.theta)
+    out = torch.full_like(q_t, float("nan"))
+    pkv.paged_decode_layer(fused.pool, 0, out, q_t, k_t, v_t, rope, fused.bt_t, fused.cl_t, fused.scale)
+    assert np.array_equal(to_bits(out), to_bits(ref_out))
+    for a, b in zip(fused.t, split.t):
+        assert torch.equal(a, b)
+    _expect_close(out, fused.oracle_layer(0), dtype, "int8 fused %s" % ((d, P, Hq, Hkv, dtype),))
+    assert pkv.kv_get_device_error() == 0
