@@ -154,9 +154,19 @@ __global__ void __launch_bounds__(kTcRows, 1) prefill_tc_kernel(const PrefillPar
             *reinterpret_cast<uint4*>(qs + (c / 8) * (kTcRows * 128) + tid * 128 + (((c % 8) ^ (tid & 7)) * 16)) = v;
         }
     }
-    // ---- K or V block loads (the same swizzled layout for both; keys past the cache are zero)
+    // ---- K or V block loads (the same swizzled layout for both; keys past the cache are zero).
+    // The page ids of a block are fetched an iteration before its copies are issued, so the
+    // copies never wait on the page table.
+    constexpr int NPB = NK / P > 0 ? NK / P : 1;    // pages per block
     const int32_t* table = p.block_tables + (long long)b * p.max_pages;
-    auto load_block = [&](const void* pool, unsigned char* dst_block, int blk) {
+    auto fetch_ids = [&](int blk, int (&ids)[NPB]) {
+#pragma unroll
+        for (int j = 0; j < NPB; ++j) {
+            const int pg = (blk * NK) / P + j;
+            ids[j] = pg * P < L ? (pg < p.max_pages ? table[pg] : -1) : -2;
+        }
+    };
+    auto load_block = [&](const void* pool, unsigned char* dst_block, int blk, const int (&ids)[NPB]) {
 #pragma unroll
         for (int n = 0; n < NKC; ++n) {
             const int idx = n * kTcRows + tid;
@@ -165,8 +175,7 @@ __global__ void __launch_bounds__(kTcRows, 1) prefill_tc_kernel(const PrefillPar
             bool valid = key < L;
             long long off = 0;
             if (valid) {
-                const int pg = key / P;
-                const int page = pg < p.max_pages ? table[pg] : -1;
+                const int page = ids[(t % NK) / P];
                 if ((unsigned)page < (unsigned)p.num_pages) {
                     off = (((long long)page * Hkv + g) * P + key % P) * D + c * 8;
                 } else {
@@ -178,15 +187,24 @@ __global__ void __launch_bounds__(kTcRows, 1) prefill_tc_kernel(const PrefillPar
             cp_async16_zfill(dst_block + dst, static_cast<const T*>(pool) + off, valid);
         }
     };
-    auto load_k = [&](int blk) { if (blk < n_blocks) load_block(p.k, kring + (blk & 1) * S::kKvBytes, blk); };
-    auto load_v = [&](int blk) { if (blk < n_blocks) load_block(p.v, vring + (blk & 1) * S::kKvBytes, blk); };
-    // cp.async groups, in commit order: K0, V0, K1, then per iteration blk: K(blk+2), V(blk+1)
-    load_k(0);
+    auto load_k = [&](int blk, const int (&ids)[NPB]) {
+        if (blk < n_blocks) load_block(p.k, kring + (blk & 1) * S::kKvBytes, blk, ids);
+    };
+    auto load_v = [&](int blk, const int (&ids)[NPB]) {
+        if (blk < n_blocks) load_block(p.v, vring + (blk & 1) * S::kKvBytes, blk, ids);
+    };
+    // cp.async groups, in commit order: K0, V0, K1, then per iteration blk: K(blk+2), V(blk+1).
+    // Page ids in flight: ids_v = block blk + 1 (for V), ids_k = block blk + 2 (for K).
+    int ids_v[NPB], ids_k[NPB], ids_n[NPB];
+    fetch_ids(0, ids_n);
+    load_k(0, ids_n);
     cp_async_commit();
-    load_v(0);
+    load_v(0, ids_n);
     cp_async_commit();
-    load_k(1);
+    fetch_ids(1, ids_v);
+    load_k(1, ids_v);
     cp_async_commit();
+    fetch_ids(2, ids_k);
 
     // ---- TMEM and barriers
     const uint32_t tmem_cols = S::kTmemCols;
@@ -201,13 +219,19 @@ __global__ void __launch_bounds__(kTcRows, 1) prefill_tc_kernel(const PrefillPar
     }
     const uint32_t idesc_s = umma_idesc<T>(kTcRows, NK, false);
     const uint32_t idesc_o = umma_idesc<T>(kTcRows, D, true);
+    // Base descriptors; an operand's start moves by adding (bytes >> 4) to the low field
+    // (every address stays below 256 KB, so the 14-bit field never carries).
+    const uint64_t dq = umma_desc_sw128(smem_addr(qs), 16, 1024);
+    const uint64_t dk = umma_desc_sw128(smem_addr(kring), 16, 1024);
+    const uint64_t dv = umma_desc_sw128(smem_addr(vring), S::kRegion, 1024);
+    const uint64_t dp = umma_desc_sw128(smem_addr(ps), 16, 1024);
     // S = Q . K^T of block blk into the S columns
     auto issue_s = [&](int blk, uint32_t tm) {
-        const unsigned char* ks = kring + (blk & 1) * S::kKvBytes;
+        const uint32_t kst = (blk & 1) * S::kKvBytes;
 #pragma unroll
         for (int kk = 0; kk < KS; ++kk) {
-            const uint64_t ad = umma_desc_sw128(smem_addr(qs) + (kk / 4) * (kTcRows * 128) + (kk % 4) * 32, 16, 1024);
-            const uint64_t bd = umma_desc_sw128(smem_addr(ks) + (kk / 4) * S::kRegion + (kk % 4) * 32, 16, 1024);
+            const uint64_t ad = dq + (((kk / 4) * (kTcRows * 128) + (kk % 4) * 32) >> 4);
+            const uint64_t bd = dk + ((kst + (kk / 4) * S::kRegion + (kk % 4) * 32) >> 4);
             ptx::tcgen05_mma(ptx::kind_f16, ptx::cta_group_1, tm + D, ad, bd, idesc_s, kk > 0);
         }
         ptx::tcgen05_commit(ptx::cta_group_1, bar_s);
@@ -233,17 +257,22 @@ __global__ void __launch_bounds__(kTcRows, 1) prefill_tc_kernel(const PrefillPar
         }
         ptx::tcgen05_fence_after_thread_sync();
         float sv[NK];
-#pragma unroll
-        for (int j = 0; j < NK / 32; ++j) {
-            uint32_t r[32];
-            ptx::tcgen05_ld_32x32b(r, t_row + D + 32 * j);
+        {
+            uint32_t r0[32], r1[32];
+            ptx::tcgen05_ld_32x32b(r0, t_row + D);
+            if constexpr (NK == 64) ptx::tcgen05_ld_32x32b(r1, t_row + D + 32);
             ptx::tcgen05_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) sv[32 * j + i] = __uint_as_float(r[i]);
+            for (int i = 0; i < 32; ++i) sv[i] = __uint_as_float(r0[i]);
+            if constexpr (NK == 64) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) sv[32 + i] = __uint_as_float(r1[i]);
+            }
         }
         // K stage blk & 1 is free again (S(blk) is done): fetch K(blk + 2) into it
-        load_k(blk + 2);
+        load_k(blk + 2, ids_k);
         cp_async_commit();
+        fetch_ids(blk + 3, ids_n);               // used an iteration from now
         // ---- causal mask and online softmax of this thread's row.  The running max is
         //      taken over the raw scores (max of s * c is max(s) * c for c > 0, min(s) * c
         //      otherwise) and each p is exp2(s * c - m) with one packed FMA per pair.
@@ -253,20 +282,38 @@ __global__ void __launch_bounds__(kTcRows, 1) prefill_tc_kernel(const PrefillPar
 #pragma unroll
             for (int i = 0; i < NK; ++i) sv[i] = blk * NK + i <= pos ? sv[i] : sgn_inf;
         }
-        float ext = sgn_inf;
-        if (sc >= 0.f) {
+        float ext;
+        {
+            float e8[8];                         // eight independent chains, then a tree
 #pragma unroll
-            for (int i = 0; i < NK; ++i) ext = fmaxf(ext, sv[i]);
-        } else {
+            for (int k = 0; k < 8; ++k) e8[k] = sv[k];
+            if (sc >= 0.f) {
 #pragma unroll
-            for (int i = 0; i < NK; ++i) ext = fminf(ext, sv[i]);
+                for (int i = 8; i < NK; i += 8)
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) e8[k] = fmaxf(e8[k], sv[i + k]);
+#pragma unroll
+                for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+                    for (int k = 0; k < w; ++k) e8[k] = fmaxf(e8[k], e8[k + w]);
+            } else {
+#pragma unroll
+                for (int i = 8; i < NK; i += 8)
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) e8[k] = fminf(e8[k], sv[i + k]);
+#pragma unroll
+                for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+                    for (int k = 0; k < w; ++k) e8[k] = fminf(e8[k], e8[k + w]);
+            }
+            ext = e8[0];
         }
         const float mx = ext * sc;                 // -inf when every key of the block is masked
         const float mn = fmaxf(m_run, mx);
         const bool none = mn == -INFINITY;       // no visible key yet (or a row past the chunk)
         const float alpha = none ? 1.f : fast_exp2(m_run - mn);
         m_run = mn;
-        float2 ls2 = make_float2(0.f, 0.f);
+        float2 ls2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
         if (none) {
 #pragma unroll
             for (int i = 0; i < NK; ++i) sv[i] = 0.f;
@@ -277,10 +324,11 @@ __global__ void __launch_bounds__(kTcRows, 1) prefill_tc_kernel(const PrefillPar
                 const float2 t = __ffma2_rn(make_float2(sv[i], sv[i + 1]), c2, nm2);
                 sv[i] = fast_exp2(t.x);
                 sv[i + 1] = fast_exp2(t.y);
-                ls2 = __fadd2_rn(ls2, make_float2(sv[i], sv[i + 1]));
+                ls2[(i >> 1) & 3] = __fadd2_rn(ls2[(i >> 1) & 3], make_float2(sv[i], sv[i + 1]));
             }
         }
-        l_run = l_run * alpha + (ls2.x + ls2.y);
+        const float2 lsa = __fadd2_rn(__fadd2_rn(ls2[0], ls2[1]), __fadd2_rn(ls2[2], ls2[3]));
+        l_run = l_run * alpha + (lsa.x + lsa.y);
         // ---- the previous P.V must be done before O is rescaled, P rewritten and its stage refilled
         if (blk > 0) {
             if (!mbar_wait_parity_bounded(bar_o, (blk - 1) & 1)) {
@@ -290,20 +338,30 @@ __global__ void __launch_bounds__(kTcRows, 1) prefill_tc_kernel(const PrefillPar
             ptx::tcgen05_fence_after_thread_sync();
             if (__any_sync(0xffffffffu, alpha != 1.f)) {        // rescale this warp's O rows
 #pragma unroll
-                for (int c0 = 0; c0 < D; c0 += 32) {
-                    uint32_t r[32];
-                    ptx::tcgen05_ld_32x32b(r, t_row + c0);
+                for (int c0 = 0; c0 < D; c0 += 64) {   // two 32-column loads per wait
+                    uint32_t r0[32], r1[32];
+                    ptx::tcgen05_ld_32x32b(r0, t_row + c0);
+                    ptx::tcgen05_ld_32x32b(r1, t_row + c0 + 32);
                     ptx::tcgen05_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-                    ptx::tcgen05_st_32x32b(t_row + c0, r);
+                    for (int i = 0; i < 32; ++i) {
+                        r0[i] = __float_as_uint(__uint_as_float(r0[i]) * alpha);
+                        r1[i] = __float_as_uint(__uint_as_float(r1[i]) * alpha);
+                    }
+                    ptx::tcgen05_st_32x32b(t_row + c0, r0);
+                    ptx::tcgen05_st_32x32b(t_row + c0 + 32, r1);
                 }
                 ptx::tcgen05_wait_st();
             }
         }
         // V stage (blk + 1) & 1 last held V(blk - 1), whose P.V is complete
-        load_v(blk + 1);
+        load_v(blk + 1, ids_v);
         cp_async_commit();
+#pragma unroll
+        for (int j = 0; j < NPB; ++j) {
+            ids_v[j] = ids_k[j];
+            ids_k[j] = ids_n[j];
+        }
         // ---- this row of P (and of its low part) -> shared memory, K-major swizzled
 #pragma unroll
         for (int c = 0; c < NK / 8; ++c) {
@@ -329,13 +387,13 @@ __global__ void __launch_bounds__(kTcRows, 1) prefill_tc_kernel(const PrefillPar
         if (tid == 0) {
             // S of the next block first (it needs neither P nor O), then O += P . V
             if (blk + 1 < n_blocks) issue_s(blk + 1, tmem);
-            const unsigned char* vs = vring + (blk & 1) * S::kKvBytes;
+            const uint32_t vst = (blk & 1) * S::kKvBytes;
 #pragma unroll
             for (int part = 0; part < (kSplitP ? 2 : 1); ++part) {
 #pragma unroll
                 for (int kk = 0; kk < NK / 16; ++kk) {
-                    const uint64_t ad = umma_desc_sw128(smem_addr(ps) + part * S::kPBytes + kk * 32, 16, 1024);
-                    const uint64_t bd = umma_desc_sw128(smem_addr(vs) + kk * 2048, S::kRegion, 1024);
+                    const uint64_t ad = dp + ((part * S::kPBytes + kk * 32) >> 4);
+                    const uint64_t bd = dv + ((vst + kk * 2048) >> 4);
                     ptx::tcgen05_mma(ptx::kind_f16, ptx::cta_group_1, tmem, ad, bd, idesc_o, blk > 0 || kk > 0 || part > 0);
                 }
             }
