@@ -484,10 +484,10 @@ int launch_prefill(const PrefillParams& prm, int grid, cudaStream_t st)
 {
     static int configured[kMaxDevices] = {0};
     using S = TcShape<D, std::is_same<T, __nv_bfloat16>::value>;
-    const int smem = S::kBytes + 4 * (prm.batch + 1);
+    const int smem = S::kBytes + std::max(S::kTailMin, 4 * (prm.batch + 1));
     if (smem > kMaxSmemPerCta) return PKV_ERR_UNSUPPORTED;
     if (ensure_smem(prefill_tc_kernel<D, P, G, T>, smem, configured) != cudaSuccess) return PKV_ERR_CUDA;
-    return status_of(launch_pdl(prefill_tc_kernel<D, P, G, T>, dim3(grid), dim3(kTcRows), smem, st, prm));
+    return status_of(launch_pdl(prefill_tc_kernel<D, P, G, T>, dim3(grid), dim3(kTcThreads), smem, st, prm));
 }
 
 template <int D, int P, typename T>

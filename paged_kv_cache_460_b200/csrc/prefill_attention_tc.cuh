@@ -7,13 +7,16 @@
 // tcgen05: one elected thread issues the MMAs, operands come from shared memory, the
 // accumulators live in tensor memory (TMEM).
 //
-// Work: one CTA of 128 threads per (sequence, kv head, tile of 128 rows), a row being one
-// (query token, query head of the group) pair; thread t owns row t (TMEM lane t).  Per
-// block of NK keys (64 for fp16; 32 for bf16, whose P takes two buffers):
+// Work: one CTA of 256 threads per (sequence, kv head, tile of 128 rows), a row being one
+// (query token, query head of the group) pair.  Two threads share a row: thread t takes
+// row t % 128 (TMEM lane t % 128, which warps w and w + 4 both reach) and half t / 128 of
+// the row's key columns and of its O columns.  Per block of NK keys (64 for fp16; 32 for
+// bf16, whose P takes two buffers):
 //   S[128 x NK] = Q . K^T          tcgen05.mma kind::f16, M 128, N NK, D/16 k-steps -> TMEM
-//   each thread: its S row from TMEM, causal mask, fp32 online softmax (log2 domain), its
-//                O row rescaled in TMEM when its warp's running max moved, its P row
-//                written to shared memory
+//   each thread: its half of the S row from TMEM, causal mask, its half's max, combined
+//                with the partner's through a per-row shared-memory slot; fp32 online
+//                softmax (log2 domain), its half of P written to shared memory, its half
+//                of the O row rescaled in TMEM when its warp's running max moved
 //   O[128 x D] += P . V            M 128, N D, NK/16 k-steps (bf16: P as hi + lo, twice)
 // Shared memory uses the 128-byte-swizzle canonical layouts: Q, K and P K-major (rows of
 // 128 bytes, 16-byte chunk c of row r at c ^ (r & 7), 8-row atoms 1024 bytes apart, a
@@ -36,7 +39,9 @@
 
 namespace pkv {
 
-constexpr int kTcRows = 128;          // query rows per CTA (= threads = TMEM lanes)
+constexpr int kTcRows = 128;          // query rows per CTA (= TMEM lanes)
+constexpr int kTcThreads = 256;       // two threads per row
+constexpr float kLazyLog2 = 8.f;      // the softmax reference max moves only by more than this (log2)
 template <int D, bool kSplitP>
 struct TcShape {
     static constexpr int kKeys = kSplitP ? 32 : 64;             // keys per block
@@ -50,6 +55,9 @@ struct TcShape {
     static constexpr int kPOff = kVOff + 2 * kKvBytes;
     static constexpr int kBarOff = kPOff + (kSplitP ? 2 : 1) * kPBytes;
     static constexpr int kBytes = kBarOff + 64;                 // 2 mbarriers, TMEM base, abort flag
+    // after the fixed part: the work-item prefix [batch + 1] ints, reused once it has been
+    // searched as the per-row max slots [kTcRows] (so at least kTcRows ints)
+    static constexpr int kTailMin = kTcRows * 4;
     static constexpr uint32_t kTmemCols = D + kKeys <= 128 ? 128u : 256u;   // O at 0, S at D
 };
 
@@ -79,8 +87,20 @@ __device__ __forceinline__ bool mbar_wait_parity_bounded(uint64_t* bar, uint32_t
     }
 }
 
+// Order-preserving code of a float as an unsigned int (a > b as floats iff code(a) > code(b))
+__device__ __forceinline__ uint32_t float_order_code(float f)
+{
+    const uint32_t u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float float_from_order_code(uint32_t c)
+{
+    return __uint_as_float((c & 0x80000000u) ? (c & 0x7fffffffu) : ~c);
+}
+
 template <int D, int P, int G, typename T>
-__global__ void __launch_bounds__(kTcRows, 1) prefill_tc_kernel(const PrefillParams p)
+__global__ void __launch_bounds__(kTcThreads, 2) prefill_tc_kernel(const PrefillParams p)
 {
     namespace ptx = cuda::ptx;
     constexpr bool kSplitP = std::is_same<T, __nv_bfloat16>::value;
@@ -89,16 +109,23 @@ __global__ void __launch_bounds__(kTcRows, 1) prefill_tc_kernel(const PrefillPar
     constexpr int KS = D / 16;                 // k-steps of Q.K^T
     constexpr int CT = kTcRows / G;            // query tokens per CTA tile
     constexpr int NK = S::kKeys;               // keys per block
-    constexpr int NKC = NK * CPR / kTcRows;    // chunks per thread per K (or V) block
+    constexpr int NKH = NK / 2;                // keys of a block per thread
+    constexpr int DH = D / 2;                  // O columns per thread
+    constexpr int NKC = NK * CPR / kTcThreads; // chunks per thread per K (or V) block
     static_assert(G >= 1 && G <= 16 && 16 % G == 0, "group size");
     static_assert(D == 64 || D == 128, "head_dim");
+    static_assert(NK * CPR % kTcThreads == 0 && NKH % 8 == 0 && DH % 32 == 0, "tiling");
     extern __shared__ __align__(1024) unsigned char smem[];
     const int tid = threadIdx.x, warp = tid >> 5;
+    const int r = tid & (kTcRows - 1);         // this thread's row (TMEM lane)
+    const int half = tid / kTcRows;            // which half of the key and O columns
+    const int pair_bar = 1 + (warp & 3);       // named barrier of warps w and w + 4 (rows of one lane quarter)
     uint64_t* bar_s = reinterpret_cast<uint64_t*>(smem + S::kBarOff);
     uint64_t* bar_o = bar_s + 1;
     uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + S::kBarOff + 16);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S::kBarOff + 20);
     int* items = reinterpret_cast<int*>(smem + S::kBytes);   // [batch + 1] after the fixed part
+    uint32_t* mslot = reinterpret_cast<uint32_t*>(smem + S::kBytes);   // the same bytes, later
     const int Hkv = p.kv_heads;
 
     if (tid == 0) {
@@ -136,22 +163,24 @@ __global__ void __launch_bounds__(kTcRows, 1) prefill_tc_kernel(const PrefillPar
     const int n_blocks = (start + cta_last) / NK + 1;
 
     // this thread's row
-    const int tok = tile * CT + tid / G;
+    const int tok = tile * CT + r / G;
     const bool rvalid = tok < n_b;
     const int pos = rvalid ? start + tok : -1;
+    const long long row_elt = ((long long)(q0 + (rvalid ? tok : 0)) * p.q_heads + g * G + r % G) * D;
 
     unsigned char* qs = smem + S::kQOff;
     unsigned char* kring = smem + S::kKOff;
     unsigned char* vring = smem + S::kVOff;
     unsigned char* ps = smem + S::kPOff;
-    // ---- Q row -> shared memory (K-major, swizzled); rows past the chunk are zero
+    // ---- this thread's half of its Q row -> shared memory (K-major, swizzled); rows past
+    //      the chunk are zero
     {
-        const uint4* src = reinterpret_cast<const uint4*>(
-            static_cast<const T*>(p.q) + ((long long)(q0 + (rvalid ? tok : 0)) * p.q_heads + g * G + tid % G) * D);
+        const uint4* src = reinterpret_cast<const uint4*>(static_cast<const T*>(p.q) + row_elt);
 #pragma unroll
-        for (int c = 0; c < CPR; ++c) {
+        for (int cc = 0; cc < CPR / 2; ++cc) {
+            const int c = half * (CPR / 2) + cc;
             const uint4 v = rvalid ? src[c] : make_uint4(0u, 0u, 0u, 0u);
-            *reinterpret_cast<uint4*>(qs + (c / 8) * (kTcRows * 128) + tid * 128 + (((c % 8) ^ (tid & 7)) * 16)) = v;
+            *reinterpret_cast<uint4*>(qs + (c / 8) * (kTcRows * 128) + r * 128 + (((c % 8) ^ (r & 7)) * 16)) = v;
         }
     }
     // ---- K or V block loads (the same swizzled layout for both; keys past the cache are zero).
@@ -169,7 +198,7 @@ __global__ void __launch_bounds__(kTcRows, 1) prefill_tc_kernel(const PrefillPar
     auto load_block = [&](const void* pool, unsigned char* dst_block, int blk, const int (&ids)[NPB]) {
 #pragma unroll
         for (int n = 0; n < NKC; ++n) {
-            const int idx = n * kTcRows + tid;
+            const int idx = n * kTcThreads + tid;
             const int t = idx / CPR, c = idx % CPR;
             const int key = blk * NK + t;
             bool valid = key < L;
@@ -239,48 +268,48 @@ __global__ void __launch_bounds__(kTcRows, 1) prefill_tc_kernel(const PrefillPar
     cp_async_wait<2>();                          // K0 landed (V0, K1 may be in flight)
     fence_proxy_async_smem();
     ptx::tcgen05_fence_before_thread_sync();
-    __syncthreads();                             // Q, block 0, TMEM base and barriers ready
+    __syncthreads();                             // Q, block 0, TMEM base and barriers ready; items searched
     ptx::tcgen05_fence_after_thread_sync();
     const uint32_t tmem = *tslot;
-    const uint32_t t_row = tmem + ((uint32_t)(32 * warp) << 16);     // this warp's lane quarter
+    const uint32_t t_row = tmem + ((uint32_t)(32 * (warp & 3)) << 16);   // this warp's lane quarter
     if (tid == 0) issue_s(0, tmem);
+    // The row's max slot holds the running max over both halves' blocks so far; it only
+    // grows, so it needs no reset, and the CTA barrier that ends an iteration keeps either
+    // half from raising it for the next block before its partner has read it.
+    if (half == 0) mslot[r] = float_order_code(-INFINITY);
+    named_barrier(pair_bar, 64);
 
-    float m_run = -INFINITY, l_run = 0.f;
+    float m_run = -INFINITY, l_run = 0.f;        // l_run: this half's share of the row sum
     bool ok = true;
     int timed_out = 0;                           // this thread gave up on a wait; every exit is decided
                                                  // by a barrier over all threads, so it is uniform
+    const float sc = p.scale_log2 != 0.f ? p.scale_log2 : 1e-30f;   // zero: uniform weights, no 0 * inf
+    const float sgn_inf = sc >= 0.f ? -INFINITY : INFINITY;          // a masked score's raw value
     for (int blk = 0; blk < n_blocks; ++blk) {
-        // ---- S of this block from TMEM
+        // ---- this half of the S row of this block from TMEM
         if (!mbar_wait_parity_bounded(bar_s, blk & 1)) {
             timed_out = 1;
             atomicOr(&g_error_word, PKV_DEVERR_TIMEOUT);
         }
         ptx::tcgen05_fence_after_thread_sync();
-        float sv[NK];
+        float sv[NKH];
         {
-            uint32_t r0[32], r1[32];
-            ptx::tcgen05_ld_32x32b(r0, t_row + D);
-            if constexpr (NK == 64) ptx::tcgen05_ld_32x32b(r1, t_row + D + 32);
+            uint32_t r0[NKH];
+            ptx::tcgen05_ld_32x32b(r0, t_row + D + half * NKH);
             ptx::tcgen05_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) sv[i] = __uint_as_float(r0[i]);
-            if constexpr (NK == 64) {
-#pragma unroll
-                for (int i = 0; i < 32; ++i) sv[32 + i] = __uint_as_float(r1[i]);
-            }
+            for (int i = 0; i < NKH; ++i) sv[i] = __uint_as_float(r0[i]);
         }
         // K stage blk & 1 is free again (S(blk) is done): fetch K(blk + 2) into it
         load_k(blk + 2, ids_k);
         cp_async_commit();
         fetch_ids(blk + 3, ids_n);               // used an iteration from now
-        // ---- causal mask and online softmax of this thread's row.  The running max is
-        //      taken over the raw scores (max of s * c is max(s) * c for c > 0, min(s) * c
-        //      otherwise) and each p is exp2(s * c - m) with one packed FMA per pair.
-        const float sc = p.scale_log2 != 0.f ? p.scale_log2 : 1e-30f;   // zero: uniform weights, no 0 * inf
-        const float sgn_inf = sc >= 0.f ? -INFINITY : INFINITY;   // a masked score's raw value
-        if (__any_sync(0xffffffffu, blk * NK + NK - 1 > pos)) {   // some key of the block is past a row
+        // ---- causal mask and this half's max.  The max is taken over the raw scores (max
+        //      of s * c is max(s) * c for c > 0, min(s) * c otherwise).
+        const int key0 = blk * NK + half * NKH;
+        if (__any_sync(0xffffffffu, key0 + NKH - 1 > pos)) {    // some key of this half is past a row
 #pragma unroll
-            for (int i = 0; i < NK; ++i) sv[i] = blk * NK + i <= pos ? sv[i] : sgn_inf;
+            for (int i = 0; i < NKH; ++i) sv[i] = key0 + i <= pos ? sv[i] : sgn_inf;
         }
         float ext;
         {
@@ -289,7 +318,7 @@ __global__ void __launch_bounds__(kTcRows, 1) prefill_tc_kernel(const PrefillPar
             for (int k = 0; k < 8; ++k) e8[k] = sv[k];
             if (sc >= 0.f) {
 #pragma unroll
-                for (int i = 8; i < NK; i += 8)
+                for (int i = 8; i < NKH; i += 8)
 #pragma unroll
                     for (int k = 0; k < 8; ++k) e8[k] = fmaxf(e8[k], sv[i + k]);
 #pragma unroll
@@ -298,7 +327,7 @@ __global__ void __launch_bounds__(kTcRows, 1) prefill_tc_kernel(const PrefillPar
                     for (int k = 0; k < w; ++k) e8[k] = fmaxf(e8[k], e8[k + w]);
             } else {
 #pragma unroll
-                for (int i = 8; i < NK; i += 8)
+                for (int i = 8; i < NKH; i += 8)
 #pragma unroll
                     for (int k = 0; k < 8; ++k) e8[k] = fminf(e8[k], sv[i + k]);
 #pragma unroll
@@ -308,19 +337,28 @@ __global__ void __launch_bounds__(kTcRows, 1) prefill_tc_kernel(const PrefillPar
             }
             ext = e8[0];
         }
-        const float mx = ext * sc;                 // -inf when every key of the block is masked
-        const float mn = fmaxf(m_run, mx);
+        // ---- the row's max: both halves raise the slot, then read it back.  The reference
+        //      m_run the weights are taken against moves only when the max passes it by more
+        //      than kLazyLog2 (the result does not depend on the reference; weights stay
+        //      <= 2^kLazyLog2, well inside fp16), so O is rarely rescaled.
+        atomicMax(&mslot[r], float_order_code(ext * sc));   // -inf when every key of the half is masked
+        named_barrier(pair_bar, 64);
+        const float mt = float_from_order_code(mslot[r]);
+        float alpha = 1.f;
+        if (mt > m_run + kLazyLog2) {            // never while mt is -inf
+            alpha = fast_exp2(m_run - mt);       // 0 when m_run was -inf
+            m_run = mt;
+        }
+        const float mn = m_run;
         const bool none = mn == -INFINITY;       // no visible key yet (or a row past the chunk)
-        const float alpha = none ? 1.f : fast_exp2(m_run - mn);
-        m_run = mn;
         float2 ls2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
         if (none) {
 #pragma unroll
-            for (int i = 0; i < NK; ++i) sv[i] = 0.f;
+            for (int i = 0; i < NKH; ++i) sv[i] = 0.f;
         } else {
             const float2 c2 = make_float2(sc, sc), nm2 = make_float2(-mn, -mn);
 #pragma unroll
-            for (int i = 0; i < NK; i += 2) {
+            for (int i = 0; i < NKH; i += 2) {
                 const float2 t = __ffma2_rn(make_float2(sv[i], sv[i + 1]), c2, nm2);
                 sv[i] = fast_exp2(t.x);
                 sv[i + 1] = fast_exp2(t.y);
@@ -329,30 +367,49 @@ __global__ void __launch_bounds__(kTcRows, 1) prefill_tc_kernel(const PrefillPar
         }
         const float2 lsa = __fadd2_rn(__fadd2_rn(ls2[0], ls2[1]), __fadd2_rn(ls2[2], ls2[3]));
         l_run = l_run * alpha + (lsa.x + lsa.y);
-        // ---- the previous P.V must be done before O is rescaled, P rewritten and its stage refilled
+        // ---- the previous P.V must be done before P is rewritten, O rescaled and its V stage refilled
         if (blk > 0) {
             if (!mbar_wait_parity_bounded(bar_o, (blk - 1) & 1)) {
                 timed_out = 1;
                 atomicOr(&g_error_word, PKV_DEVERR_TIMEOUT);
             }
             ptx::tcgen05_fence_after_thread_sync();
-            if (__any_sync(0xffffffffu, alpha != 1.f)) {        // rescale this warp's O rows
+        }
+        // ---- this half of the row of P (and of its low part) -> shared memory, K-major swizzled
 #pragma unroll
-                for (int c0 = 0; c0 < D; c0 += 64) {   // two 32-column loads per wait
-                    uint32_t r0[32], r1[32];
-                    ptx::tcgen05_ld_32x32b(r0, t_row + c0);
-                    ptx::tcgen05_ld_32x32b(r1, t_row + c0 + 32);
-                    ptx::tcgen05_wait_ld();
+        for (int cc = 0; cc < NKH / 8; ++cc) {
+            const int c = half * (NKH / 8) + cc;
+            uint32_t w[4], wl[4];
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        r0[i] = __float_as_uint(__uint_as_float(r0[i]) * alpha);
-                        r1[i] = __float_as_uint(__uint_as_float(r1[i]) * alpha);
-                    }
-                    ptx::tcgen05_st_32x32b(t_row + c0, r0);
+            for (int e = 0; e < 4; ++e) {
+                const float a = sv[8 * cc + 2 * e], bb = sv[8 * cc + 2 * e + 1];
+                w[e] = MmaOps<T>::pack(a, bb);
+                if constexpr (kSplitP)
+                    wl[e] = MmaOps<T>::pack(a - __uint_as_float(w[e] << 16), bb - __uint_as_float(w[e] & 0xffff0000u));
+            }
+            const int off = r * 128 + ((c ^ (r & 7)) * 16);
+            *reinterpret_cast<uint4*>(ps + off) = make_uint4(w[0], w[1], w[2], w[3]);
+            if constexpr (kSplitP)
+                *reinterpret_cast<uint4*>(ps + S::kPBytes + off) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+        }
+        // ---- rescale this half of the warp's O rows
+        if (blk > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+            for (int c0 = half * DH; c0 < half * DH + DH; c0 += 64) {
+                uint32_t r0[32], r1[32];
+                ptx::tcgen05_ld_32x32b(r0, t_row + c0);
+                if constexpr (DH >= 64) ptx::tcgen05_ld_32x32b(r1, t_row + c0 + 32);
+                ptx::tcgen05_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) r0[i] = __float_as_uint(__uint_as_float(r0[i]) * alpha);
+                ptx::tcgen05_st_32x32b(t_row + c0, r0);
+                if constexpr (DH >= 64) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) r1[i] = __float_as_uint(__uint_as_float(r1[i]) * alpha);
                     ptx::tcgen05_st_32x32b(t_row + c0 + 32, r1);
                 }
-                ptx::tcgen05_wait_st();
             }
+            ptx::tcgen05_wait_st();
         }
         // V stage (blk + 1) & 1 last held V(blk - 1), whose P.V is complete
         load_v(blk + 1, ids_v);
@@ -361,22 +418,6 @@ __global__ void __launch_bounds__(kTcRows, 1) prefill_tc_kernel(const PrefillPar
         for (int j = 0; j < NPB; ++j) {
             ids_v[j] = ids_k[j];
             ids_k[j] = ids_n[j];
-        }
-        // ---- this row of P (and of its low part) -> shared memory, K-major swizzled
-#pragma unroll
-        for (int c = 0; c < NK / 8; ++c) {
-            uint32_t w[4], wl[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float a = sv[8 * c + 2 * e], bb = sv[8 * c + 2 * e + 1];
-                w[e] = MmaOps<T>::pack(a, bb);
-                if constexpr (kSplitP)
-                    wl[e] = MmaOps<T>::pack(a - __uint_as_float(w[e] << 16), bb - __uint_as_float(w[e] & 0xffff0000u));
-            }
-            const int off = tid * 128 + ((c ^ (tid & 7)) * 16);
-            *reinterpret_cast<uint4*>(ps + off) = make_uint4(w[0], w[1], w[2], w[3]);
-            if constexpr (kSplitP)
-                *reinterpret_cast<uint4*>(ps + S::kPBytes + off) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
         }
         cp_async_wait<2>();                      // K(blk + 1) and V(blk) landed (K(blk + 2), V(blk + 1) may not)
         fence_proxy_async_smem();
@@ -400,18 +441,25 @@ __global__ void __launch_bounds__(kTcRows, 1) prefill_tc_kernel(const PrefillPar
             ptx::tcgen05_commit(ptx::cta_group_1, bar_o);
         }
     }
-    // ---- out = O / l
+    // ---- out = O / l, l being the sum of the two halves' shares
     if (ok) {
         if (!mbar_wait_parity_bounded(bar_o, (n_blocks - 1) & 1)) timed_out = 1;
         ok = !__syncthreads_or(timed_out);
         if (!ok && tid == 0) atomicOr(&g_error_word, PKV_DEVERR_TIMEOUT);
         ptx::tcgen05_fence_after_thread_sync();
-        const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-        T* orow = static_cast<T*>(p.out) + ((long long)(q0 + (rvalid ? tok : 0)) * p.q_heads + g * G + tid % G) * D;
+        float l_row = 0.f;
+        if (ok) {                                // uniform; every MMA has completed, so P's bytes are free
+            float* lx = reinterpret_cast<float*>(ps);
+            lx[half * kTcRows + r] = l_run;
+            named_barrier(pair_bar, 64);
+            l_row = lx[r] + lx[kTcRows + r];
+        }
+        const float inv = l_row > 0.f ? 1.f / l_row : 0.f;
+        T* orow = static_cast<T*>(p.out) + row_elt;
 #pragma unroll
-        for (int c0 = 0; c0 < D; c0 += 32) {
-            uint32_t r[32];
-            ptx::tcgen05_ld_32x32b(r, t_row + c0);
+        for (int c0 = half * DH; c0 < half * DH + DH; c0 += 32) {
+            uint32_t rr[32];
+            ptx::tcgen05_ld_32x32b(rr, t_row + c0);
             ptx::tcgen05_wait_ld();
             if (ok && rvalid) {
 #pragma unroll
@@ -420,7 +468,7 @@ __global__ void __launch_bounds__(kTcRows, 1) prefill_tc_kernel(const PrefillPar
                     uint32_t* uw = reinterpret_cast<uint32_t*>(&u);
 #pragma unroll
                     for (int h = 0; h < 4; ++h)
-                        uw[h] = MmaOps<T>::pack(__uint_as_float(r[e + 2 * h]) * inv, __uint_as_float(r[e + 2 * h + 1]) * inv);
+                        uw[h] = MmaOps<T>::pack(__uint_as_float(rr[e + 2 * h]) * inv, __uint_as_float(rr[e + 2 * h + 1]) * inv);
                     *reinterpret_cast<uint4*>(orow + c0 + e) = u;
                 }
             }
