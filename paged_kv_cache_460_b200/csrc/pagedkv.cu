@@ -7,6 +7,7 @@
 // each kernel waits (griddepcontrol.wait) before touching data the previous kernel
 // may write.
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include <cstdint>
 #include <cstring>
@@ -479,13 +480,49 @@ extern "C" int paged_decode_layer(const pkv_pool* pool, int layer, void* out, co
 namespace pkv {
 namespace {
 
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
+{
+    static const PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return static_cast<PFN_cuTensorMapEncodeTiled_v12000>(nullptr);
+        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    }();
+    return fn;
+}
+
+// One layer's K or V pool [pages][kv_heads][P][D] as a 4-D tensor (D, P, kv_heads, pages),
+// box 64 x P x 1 x 1 with the 128-byte swizzle: one copy is one 64-column region of a page.
+template <int D, int P, typename T>
+bool encode_page_map(CUtensorMap* map, const void* base, int kv_heads, int num_pages)
+{
+    const PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)P, (cuuint64_t)kv_heads, (cuuint64_t)num_pages};
+    const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)P * D * 2, (cuuint64_t)kv_heads * P * D * 2};
+    const cuuint32_t box[4] = {64, (cuuint32_t)P, 1, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    const CUtensorMapDataType dt =
+        std::is_same<T, __half>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    return enc(map, dt, 4, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int D, int P, int G, typename T>
-int launch_prefill(const PrefillParams& prm, int grid, cudaStream_t st)
+int launch_prefill(const PrefillParams& prm_in, int grid, cudaStream_t st)
 {
     static int configured[kMaxDevices] = {0};
     using S = TcShape<D, std::is_same<T, __nv_bfloat16>::value>;
-    const int smem = S::kBytes + std::max(S::kTailMin, 4 * (prm.batch + 1));
+    const int smem = S::kBytes + std::max(S::kTailMin, 4 * (prm_in.batch + 1));
     if (smem > kMaxSmemPerCta) return PKV_ERR_UNSUPPORTED;
+    PrefillParams prm = prm_in;
+    if (!encode_page_map<D, P, T>(&prm.k_map, prm.k, prm.kv_heads, prm.num_pages) ||
+        !encode_page_map<D, P, T>(&prm.v_map, prm.v, prm.kv_heads, prm.num_pages))
+        return PKV_ERR_CUDA;
     if (ensure_smem(prefill_tc_kernel<D, P, G, T>, smem, configured) != cudaSuccess) return PKV_ERR_CUDA;
     return status_of(launch_pdl(prefill_tc_kernel<D, P, G, T>, dim3(grid), dim3(kTcThreads), smem, st, prm));
 }

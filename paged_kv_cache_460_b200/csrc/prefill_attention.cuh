@@ -1,6 +1,6 @@
 // Chunked prefill attention: the parameters shared by the host launcher and the
-// tensor-core kernel (prefill_attention_tc.cuh), and the zero-filling 16-byte copy used to
-// stage K/V blocks from the pages.
+// tensor-core kernel (prefill_attention_tc.cuh), and the tiled TMA load that stages K/V
+// blocks from the pages.
 //
 // "为什么要自己动手写一个LLM推理引擎" (wzjinhao.cn/news/61427) s4.3: the forward of a chunk
 // of seq_len new tokens at start_pos appends their k, v to the cache and applies the
@@ -9,6 +9,7 @@
 #ifndef PKV_PREFILL_ATTENTION_CUH_
 #define PKV_PREFILL_ATTENTION_CUH_
 
+#include <cuda.h>
 #include <type_traits>
 
 #include "decode_attention_mma.cuh"
@@ -16,6 +17,11 @@
 namespace pkv {
 
 struct PrefillParams {
+    // this layer's K and V pools [pages][kv_heads][P][D] as 4-D tensors (D, P, kv_heads,
+    // pages; box 64 x P x 1 x 1, 128-byte swizzle): one copy lands one 64-column region of
+    // one page in the canonical K-major layout
+    CUtensorMap k_map;
+    CUtensorMap v_map;
     const void* k;                 // this layer's K pool [pages][kv_heads][P][D]
     const void* v;
     const void* q;                 // [total_q][q_heads][D]
@@ -31,13 +37,15 @@ struct PrefillParams {
     float scale_log2;
 };
 
-// 16-byte cp.async that writes zeros instead when `valid` is false (src-size 0: nothing is
-// read from `src`, which must still be a mapped address).
-__device__ __forceinline__ void cp_async16_zfill(void* dst, const void* src, bool valid)
+// Tiled TMA load of box (x, y, z, w) of a 4-D tensor map into shared memory; completion is
+// counted in bytes on `bar`.  x must be a multiple of 8 elements (16 bytes).
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, int x, int y, int z, int w, uint64_t* bar)
 {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(dst)), "l"(src),
-                 "r"(valid ? 16u : 0u)
-                 : "memory");
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(
+            smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_addr(bar))
+        : "memory");
 }
 
 }  // namespace pkv

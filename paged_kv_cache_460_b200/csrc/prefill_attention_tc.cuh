@@ -54,7 +54,7 @@ struct TcShape {
     static constexpr int kVOff = kKOff + 2 * kKvBytes;          // V ring, 2 stages
     static constexpr int kPOff = kVOff + 2 * kKvBytes;
     static constexpr int kBarOff = kPOff + (kSplitP ? 2 : 1) * kPBytes;
-    static constexpr int kBytes = kBarOff + 64;                 // 2 mbarriers, TMEM base, abort flag
+    static constexpr int kBytes = kBarOff + 64;                 // 6 mbarriers, TMEM base, abort flag
     // after the fixed part: the work-item prefix [batch + 1] ints, reused once it has been
     // searched as the per-row max slots [kTcRows] (so at least kTcRows ints)
     static constexpr int kTailMin = kTcRows * 4;
@@ -100,7 +100,7 @@ __device__ __forceinline__ float float_from_order_code(uint32_t c)
 }
 
 template <int D, int P, int G, typename T>
-__global__ void __launch_bounds__(kTcThreads, 2) prefill_tc_kernel(const PrefillParams p)
+__global__ void __launch_bounds__(kTcThreads, 2) prefill_tc_kernel(const __grid_constant__ PrefillParams p)
 {
     namespace ptx = cuda::ptx;
     constexpr bool kSplitP = std::is_same<T, __nv_bfloat16>::value;
@@ -111,19 +111,24 @@ __global__ void __launch_bounds__(kTcThreads, 2) prefill_tc_kernel(const Prefill
     constexpr int NK = S::kKeys;               // keys per block
     constexpr int NKH = NK / 2;                // keys of a block per thread
     constexpr int DH = D / 2;                  // O columns per thread
-    constexpr int NKC = NK * CPR / kTcThreads; // chunks per thread per K (or V) block
+    constexpr int NPB = NK / P;                // pages per block
+    constexpr uint32_t kPageBytes = (D / 64) * P * 128;   // one page of one block (all its regions)
     static_assert(G >= 1 && G <= 16 && 16 % G == 0, "group size");
     static_assert(D == 64 || D == 128, "head_dim");
-    static_assert(NK * CPR % kTcThreads == 0 && NKH % 8 == 0 && DH % 32 == 0, "tiling");
-    extern __shared__ __align__(1024) unsigned char smem[];
+    static_assert(NK % P == 0 && NKH % 8 == 0 && DH % 32 == 0, "tiling");
+    extern __shared__ __align__(1024) unsigned char tc_smem[];    // own name: other kernels align theirs to 128
+    unsigned char* const smem = tc_smem;
     const int tid = threadIdx.x, warp = tid >> 5;
     const int r = tid & (kTcRows - 1);         // this thread's row (TMEM lane)
     const int half = tid / kTcRows;            // which half of the key and O columns
     const int pair_bar = 1 + (warp & 3);       // named barrier of warps w and w + 4 (rows of one lane quarter)
+    const bool k_loader = tid == 32, v_loader = tid == 64;
     uint64_t* bar_s = reinterpret_cast<uint64_t*>(smem + S::kBarOff);
     uint64_t* bar_o = bar_s + 1;
-    uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + S::kBarOff + 16);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S::kBarOff + 20);
+    uint64_t* full_k = bar_s + 2;              // [2]: K stage landed
+    uint64_t* full_v = bar_s + 4;              // [2]: V stage landed
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + S::kBarOff + 48);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S::kBarOff + 52);
     int* items = reinterpret_cast<int*>(smem + S::kBytes);   // [batch + 1] after the fixed part
     uint32_t* mslot = reinterpret_cast<uint32_t*>(smem + S::kBytes);   // the same bytes, later
     const int Hkv = p.kv_heads;
@@ -137,6 +142,8 @@ __global__ void __launch_bounds__(kTcThreads, 2) prefill_tc_kernel(const Prefill
         }
         items[p.batch] = run;
         *abort_flag = (smem_addr(smem) & 1023u) != 0;     // the swizzle atoms need 1024-byte alignment
+        for (int i = 0; i < 6; ++i) mbar_init(bar_s + i, 1);
+        fence_barrier_init();
     }
     __syncthreads();
     pdl_wait();
@@ -172,6 +179,53 @@ __global__ void __launch_bounds__(kTcThreads, 2) prefill_tc_kernel(const Prefill
     unsigned char* kring = smem + S::kKOff;
     unsigned char* vring = smem + S::kVOff;
     unsigned char* ps = smem + S::kPOff;
+    // ---- K and V blocks: one thread each issues the block's TMA copies, a 64-column region
+    //      of a page at a time, into the stage's canonical swizzled layout, and counts the
+    //      bytes on the stage's barrier.  Page ids are fetched a block ahead.  Pages past the
+    //      cache are not read; a page id out of range is flagged and never read.
+    const int32_t* table = p.block_tables + (long long)b * p.max_pages;
+    auto fetch_ids = [&](int blk, int (&ids)[NPB]) {
+#pragma unroll
+        for (int j = 0; j < NPB; ++j) {
+            const int pg = blk * NPB + j;
+            ids[j] = pg * P < L ? (pg < p.max_pages ? table[pg] : -1) : -2;
+        }
+    };
+    auto tma_block = [&](const CUtensorMap* map, unsigned char* dst_block, uint64_t* full, const int (&ids)[NPB]) {
+        uint32_t bytes = 0;
+#pragma unroll
+        for (int j = 0; j < NPB; ++j) bytes += (unsigned)ids[j] < (unsigned)p.num_pages ? kPageBytes : 0u;
+        mbar_arrive_expect_tx(full, bytes);
+#pragma unroll
+        for (int j = 0; j < NPB; ++j) {
+            if ((unsigned)ids[j] < (unsigned)p.num_pages) {
+#pragma unroll
+                for (int rg = 0; rg < D / 64; ++rg)
+                    tma_load_4d(dst_block + rg * S::kRegion + j * P * 128, map, 64 * rg, 0, g, ids[j], full);
+            } else if (ids[j] != -2) {
+                atomicOr(&g_error_word, PKV_DEVERR_BAD_PAGE);
+            }
+        }
+    };
+    int ids_a[NPB];                             // the next block the loader copies
+    int issued = 0;                             // blocks this loader has copied: 0 .. issued - 1
+    if (k_loader) {
+        fetch_ids(0, ids_a);
+        tma_block(&p.k_map, kring, full_k, ids_a);
+        issued = 1;
+        if (n_blocks > 1) {
+            fetch_ids(1, ids_a);
+            tma_block(&p.k_map, kring + S::kKvBytes, full_k + 1, ids_a);
+            issued = 2;
+        }
+        fetch_ids(2, ids_a);
+    }
+    if (v_loader) {
+        fetch_ids(0, ids_a);
+        tma_block(&p.v_map, vring, full_v, ids_a);
+        issued = 1;
+        fetch_ids(1, ids_a);
+    }
     // ---- this thread's half of its Q row -> shared memory (K-major, swizzled); rows past
     //      the chunk are zero
     {
@@ -183,68 +237,12 @@ __global__ void __launch_bounds__(kTcThreads, 2) prefill_tc_kernel(const Prefill
             *reinterpret_cast<uint4*>(qs + (c / 8) * (kTcRows * 128) + r * 128 + (((c % 8) ^ (r & 7)) * 16)) = v;
         }
     }
-    // ---- K or V block loads (the same swizzled layout for both; keys past the cache are zero).
-    // The page ids of a block are fetched an iteration before its copies are issued, so the
-    // copies never wait on the page table.
-    constexpr int NPB = NK / P > 0 ? NK / P : 1;    // pages per block
-    const int32_t* table = p.block_tables + (long long)b * p.max_pages;
-    auto fetch_ids = [&](int blk, int (&ids)[NPB]) {
-#pragma unroll
-        for (int j = 0; j < NPB; ++j) {
-            const int pg = (blk * NK) / P + j;
-            ids[j] = pg * P < L ? (pg < p.max_pages ? table[pg] : -1) : -2;
-        }
-    };
-    auto load_block = [&](const void* pool, unsigned char* dst_block, int blk, const int (&ids)[NPB]) {
-#pragma unroll
-        for (int n = 0; n < NKC; ++n) {
-            const int idx = n * kTcThreads + tid;
-            const int t = idx / CPR, c = idx % CPR;
-            const int key = blk * NK + t;
-            bool valid = key < L;
-            long long off = 0;
-            if (valid) {
-                const int page = ids[(t % NK) / P];
-                if ((unsigned)page < (unsigned)p.num_pages) {
-                    off = (((long long)page * Hkv + g) * P + key % P) * D + c * 8;
-                } else {
-                    valid = false;
-                    if (c == 0) atomicOr(&g_error_word, PKV_DEVERR_BAD_PAGE);   // never dereferenced
-                }
-            }
-            const int dst = (c / 8) * S::kRegion + t * 128 + (((c % 8) ^ (t & 7)) * 16);
-            cp_async16_zfill(dst_block + dst, static_cast<const T*>(pool) + off, valid);
-        }
-    };
-    auto load_k = [&](int blk, const int (&ids)[NPB]) {
-        if (blk < n_blocks) load_block(p.k, kring + (blk & 1) * S::kKvBytes, blk, ids);
-    };
-    auto load_v = [&](int blk, const int (&ids)[NPB]) {
-        if (blk < n_blocks) load_block(p.v, vring + (blk & 1) * S::kKvBytes, blk, ids);
-    };
-    // cp.async groups, in commit order: K0, V0, K1, then per iteration blk: K(blk+2), V(blk+1).
-    // Page ids in flight: ids_v = block blk + 1 (for V), ids_k = block blk + 2 (for K).
-    int ids_v[NPB], ids_k[NPB], ids_n[NPB];
-    fetch_ids(0, ids_n);
-    load_k(0, ids_n);
-    cp_async_commit();
-    load_v(0, ids_n);
-    cp_async_commit();
-    fetch_ids(1, ids_v);
-    load_k(1, ids_v);
-    cp_async_commit();
-    fetch_ids(2, ids_k);
 
-    // ---- TMEM and barriers
+    // ---- TMEM
     const uint32_t tmem_cols = S::kTmemCols;
     if (warp == 0) {
         ptx::tcgen05_alloc(ptx::cta_group_1, tslot, tmem_cols);
         ptx::tcgen05_relinquish_alloc_permit(ptx::cta_group_1);
-    }
-    if (tid == 0) {
-        mbar_init(bar_s, 1);
-        mbar_init(bar_o, 1);
-        fence_barrier_init();
     }
     const uint32_t idesc_s = umma_idesc<T>(kTcRows, NK, false);
     const uint32_t idesc_o = umma_idesc<T>(kTcRows, D, true);
@@ -265,14 +263,19 @@ __global__ void __launch_bounds__(kTcThreads, 2) prefill_tc_kernel(const Prefill
         }
         ptx::tcgen05_commit(ptx::cta_group_1, bar_s);
     };
-    cp_async_wait<2>();                          // K0 landed (V0, K1 may be in flight)
+    int timed_out = 0;                           // this thread gave up on a wait; every exit is decided
+                                                 // by a barrier over all threads, so it is uniform
+    if (tid == 0 && !mbar_wait_parity_bounded(full_k, 0)) {     // K0 landed
+        timed_out = 1;
+        atomicOr(&g_error_word, PKV_DEVERR_TIMEOUT);
+    }
     fence_proxy_async_smem();
     ptx::tcgen05_fence_before_thread_sync();
-    __syncthreads();                             // Q, block 0, TMEM base and barriers ready; items searched
+    bool ok = !__syncthreads_or(timed_out);      // Q, K0 and the TMEM base ready; items searched
     ptx::tcgen05_fence_after_thread_sync();
     const uint32_t tmem = *tslot;
     const uint32_t t_row = tmem + ((uint32_t)(32 * (warp & 3)) << 16);   // this warp's lane quarter
-    if (tid == 0) issue_s(0, tmem);
+    if (tid == 0 && ok) issue_s(0, tmem);
     // The row's max slot holds the running max over both halves' blocks so far; it only
     // grows, so it needs no reset, and the CTA barrier that ends an iteration keeps either
     // half from raising it for the next block before its partner has read it.
@@ -280,12 +283,9 @@ __global__ void __launch_bounds__(kTcThreads, 2) prefill_tc_kernel(const Prefill
     named_barrier(pair_bar, 64);
 
     float m_run = -INFINITY, l_run = 0.f;        // l_run: this half's share of the row sum
-    bool ok = true;
-    int timed_out = 0;                           // this thread gave up on a wait; every exit is decided
-                                                 // by a barrier over all threads, so it is uniform
     const float sc = p.scale_log2 != 0.f ? p.scale_log2 : 1e-30f;   // zero: uniform weights, no 0 * inf
     const float sgn_inf = sc >= 0.f ? -INFINITY : INFINITY;          // a masked score's raw value
-    for (int blk = 0; blk < n_blocks; ++blk) {
+    for (int blk = 0; ok && blk < n_blocks; ++blk) {
         // ---- this half of the S row of this block from TMEM
         if (!mbar_wait_parity_bounded(bar_s, blk & 1)) {
             timed_out = 1;
@@ -301,9 +301,13 @@ __global__ void __launch_bounds__(kTcThreads, 2) prefill_tc_kernel(const Prefill
             for (int i = 0; i < NKH; ++i) sv[i] = __uint_as_float(r0[i]);
         }
         // K stage blk & 1 is free again (S(blk) is done): fetch K(blk + 2) into it
-        load_k(blk + 2, ids_k);
-        cp_async_commit();
-        fetch_ids(blk + 3, ids_n);               // used an iteration from now
+        if (k_loader) {
+            if (blk + 2 < n_blocks) {
+                tma_block(&p.k_map, kring + (blk & 1) * S::kKvBytes, full_k + (blk & 1), ids_a);
+                issued = blk + 3;
+            }
+            fetch_ids(blk + 3, ids_a);           // used an iteration from now
+        }
         // ---- causal mask and this half's max.  The max is taken over the raw scores (max
         //      of s * c is max(s) * c for c > 0, min(s) * c otherwise).
         const int key0 = blk * NK + half * NKH;
@@ -375,6 +379,14 @@ __global__ void __launch_bounds__(kTcThreads, 2) prefill_tc_kernel(const Prefill
             }
             ptx::tcgen05_fence_after_thread_sync();
         }
+        // V stage (blk + 1) & 1 last held V(blk - 1), whose P.V is complete
+        if (v_loader) {
+            if (blk + 1 < n_blocks) {
+                tma_block(&p.v_map, vring + ((blk + 1) & 1) * S::kKvBytes, full_v + ((blk + 1) & 1), ids_a);
+                issued = blk + 2;
+            }
+            fetch_ids(blk + 2, ids_a);
+        }
         // ---- this half of the row of P (and of its low part) -> shared memory, K-major swizzled
 #pragma unroll
         for (int cc = 0; cc < NKH / 8; ++cc) {
@@ -411,15 +423,30 @@ __global__ void __launch_bounds__(kTcThreads, 2) prefill_tc_kernel(const Prefill
             }
             ptx::tcgen05_wait_st();
         }
-        // V stage (blk + 1) & 1 last held V(blk - 1), whose P.V is complete
-        load_v(blk + 1, ids_v);
-        cp_async_commit();
-#pragma unroll
-        for (int j = 0; j < NPB; ++j) {
-            ids_v[j] = ids_k[j];
-            ids_k[j] = ids_n[j];
+        // ---- the block holding the end of the cache: its V rows past the cache (stale or
+        //      never written) become zeros, so that their zero weights give exact zeros
+        const int past = L - blk * NK;           // rows [past, NK) of this block lie past the cache
+        if (past < NK) {
+            if (!mbar_wait_parity_bounded(full_v + (blk & 1), (blk >> 1) & 1)) {
+                timed_out = 1;
+                atomicOr(&g_error_word, PKV_DEVERR_TIMEOUT);
+            } else {
+                unsigned char* vb = vring + (blk & 1) * S::kKvBytes;
+                const int chunks = (NK - past) * 8 * (D / 64);
+                for (int i = tid; i < chunks; i += kTcThreads) {
+                    const int rg = i / ((NK - past) * 8), rest = i % ((NK - past) * 8);
+                    *reinterpret_cast<uint4*>(vb + rg * S::kRegion + (past + rest / 8) * 128 + (rest % 8) * 16) =
+                        make_uint4(0u, 0u, 0u, 0u);
+                }
+            }
         }
-        cp_async_wait<2>();                      // K(blk + 1) and V(blk) landed (K(blk + 2), V(blk + 1) may not)
+        // ---- the MMA issuer: K(blk + 1) and V(blk) must have landed
+        if (tid == 0) {
+            if (blk + 1 < n_blocks && !mbar_wait_parity_bounded(full_k + ((blk + 1) & 1), ((blk + 1) >> 1) & 1))
+                timed_out = 1;
+            if (!mbar_wait_parity_bounded(full_v + (blk & 1), (blk >> 1) & 1)) timed_out = 1;
+            if (timed_out) atomicOr(&g_error_word, PKV_DEVERR_TIMEOUT);
+        }
         fence_proxy_async_smem();
         ptx::tcgen05_fence_before_thread_sync();
         const int stop = __syncthreads_or(timed_out);   // P, rescaled O, S reads and block blk + 1 ready
@@ -474,7 +501,12 @@ __global__ void __launch_bounds__(kTcThreads, 2) prefill_tc_kernel(const Prefill
             }
         }
     }
-    cp_async_wait<0>();
+    // ---- copies still in flight (only after a timeout): each loader waits, bounded, for the
+    //      last copy it issued into each stage before the CTA's shared memory is released
+    if (k_loader || v_loader) {
+        uint64_t* full = k_loader ? full_k : full_v;
+        for (int j = max(0, issued - 2); j < issued; ++j) mbar_wait_parity_bounded(full + (j & 1), (j >> 1) & 1);
+    }
     ptx::tcgen05_fence_before_thread_sync();
     __syncthreads();
     if (warp == 0) ptx::tcgen05_dealloc(ptx::cta_group_1, tmem, tmem_cols);
