@@ -15,20 +15,23 @@
 //   S[128 x NK] = Q . K^T          tcgen05.mma kind::f16, M 128, N NK, D/16 k-steps -> TMEM
 //   each thread: its half of the S row from TMEM, causal mask, its half's max, combined
 //                with the partner's through a per-row shared-memory slot; fp32 online
-//                softmax (log2 domain), its half of P written to shared memory, its half
-//                of the O row rescaled in TMEM when its warp's running max moved
+//                softmax (log2 domain) against a reference max that moves only when the
+//                row max passes it by more than 2^8, so O is rarely rescaled; its half of
+//                P written to shared memory, its half of the O row rescaled in TMEM when
+//                the reference moved
 //   O[128 x D] += P . V            M 128, N D, NK/16 k-steps (bf16: P as hi + lo, twice)
 // Shared memory uses the 128-byte-swizzle canonical layouts: Q, K and P K-major (rows of
 // 128 bytes, 16-byte chunk c of row r at c ^ (r & 7), 8-row atoms 1024 bytes apart, a
 // region per 64 columns), V MN-major -- which is the same bytes as K's layout read with
-// the other major-ness, so K and V blocks are staged identically by cp.async from the
-// pages (keys past the cache zero-filled by the copy).  K and V blocks go through rings of
-// their own (two stages each): K(b) is refilled as soon as S(b) is done, V(b) as soon as
-// P.V(b) is, so each load has an iteration to land; and the elected thread issues S of the
-// next block before P.V of the current one (each with its own commit), so the next softmax
-// can start while P.V is still on the tensor cores.  Every wait on
-// an MMA is bounded: on timeout the kernel sets PKV_DEVERR_TIMEOUT, skips its output and
-// still frees its TMEM.
+// the other major-ness, so K and V blocks are staged identically: one thread each issues
+// tiled TMA copies (a 64-column region of one page per copy) into two-stage rings, counted
+// in bytes on a barrier per stage.  K(b) is refilled as soon as S(b) is done, V(b) as soon
+// as P.V(b) is; V rows past the cache are zeroed after their copy lands.  S has two TMEM
+// buffers: at the end of block b warp 0 (one elected lane) issues P.V(b), then S(b + 2)
+// into the buffer block b has emptied, so S of the next block is already on hand when its
+// softmax starts.  Every wait on an MMA or a copy is bounded: on timeout the kernel sets
+// PKV_DEVERR_TIMEOUT, skips its output, waits (bounded) for its copies in flight and still
+// frees its TMEM.
 #ifndef PKV_PREFILL_ATTENTION_TC_CUH_
 #define PKV_PREFILL_ATTENTION_TC_CUH_
 
@@ -58,7 +61,7 @@ struct TcShape {
     // after the fixed part: the work-item prefix [batch + 1] ints, reused once it has been
     // searched as the per-row max slots [kTcRows] (so at least kTcRows ints)
     static constexpr int kTailMin = kTcRows * 4;
-    static constexpr uint32_t kTmemCols = D + kKeys <= 128 ? 128u : 256u;   // O at 0, S at D
+    static constexpr uint32_t kTmemCols = D + 2 * kKeys <= 128 ? 128u : 256u;   // O at 0, S twice from D
 };
 
 // UMMA shared-memory descriptor, 128-byte swizzle (start, leading and stride byte offsets)
@@ -99,6 +102,31 @@ __device__ __forceinline__ float float_from_order_code(uint32_t c)
     return __uint_as_float((c & 0x80000000u) ? (c & 0x7fffffffu) : ~c);
 }
 
+// tcgen05.mma kind::f16 / tcgen05.commit issued by one elected lane of a converged warp; the
+// whole warp computes the (warp-uniform) operands
+__device__ __forceinline__ void umma_f16_elected(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                 bool accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred e, p;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+        "}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"((uint32_t)accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void umma_commit_elected(uint64_t* bar)
+{
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t"
+        "}" ::"r"(smem_addr(bar))
+        : "memory");
+}
+
 template <int D, int P, int G, typename T>
 __global__ void __launch_bounds__(kTcThreads, 2) prefill_tc_kernel(const __grid_constant__ PrefillParams p)
 {
@@ -123,12 +151,12 @@ __global__ void __launch_bounds__(kTcThreads, 2) prefill_tc_kernel(const __grid_
     const int half = tid / kTcRows;            // which half of the key and O columns
     const int pair_bar = 1 + (warp & 3);       // named barrier of warps w and w + 4 (rows of one lane quarter)
     const bool k_loader = tid == 32, v_loader = tid == 64;
-    uint64_t* bar_s = reinterpret_cast<uint64_t*>(smem + S::kBarOff);
-    uint64_t* bar_o = bar_s + 1;
-    uint64_t* full_k = bar_s + 2;              // [2]: K stage landed
-    uint64_t* full_v = bar_s + 4;              // [2]: V stage landed
-    uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + S::kBarOff + 48);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S::kBarOff + 52);
+    uint64_t* bar_s = reinterpret_cast<uint64_t*>(smem + S::kBarOff);   // [2]: S buffer done
+    uint64_t* bar_o = bar_s + 2;
+    uint64_t* full_k = bar_s + 3;              // [2]: K stage landed
+    uint64_t* full_v = bar_s + 5;              // [2]: V stage landed
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + S::kBarOff + 56);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S::kBarOff + 60);
     int* items = reinterpret_cast<int*>(smem + S::kBytes);   // [batch + 1] after the fixed part
     uint32_t* mslot = reinterpret_cast<uint32_t*>(smem + S::kBytes);   // the same bytes, later
     const int Hkv = p.kv_heads;
@@ -142,7 +170,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) prefill_tc_kernel(const __grid_
         }
         items[p.batch] = run;
         *abort_flag = (smem_addr(smem) & 1023u) != 0;     // the swizzle atoms need 1024-byte alignment
-        for (int i = 0; i < 6; ++i) mbar_init(bar_s + i, 1);
+        for (int i = 0; i < 7; ++i) mbar_init(bar_s + i, 1);
         fence_barrier_init();
     }
     __syncthreads();
@@ -259,13 +287,14 @@ __global__ void __launch_bounds__(kTcThreads, 2) prefill_tc_kernel(const __grid_
         for (int kk = 0; kk < KS; ++kk) {
             const uint64_t ad = dq + (((kk / 4) * (kTcRows * 128) + (kk % 4) * 32) >> 4);
             const uint64_t bd = dk + ((kst + (kk / 4) * S::kRegion + (kk % 4) * 32) >> 4);
-            ptx::tcgen05_mma(ptx::kind_f16, ptx::cta_group_1, tm + D, ad, bd, idesc_s, kk > 0);
+            umma_f16_elected(tm + D + (blk & 1) * NK, ad, bd, idesc_s, kk > 0);
         }
-        ptx::tcgen05_commit(ptx::cta_group_1, bar_s);
+        umma_commit_elected(bar_s + (blk & 1));
     };
     int timed_out = 0;                           // this thread gave up on a wait; every exit is decided
                                                  // by a barrier over all threads, so it is uniform
-    if (tid == 0 && !mbar_wait_parity_bounded(full_k, 0)) {     // K0 landed
+    if (tid == 0 && (!mbar_wait_parity_bounded(full_k, 0) ||
+                     (n_blocks > 1 && !mbar_wait_parity_bounded(full_k + 1, 0)))) {     // K0, K1 landed
         timed_out = 1;
         atomicOr(&g_error_word, PKV_DEVERR_TIMEOUT);
     }
@@ -275,7 +304,10 @@ __global__ void __launch_bounds__(kTcThreads, 2) prefill_tc_kernel(const __grid_
     ptx::tcgen05_fence_after_thread_sync();
     const uint32_t tmem = *tslot;
     const uint32_t t_row = tmem + ((uint32_t)(32 * (warp & 3)) << 16);   // this warp's lane quarter
-    if (tid == 0 && ok) issue_s(0, tmem);
+    if (warp == 0 && ok) {                       // the whole warp: one elected lane issues
+        issue_s(0, tmem);
+        if (n_blocks > 1) issue_s(1, tmem);
+    }
     // The row's max slot holds the running max over both halves' blocks so far; it only
     // grows, so it needs no reset, and the CTA barrier that ends an iteration keeps either
     // half from raising it for the next block before its partner has read it.
@@ -287,7 +319,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) prefill_tc_kernel(const __grid_
     const float sgn_inf = sc >= 0.f ? -INFINITY : INFINITY;          // a masked score's raw value
     for (int blk = 0; ok && blk < n_blocks; ++blk) {
         // ---- this half of the S row of this block from TMEM
-        if (!mbar_wait_parity_bounded(bar_s, blk & 1)) {
+        if (!mbar_wait_parity_bounded(bar_s + (blk & 1), (blk >> 1) & 1)) {
             timed_out = 1;
             atomicOr(&g_error_word, PKV_DEVERR_TIMEOUT);
         }
@@ -295,7 +327,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) prefill_tc_kernel(const __grid_
         float sv[NKH];
         {
             uint32_t r0[NKH];
-            ptx::tcgen05_ld_32x32b(r0, t_row + D + half * NKH);
+            ptx::tcgen05_ld_32x32b(r0, t_row + D + (blk & 1) * NK + half * NKH);
             ptx::tcgen05_wait_ld();
 #pragma unroll
             for (int i = 0; i < NKH; ++i) sv[i] = __uint_as_float(r0[i]);
@@ -440,9 +472,9 @@ __global__ void __launch_bounds__(kTcThreads, 2) prefill_tc_kernel(const __grid_
                 }
             }
         }
-        // ---- the MMA issuer: K(blk + 1) and V(blk) must have landed
+        // ---- the MMA issuer: K(blk + 2) and V(blk) must have landed
         if (tid == 0) {
-            if (blk + 1 < n_blocks && !mbar_wait_parity_bounded(full_k + ((blk + 1) & 1), ((blk + 1) >> 1) & 1))
+            if (blk + 2 < n_blocks && !mbar_wait_parity_bounded(full_k + (blk & 1), ((blk + 2) >> 1) & 1))
                 timed_out = 1;
             if (!mbar_wait_parity_bounded(full_v + (blk & 1), (blk >> 1) & 1)) timed_out = 1;
             if (timed_out) atomicOr(&g_error_word, PKV_DEVERR_TIMEOUT);
@@ -452,9 +484,8 @@ __global__ void __launch_bounds__(kTcThreads, 2) prefill_tc_kernel(const __grid_
         const int stop = __syncthreads_or(timed_out);   // P, rescaled O, S reads and block blk + 1 ready
         ptx::tcgen05_fence_after_thread_sync();
         if (stop) { ok = false; break; }
-        if (tid == 0) {
-            // S of the next block first (it needs neither P nor O), then O += P . V
-            if (blk + 1 < n_blocks) issue_s(blk + 1, tmem);
+        if (warp == 0) {
+            // O += P . V, then S two blocks ahead into the S buffer this block has emptied
             const uint32_t vst = (blk & 1) * S::kKvBytes;
 #pragma unroll
             for (int part = 0; part < (kSplitP ? 2 : 1); ++part) {
@@ -462,10 +493,11 @@ __global__ void __launch_bounds__(kTcThreads, 2) prefill_tc_kernel(const __grid_
                 for (int kk = 0; kk < NK / 16; ++kk) {
                     const uint64_t ad = dp + ((part * S::kPBytes + kk * 32) >> 4);
                     const uint64_t bd = dv + ((vst + kk * 2048) >> 4);
-                    ptx::tcgen05_mma(ptx::kind_f16, ptx::cta_group_1, tmem, ad, bd, idesc_o, blk > 0 || kk > 0 || part > 0);
+                    umma_f16_elected(tmem, ad, bd, idesc_o, blk > 0 || kk > 0 || part > 0);
                 }
             }
-            ptx::tcgen05_commit(ptx::cta_group_1, bar_o);
+            umma_commit_elected(bar_o);
+            if (blk + 2 < n_blocks) issue_s(blk + 2, tmem);
         }
     }
     // ---- out = O / l, l being the sum of the two halves' shares
