@@ -302,8 +302,11 @@ int paged_decode_attention_noalloc(const pkv_pool* pool, int layer, void* out, c
  *   block_tables, max_pages_per_seq, kv_heads, scale: as for paged_decode_attention;
  *   q_heads / kv_heads in {1, 2, 4, 8}.
  * One CTA per (sequence, kv head, 128 query rows) on the fifth-generation tensor cores
- * (tcgen05.mma, S and O accumulated in tensor memory; fp32 online softmax); no workspace.
- * Errors as for paged_decode_attention; on an int8 pool, UNSUPPORTED.
+ * (tcgen05.mma, S and O accumulated in tensor memory; fp32 online softmax); K and V pages
+ * are staged by tiled TMA through tensor maps of this layer's pools, encoded on the host
+ * for each call; no workspace.
+ * Errors as for paged_decode_attention; PKV_ERR_CUDA also when the driver's tensor-map
+ * encoder cannot be found or rejects the pool; on an int8 pool, UNSUPPORTED.
  */
 int paged_prefill_attention(const pkv_pool* pool, int layer, void* out, const void* q, const int32_t* cu_q,
                             int total_q, const int32_t* block_tables, int max_pages_per_seq,
