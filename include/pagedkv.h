@@ -301,8 +301,9 @@ int paged_decode_attention_noalloc(const pkv_pool* pool, int layer, void* out, c
  *           attends to tokens 0 .. L_b - n_b + i.
  *   block_tables, max_pages_per_seq, kv_heads, scale: as for paged_decode_attention;
  *   q_heads / kv_heads in {1, 2, 4, 8}.
- * One CTA per (sequence, kv head, 128 query rows) on the fifth-generation tensor cores
- * (tcgen05.mma, S and O accumulated in tensor memory; fp32 online softmax); K and V pages
+ * One CTA per (sequence, kv head, two tiles of 128 query rows) on the fifth-generation
+ * tensor cores (tcgen05.mma, S and O accumulated in tensor memory; fp32 online softmax;
+ * softmax, MMA and copy warps meet on mbarriers); K and V pages
  * are staged by tiled TMA through tensor maps of this layer's pools, encoded on the host
  * for each call; no workspace.
  * Errors as for paged_decode_attention; PKV_ERR_CUDA also when the driver's tensor-map

@@ -517,7 +517,7 @@ int launch_prefill(const PrefillParams& prm_in, int grid, cudaStream_t st)
 {
     static int configured[kMaxDevices] = {0};
     using S = TcShape<D, std::is_same<T, __nv_bfloat16>::value>;
-    const int smem = S::kBytes + std::max(S::kTailMin, 4 * (prm_in.batch + 1));
+    const int smem = std::max(S::kBytes + 4 * (prm_in.batch + 1), S::kMinBytes);
     if (smem > kMaxSmemPerCta) return PKV_ERR_UNSUPPORTED;
     PrefillParams prm = prm_in;
     if (!encode_page_map<D, P, T>(&prm.k_map, prm.k, prm.kv_heads, prm.num_pages) ||
@@ -581,10 +581,10 @@ extern "C" int paged_prefill_attention(const pkv_pool* pool, int layer, void* ou
     prm.kv_heads = kv_heads;
     prm.num_pages = pool->num_pages;
     prm.scale_log2 = scale * 1.4426950408889634f;
-    // work items (one CTA each): kv_heads * sum_b ceil(n_b * group / R), R = kTcRows,
-    // at most kv_heads * ((total_q * group + (R - 1) * batch) / R + 1)
-    const long long grid = (long long)kv_heads *
-                           (((long long)total_q * group + (long long)(kTcRows - 1) * batch) / kTcRows + 1);
+    // work items (one CTA each): kv_heads * sum_b ceil(ceil(n_b * group / R) / 2), R = kTcRows
+    // (a CTA takes two row tiles), at most kv_heads * ((total_q * group + (2R - 1) * batch) / 2R + 1)
+    const long long grid = (long long)kv_heads * (((long long)total_q * group + (long long)(2 * kTcRows - 1) * batch) /
+                                                      (2 * kTcRows) + 1);
     if (grid > 0x7fffffffLL) return PKV_ERR_UNSUPPORTED;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (pool->dtype == PKV_F16)
