@@ -7,9 +7,9 @@
 // tcgen05: one elected lane issues the MMAs, operands come from shared memory, the
 // accumulators live in tensor memory (TMEM).
 //
-// Work: one CTA per SM-sized item -- a pair of 128-row tiles of one (sequence, kv head), a
-// row being one (query token, query head of the group) pair -- so each K/V block is staged
-// once for 256 rows.  The warps specialise and meet only on mbarriers:
+// Work: one CTA (one per SM) per pair of 128-row tiles of one (sequence, kv head), a row
+// being one (query token, query head of the group) pair, so each K/V block is staged once
+// for 256 rows.  The warps specialise and meet only on mbarriers:
 //   warps 0-3, 4-7  softmax of tile A, tile B: one thread per row (TMEM lane); per block of
 //                   NK keys (64 for fp16; 32 for bf16, whose P takes two buffers) it reads
 //                   its S row from TMEM, applies the causal mask, runs the fp32 online
