@@ -307,7 +307,10 @@ int paged_decode_attention_noalloc(const pkv_pool* pool, int layer, void* out, c
  * are staged by tiled TMA through tensor maps of this layer's pools, encoded on the host
  * for each call; no workspace.
  * Errors as for paged_decode_attention; PKV_ERR_CUDA also when the driver's tensor-map
- * encoder cannot be found or rejects the pool; on an int8 pool, UNSUPPORTED.
+ * encoder cannot be found or rejects the pool; on an int8 pool, UNSUPPORTED.  A CTA keeps
+ * one int per sequence (batch + 1) in shared memory beside its tiles, so batch is bounded
+ * (about 8900 sequences at head_dim 128 fp16, 13000 bf16, 27000-29000 at head_dim 64):
+ * UNSUPPORTED above.
  */
 int paged_prefill_attention(const pkv_pool* pool, int layer, void* out, const void* q, const int32_t* cu_q,
                             int total_q, const int32_t* block_tables, int max_pages_per_seq,

@@ -225,6 +225,9 @@ def test_prefill_validates(L):
     assert L.paged_prefill_attention(h, 1, f(), f(), f(), 4, f(), 4, f(), 1, 2, 2, 0.1, None) == _lib.PKV_ERR_INVALID_ARG
     assert L.paged_prefill_attention(h, 0, None, f(), f(), 4, f(), 4, f(), 1, 2, 2, 0.1, None) == _lib.PKV_ERR_INVALID_ARG
     assert L.paged_prefill_attention(h, 0, f(), f(), f(), 0, f(), 4, f(), 1, 2, 2, 0.1, None) == 0
+    # the per-sequence work prefix no longer fits beside the tiles in one CTA's shared memory
+    assert L.paged_prefill_attention(h, 0, f(), f(), f(), 30000, f(), 4, f(), 30000, 2, 2, 0.1, None) == \
+        _lib.PKV_ERR_UNSUPPORTED
     L.kv_pool_destroy(h)
 
 
