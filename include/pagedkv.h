@@ -28,7 +28,13 @@
  *     cudaStream_t; NULL = legacy default stream); no entry point synchronises the
  *     host except kv_get_device_error().  Consecutive kernels of the library use
  *     programmatic dependent launch, so a kernel's prologue may overlap the tail of the
- *     library kernel before it on the same stream.
+ *     library kernel before it on the same stream.  The decode calls read cached pages
+ *     in that prologue, all but the page of each sequence's newest token; so the calls
+ *     that write pages (paged_kv_append, rope_append) let the next kernel start only once
+ *     their rows are written, whatever tokens and slots they are given, and
+ *     paged_decode_layer, which lets it start earlier, writes only the newest token of
+ *     each sequence (position context_lens[b] - 1).  A decode call that directly follows
+ *     paged_decode_layer on the same layer must be given the same context_lens.
  *   - Layouts are row-major, innermost index last.  Element type: PKV_F16 (IEEE
  *     binary16) or PKV_BF16 (bfloat16), the same for q, k, v, the pool and the output.
  *   - Device-side index checks: an out-of-range page id or slot is never dereferenced;
@@ -57,6 +63,10 @@ extern "C" {
 #define PKV_F16 0
 #define PKV_BF16 1
 #define PKV_I8 2     /* KV storage only: int8 codes with one fp32 scale per (token, head) row */
+
+/* Largest num_splits that paged_decode_attention and paged_decode_layer accept.  A decode
+ * workspace starts with a counter region of this many int32 slots whatever num_splits is. */
+#define PKV_MAX_DECODE_SPLITS 4096
 
 /* device error word bits (kv_get_device_error) */
 #define PKV_DEVERR_BAD_PAGE 0x1u     /* block-table entry outside [0, num_pages) */
@@ -213,17 +223,19 @@ int rms_norm(void* out, const void* x, void* residual, const void* weight, int r
 
 /*
  * Number of work partitions paged_decode_attention uses when called with num_splits = 0 on
- * the current device (SM count x resident CTAs per SM for this shape).  Needs a CUDA
- * device; PKV_ERR_CUDA without one.
+ * the current device (SM count x resident CTAs per SM for this shape, at most
+ * PKV_MAX_DECODE_SPLITS).  Needs a CUDA device; PKV_ERR_CUDA without one.
  */
 int pkv_decode_default_splits(int q_heads, int kv_heads, int head_dim, int page_size, int dtype,
                               int* num_splits_out);
 
 /*
- * Workspace bytes paged_decode_attention needs for `num_splits` (>= 1) partitions: per
+ * Workspace bytes paged_decode_attention needs for `num_splits` (1 .. PKV_MAX_DECODE_SPLITS)
+ * partitions: a fixed region of PKV_MAX_DECODE_SPLITS int32 counters (16 KiB), then per
  * partition two fp32 partial results (running max, sum and the unnormalised output of every
- * query head of a kv-head group) and one int32 counter.  `batch` is accepted for
- * compatibility and does not change the size.  0 on bad input.
+ * query head of a kv-head group).  The counters do not move with num_splits, so one
+ * workspace serves calls with any split count up to the one it was sized for.  `batch` is
+ * accepted for compatibility and does not change the size.  0 on bad input.
  */
 size_t pkv_decode_workspace_size(int batch, int q_heads, int kv_heads, int head_dim,
                                  int num_splits);
@@ -243,16 +255,19 @@ size_t pkv_decode_workspace_size(int batch, int q_heads, int kv_heads, int head_
  *   context_lens: device [batch] int32, the new token included.
  *   kv_heads must equal the pool's; q_heads a multiple of it with q_heads / kv_heads in
  *   {1, 2, 4, 8}.
- *   num_splits: number of work partitions (0 = pkv_decode_default_splits).  The batch's
+ *   num_splits: number of work partitions, at most PKV_MAX_DECODE_SPLITS
+ *           (0 = pkv_decode_default_splits).  The batch's
  *           pages x kv heads are laid end to end and cut into num_splits equal ranges, one
  *           per CTA; a (sequence, kv head) cut by a range boundary is finished by the CTA
  *           that delivers its last partial, which rescales the partial softmax sums
  *           (log-sum-exp).  One kernel launch per call.
  *   workspace: device scratch of >= pkv_decode_workspace_size(batch, q_heads, kv_heads,
  *           head_dim, num_splits) bytes, 256-byte aligned, zero-filled before its first use
- *           (pkv_decode_workspace_clear or any memset); every call leaves it ready for the
- *           next one.  Calls that share a workspace must be ordered on one stream.
- * Errors: INVALID_ARG (bad pointer/shape/layer), UNSUPPORTED (group/head_dim/page/dtype
+ *           (pkv_decode_workspace_clear or any memset); every call leaves its counter region
+ *           at zero, so the next call may use any split count the workspace is large enough
+ *           for.  Calls that share a workspace must be ordered on one stream.
+ * Errors: INVALID_ARG (bad pointer/shape/layer, num_splits above PKV_MAX_DECODE_SPLITS),
+ * UNSUPPORTED (group/head_dim/page/dtype
  * combination), NO_SPACE (workspace too small), CUDA (launch failure).
  */
 int paged_decode_attention(const pkv_pool* pool, int layer, void* out, const void* q,
@@ -270,16 +285,18 @@ int paged_decode_attention(const pkv_pool* pool, int layer, void* out, const voi
  * Arguments, results and errors are those of paged_decode_attention, without the
  * workspace: the scratch is a fixed 4 MiB array inside the library, in device memory
  * that every GPU which loads the library holds until the process exits.
- *   - A call whose scratch would exceed 4 MiB (2 x num_splits x (q_heads / kv_heads) x
- *     (head_dim + 2) fp32 values plus num_splits counters) is rejected with
- *     PKV_ERR_NO_SPACE and launches nothing.  On B200 the automatic split count
- *     (num_splits = 0) fits for every shape the kernels accept.
+ *   - A call whose scratch would exceed 4 MiB (the 16 KiB counter region plus
+ *     2 x num_splits x (q_heads / kv_heads) x (head_dim + 2) fp32 values, each part rounded
+ *     up to 256 bytes) is rejected with PKV_ERR_NO_SPACE and launches nothing; the pool,
+ *     layer and shape are checked first, as in paged_decode_attention.  On B200 the
+ *     automatic split count (num_splits = 0) fits for every shape the kernels accept.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call before any
  *     stream capture begins.
  *   - All calls on a device share the one array, which keeps the previous call's
- *     contents; nothing in it needs clearing (its counters are zero when the library is
- *     loaded and every call leaves them at zero).  Calls that overlap on the GPU
+ *     contents; nothing in it needs clearing (its counter region is zero when the library
+ *     is loaded, every call leaves it at zero, and no call's partial results overlap it,
+ *     whatever the split counts of consecutive calls).  Calls that overlap on the GPU
  *     (different streams, or several host threads) race on it: order them on one stream.
  *   - No cudaMalloc, cudaFree or allocating library routine is called.
  */

@@ -20,14 +20,14 @@ import numpy as np
 
 from . import _lib
 from ._lib import (PKV_BF16, PKV_DEVERR_BAD_PAGE, PKV_DEVERR_BAD_SLOT, PKV_DEVERR_TIMEOUT, PKV_F16, PKV_I8,
-                   PagedKVError, lib)
+                   PKV_MAX_DECODE_SPLITS, PagedKVError, lib)
 
 __all__ = [
     "KVPool", "rope_apply", "paged_kv_append", "rope_append", "paged_decode_attention", "rope_table",
     "paged_decode_layer", "paged_prefill_attention", "rms_norm", "pkv_slot_mapping",
     "pkv_kv_cache_bytes", "pkv_decode_workspace_size", "pkv_decode_default_splits",
     "kv_get_device_error", "DecodeWorkspace", "PagedKVError", "PKV_F16", "PKV_BF16", "PKV_I8",
-    "PKV_DEVERR_BAD_PAGE", "PKV_DEVERR_BAD_SLOT", "PKV_DEVERR_TIMEOUT",
+    "PKV_DEVERR_BAD_PAGE", "PKV_DEVERR_BAD_SLOT", "PKV_DEVERR_TIMEOUT", "PKV_MAX_DECODE_SPLITS",
 ]
 
 
@@ -249,7 +249,8 @@ def rms_norm(out, x, weight, eps=1e-6, residual=None, stream=None):
 class DecodeWorkspace:
     """Device scratch for paged_decode_attention, sized for a batch and a split count.
     Allocated zero-filled, as the kernel's per-partition counters require; every call
-    leaves it ready for the next one."""
+    leaves them at zero, and they sit in a fixed region that no call's partial results
+    overlap, so the workspace serves any split count up to the one it was sized for."""
 
     def __init__(self, batch, q_heads, kv_heads, head_dim, page_size, dtype, num_splits=0, device=None,
                  storage=None):

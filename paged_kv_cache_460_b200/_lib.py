@@ -20,6 +20,7 @@ PKV_I8 = 2
 PKV_DEVERR_BAD_PAGE = 0x1
 PKV_DEVERR_BAD_SLOT = 0x2
 PKV_DEVERR_TIMEOUT = 0x4
+PKV_MAX_DECODE_SPLITS = 4096
 
 _lib = None
 

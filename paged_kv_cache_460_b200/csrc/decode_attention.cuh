@@ -277,11 +277,12 @@ __global__ void __launch_bounds__(kDecodeThreads, G == 1 ? 4 : 1) decode_pass1_k
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     // Prologue, before waiting on the previous kernel of the stream: the caller's lengths
-    // and page table, and the first cached pages (see below).  Library kernels only let
-    // their successor start once their own predecessor has finished (RoPE/append, which
-    // writes just the newest token of each sequence, is the one that lets it start
-    // earlier), so none of these is still being written; q, the newest tokens, the
-    // outputs and the workspace are touched only after pdl_wait.
+    // and page table, and the first cached pages (see below).  A library kernel that
+    // appends rows lets its successor start only once they are written and fenced, and
+    // every other library kernel only after its own predecessor has finished; the one
+    // exception, the fused layer, writes nothing but each sequence's newest token, whose
+    // page is not prefetched here.  So none of these is still being written; q, the
+    // newest tokens, the outputs and the workspace are touched only after pdl_wait.
     block_page_prefix<P>(p.context_lens, p.batch, prefix, lens, warp_tot);
     __syncthreads();
     const int Hkv = p.kv_heads;
@@ -361,8 +362,8 @@ __global__ void __launch_bounds__(kDecodeThreads, G == 1 ? 4 : 1) decode_pass1_k
         advance();
     };
     // Before waiting on the previous kernel: prefetch this warp's first pages, except a
-    // page holding a sequence's newest token (the append before this kernel may still be
-    // writing it) and the q rows (the kernel before may still be producing them).
+    // page holding a sequence's newest token (a fused layer before this kernel may still
+    // be writing it) and the q rows (the kernel before may still be producing them).
     int m_pre = 0, pre_qb[DEPTH], pre_qg[DEPTH];
     for (; m_pre < DEPTH && m_pre < n_mine; ++m_pre) {
         if (!kFused && ij == inp - 1) break;

@@ -112,7 +112,8 @@ struct DecodeImpl {
         if (ensure_smem(K::fn, smem, configured) != cudaSuccess) return PKV_ERR_CUDA;
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, K::fn, kDecodeThreads, smem) != cudaSuccess)
             return PKV_ERR_CUDA;
-        *out = sms * (per_sm > 3 ? 3 : (per_sm > 0 ? per_sm : 1));
+        const int n = sms * (per_sm > 3 ? 3 : (per_sm > 0 ? per_sm : 1));
+        *out = n < PKV_MAX_DECODE_SPLITS ? n : PKV_MAX_DECODE_SPLITS;
         return PKV_OK;
     }
 };
@@ -162,12 +163,15 @@ struct WorkspaceLayout {
     size_t counters, part_o, part_ml, total;
 };
 
+// The per-partition counters sit in a region of fixed size at the start of the
+// workspace, whatever num_splits is: a call with more partitions than the previous call
+// on the same scratch must find zeros there, never the previous call's partial results.
 WorkspaceLayout workspace_layout(int batch, int group, int head_dim, int num_splits)
 {
     (void)batch;
     WorkspaceLayout w;
     w.counters = 0;
-    w.part_o = align256(sizeof(int) * (size_t)num_splits);
+    w.part_o = align256(sizeof(int) * (size_t)PKV_MAX_DECODE_SPLITS);
     w.part_ml = w.part_o + align256(sizeof(float) * 2 * (size_t)num_splits * group * head_dim);
     w.total = w.part_ml + align256(sizeof(float) * 2 * (size_t)num_splits * group * 2);
     return w;
@@ -241,7 +245,7 @@ extern "C" int rope_apply(void* q, void* k, const int32_t* positions, int n_toke
     prm.kv_heads = kv_heads;
     prm.head_dim = head_dim;
     prm.theta = theta;
-    prm.mode = kRopeRotate;
+    prm.mode = kRopeRotate | kRopeEarlyRelease;     // writes no pool page
     return launch_rope_append(prm, n_tokens, dtype, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -315,7 +319,8 @@ extern "C" int pkv_decode_default_splits(int q_heads, int kv_heads, int head_dim
 
 extern "C" size_t pkv_decode_workspace_size(int batch, int q_heads, int kv_heads, int head_dim, int num_splits)
 {
-    if (batch < 0 || q_heads <= 0 || kv_heads <= 0 || q_heads % kv_heads || head_dim <= 0 || num_splits <= 0)
+    if (batch < 0 || q_heads <= 0 || kv_heads <= 0 || q_heads % kv_heads || head_dim <= 0 || num_splits <= 0 ||
+        num_splits > PKV_MAX_DECODE_SPLITS)
         return 0;
     return workspace_layout(batch, q_heads / kv_heads, head_dim, num_splits).total;
 }
@@ -327,7 +332,8 @@ extern "C" int paged_decode_attention(const pkv_pool* pool, int layer, void* out
 {
     if (!pool || layer < 0 || layer >= pool->num_layers) return PKV_ERR_INVALID_ARG;
     if (batch < 0 || q_heads <= 0 || kv_heads != pool->kv_heads || q_heads % kv_heads) return PKV_ERR_INVALID_ARG;
-    if (num_splits < 0 || max_pages_per_seq <= 0 || !(scale == scale)) return PKV_ERR_INVALID_ARG;
+    if (num_splits < 0 || num_splits > PKV_MAX_DECODE_SPLITS || max_pages_per_seq <= 0 || !(scale == scale))
+        return PKV_ERR_INVALID_ARG;
     if (batch == 0) return PKV_OK;
     if (!out || !q || !block_tables || !context_lens || !workspace) return PKV_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(out) | reinterpret_cast<uintptr_t>(q)) & 15u) return PKV_ERR_INVALID_ARG;
@@ -429,7 +435,8 @@ extern "C" int paged_decode_layer(const pkv_pool* pool, int layer, void* out, co
 {
     if (!pool || layer < 0 || layer >= pool->num_layers) return PKV_ERR_INVALID_ARG;
     if (batch < 0 || q_heads <= 0 || kv_heads != pool->kv_heads || q_heads % kv_heads) return PKV_ERR_INVALID_ARG;
-    if (num_splits < 0 || max_pages_per_seq <= 0 || !(scale == scale)) return PKV_ERR_INVALID_ARG;
+    if (num_splits < 0 || num_splits > PKV_MAX_DECODE_SPLITS || max_pages_per_seq <= 0 || !(scale == scale))
+        return PKV_ERR_INVALID_ARG;
     const bool i8 = pool->storage == kStorageI8;
     const int group = q_heads / kv_heads;
     if (!i8 && group != 1) return PKV_ERR_UNSUPPORTED;
@@ -655,16 +662,19 @@ extern "C" int paged_decode_attention_noalloc(const pkv_pool* pool, int layer, v
                                               const int32_t* context_lens, int batch, int q_heads, int kv_heads,
                                               float scale, int num_splits, pkv_stream_t stream)
 {
-    if (!pool || batch < 0 || q_heads <= 0 || kv_heads <= 0 || q_heads % kv_heads || num_splits < 0)
-        return PKV_ERR_INVALID_ARG;
+    // the same argument checks as paged_decode_attention, before the size check
+    if (!pool || layer < 0 || layer >= pool->num_layers) return PKV_ERR_INVALID_ARG;
+    if (batch < 0 || q_heads <= 0 || kv_heads != pool->kv_heads || q_heads % kv_heads) return PKV_ERR_INVALID_ARG;
+    if (num_splits < 0 || num_splits > PKV_MAX_DECODE_SPLITS) return PKV_ERR_INVALID_ARG;
     if (num_splits > 0 && workspace_layout(batch, q_heads / kv_heads, pool->head_dim, num_splits).total >
                               kStaticScratchBytes)
         return PKV_ERR_NO_SPACE;
     void* scratch = nullptr;
     const int st = static_scratch_address(&scratch);
     if (st != PKV_OK) return st;
-    // The scratch's only state that outlives a call is its counters, which are zero when
-    // the library is loaded and which every call leaves at zero.
+    // The scratch's only state that outlives a call is its counter region, which is zero
+    // when the library is loaded, which every call leaves at zero, and which no call's
+    // partial results overlap, whatever its split count.
     return paged_decode_attention(pool, layer, out, q, block_tables, max_pages_per_seq, context_lens, batch,
                                   q_heads, kv_heads, scale, num_splits, scratch, kStaticScratchBytes, stream);
 }

@@ -14,6 +14,10 @@ namespace pkv {
 constexpr int kRopeRotate = 1;   // turn q and k in place
 constexpr int kRopeAppend = 2;   // write k and v into their pool slots
 constexpr int kRopeQuantI8 = 4;  // ... as int8 codes plus a per-row fp32 scale
+// Let the next kernel of the stream start before this one waits on its predecessor.  Only
+// for launches that write no pool page: the decode kernels read cached pages before their
+// own wait, so a launch that appends releases them only once its rows are written.
+constexpr int kRopeEarlyRelease = 8;
 
 struct RopeAppendParams {
     void* q;                 // [n][q_heads][d]   (rotated in place)
@@ -76,9 +80,12 @@ __global__ void __launch_bounds__(64) rope_table_kernel(const int32_t* __restric
 // Grid: (token, part).  Each thread handles one 16-byte vector (8 elements, 4 pairs)
 // of the token's q, k or v rows.  The head_dim/2 angles pos * theta^(-2i/d) and their
 // cosines and sines are evaluated once per CTA in fp64 before griddepcontrol.wait, so
-// this prologue overlaps the previous kernel on the stream (and the attention kernel
-// after it may start its prefetch during this one); each pair is then turned in
+// this prologue overlaps the previous kernel on the stream; each pair is then turned in
 // fp64 (explicit _rn products: no fused rounding) and rounded once to the storage type.
+// A rotate-only launch lets the kernel after it start at once; a launch that appends lets
+// it start only after every CTA has written its rows and fenced them at gpu scope, since
+// the decode kernels prefetch cached pages (which an append of several tokens per
+// sequence, or of any slots, may be writing) before their own wait.
 // Appending copies the rotated k and the v vector bit for bit into row slot % P of page
 // slot / P; a negative slot skips the token, a slot past the pool is skipped and flagged.
 // On an int8 pool the head row is quantised instead ([ENGINE] s3.4 compression):
@@ -102,9 +109,7 @@ __global__ void __launch_bounds__(256) rope_append_kernel(const RopeAppendParams
         }
     }
     __syncthreads();
-    // Let the attention kernel that follows start now: before its own wait it reads only
-    // pages that this kernel does not write (it skips those holding a newest token).
-    pdl_launch_dependents();
+    if (p.mode & kRopeEarlyRelease) pdl_launch_dependents();
     pdl_wait();
     int64_t slot = -1;
     if (p.mode & kRopeAppend) {
@@ -176,6 +181,11 @@ __global__ void __launch_bounds__(256) rope_append_kernel(const RopeAppendParams
                 *dst = u;
             }
         }
+    }
+    if (!(p.mode & kRopeEarlyRelease)) {
+        __threadfence();            // this thread's pool and q/k writes, visible at gpu scope,
+        __syncthreads();            // for every thread of the CTA, before the CTA releases
+        pdl_launch_dependents();    // the next kernel
     }
 }
 

@@ -196,6 +196,52 @@ def test_workspace_size_and_host_validation(L):
     L.kv_pool_destroy(h)
 
 
+def test_header_constants_match_the_binding():
+    text = open(HEADER).read()
+    for name in ("PKV_MAX_DECODE_SPLITS", "PKV_ERR_NO_SPACE", "PKV_DEVERR_TIMEOUT", "PKV_I8"):
+        m = re.search(r"#define\s+%s\s+(0x[0-9a-fA-F]+|\d+)" % name, text)
+        assert m, name
+        assert int(m.group(1), 0) == getattr(_lib, name), name
+
+
+def test_workspace_counter_region_is_fixed(L):
+    """The counters occupy the same 16 KiB at the start of every workspace, whatever the split
+    count: only the partials after them grow with num_splits."""
+    cap = _lib.PKV_MAX_DECODE_SPLITS
+    sizes = {n: L.pkv_decode_workspace_size(4, 8, 8, 64, n) for n in (1, 7, 444, 1000, cap)}
+    assert sizes[1] >= 4 * cap + 2 * 1 * 64 * 4
+    for n, ws in sizes.items():
+        parts = 2 * n * 64 * 4 + 2 * n * 2 * 4             # o and (m, l) of both slots of every CTA
+        assert ws >= 4 * cap + parts and ws % 256 == 0, n
+        assert ws <= 4 * cap + parts + 3 * 256, n
+    assert L.pkv_decode_workspace_size(4, 8, 8, 64, cap + 1) == 0
+    h = _pool(L, num_pages=8, page_size=16, kv_heads=2, head_dim=64)
+    f = _fake_ptr
+    assert L.paged_decode_attention(h, 0, f(), f(), f(), 4, f(), 1, 2, 2, 0.1, cap + 1, f(0x100000), 1 << 30,
+                                    None) == _lib.PKV_ERR_INVALID_ARG
+    assert L.paged_decode_layer(h, 0, f(), f(), f(), f(), f(), f(), 4, f(), 1, 2, 2, 0.1, cap + 1, f(0x100000),
+                                1 << 30, None) == _lib.PKV_ERR_INVALID_ARG
+    L.kv_pool_destroy(h)
+
+
+def test_noalloc_checks_arguments_before_its_scratch_limit(L):
+    """The no-alloc entry point refuses a bad layer or kv-head count as paged_decode_attention
+    does (INVALID_ARG), even with a split count whose scratch would not fit; with valid
+    arguments that split count gets NO_SPACE.  No device work is launched."""
+    h = _pool(L, num_pages=8, page_size=16, kv_heads=8, head_dim=128)
+    f = _fake_ptr
+    too_many = 4000           # 16 KiB + 2 x 4000 x 8 x 130 fp32 values: far above 4 MiB at group 8
+    assert L.paged_decode_attention_noalloc(h, 1, f(), f(), f(), 4, f(), 1, 64, 8, 0.1, too_many, None) \
+        == _lib.PKV_ERR_INVALID_ARG                                      # layer out of range
+    assert L.paged_decode_attention_noalloc(h, 0, f(), f(), f(), 4, f(), 1, 64, 4, 0.1, too_many, None) \
+        == _lib.PKV_ERR_INVALID_ARG                                      # kv_heads != pool's
+    assert L.paged_decode_attention_noalloc(h, 0, f(), f(), f(), 4, f(), 1, 64, 8, 0.1,
+                                            _lib.PKV_MAX_DECODE_SPLITS + 1, None) == _lib.PKV_ERR_INVALID_ARG
+    assert L.paged_decode_attention_noalloc(h, 0, f(), f(), f(), 4, f(), 1, 64, 8, 0.1, too_many, None) \
+        == _lib.PKV_ERR_NO_SPACE
+    L.kv_pool_destroy(h)
+
+
 def test_rope_append_validates(L):
     h = _pool(L, num_pages=8, page_size=16, kv_heads=2, head_dim=64)
     f = _fake_ptr

@@ -180,7 +180,8 @@ def _sample_pairs(s, n, seed):
     return sorted(pairs)
 
 
-@pytest.mark.parametrize("name,layers,check_layers", [("batch10", 32, (0, 31)), ("cbatch", 1, (0,))])
+@pytest.mark.parametrize("name,layers,check_layers",
+                         [("batch10", 32, (0, 31)), ("cbatch", 1, (0,)), ("longctx", 1, (0,))])
 def test_int8_full_size_workload_sampled(name, layers, check_layers):
     """The benchmark's int8 configuration at full size; sampled (sequence, kv head) pairs
     are recomputed by the oracle from page snapshots taken before any kernel runs."""
