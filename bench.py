@@ -196,41 +196,82 @@ def max_over_ranks(value, world, device=None):
 
 
 # ------------------------------------------------------------------ CPU oracle timing
-def time_oracle_sample(s, seconds, seed=0, max_pairs=None, kv="native"):
-    """Time the fp64 oracle (single thread) on (b, kv head) pairs of the workload, each
-    pair a standalone mini pool, until ~`seconds` have passed.  Returns
-    (GB/s of algorithmic KV bytes, description)."""
+def host_cpu():
+    """(usable host cores, CPU model name)."""
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except AttributeError:
+        cores = os.cpu_count() or 1
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return cores, model
+
+
+def time_oracle_sample(s, seconds, seed=0, kv="native", all_cores=True):
+    """Time the fp64 oracle on batches of random (sequence, kv head) pairs of the workload
+    (each pair a standalone sequence with the group's query heads; inputs drawn outside the
+    timed calls) until about `seconds` of single-thread time.  Each batch runs twice: the
+    plain build on one thread, then the OpenMP build with its pairs spread over every host
+    core.  Returns a dict with both legs' GB/s of algorithmic KV bytes."""
     import oracle
     r = np.random.Generator(np.random.PCG64(seed))
     G = s.q_heads // s.kv_heads
     live = np.nonzero(s.context_lens > 0)[0]
     scale = 1.0 / math.sqrt(s.head_dim)
-    total_bytes, total_t, n = 0, 0.0, 0
-    while total_t < seconds and (max_pairs is None or n < max_pairs):
-        b = int(r.choice(live))
-        g = int(r.integers(0, s.kv_heads))
-        kmini, vmini = synth.mini_pool_numpy(s, b, g, seed=int(r.integers(1 << 30)))
-        q = synth.round_f32(r.standard_normal((1, G, s.head_dim), dtype=np.float32), s.dtype)
-        table = np.arange(kmini.shape[0], dtype=np.int32)[None, :]
-        cl = np.array([s.context_lens[b]], np.int32)
-        pairs = [(0, h) for h in range(G)]
+    cores, model = host_cpu()
+    threads = oracle.set_threads(cores) if all_cores else 1
+    row_bytes = 2 * (s.head_dim + 4) if kv == "int8" else 2 * s.head_dim * s.elt_bytes
+    mean_len = float(s.context_lens[live].mean())
+    # pairs per batch: about a second of single-thread work (the oracle reads ~0.1 GB/s),
+    # less for a short budget; at least two per thread, at most 1 GB of pages
+    target = min(0.15e9, max(2e6, 0.1e9 * seconds))
+    want = max(2 * threads, int(target / (mean_len * row_bytes)))
+    n_pairs = max(1, min(want, int(1e9 / (float(s.context_lens.max()) * row_bytes))))
+    t1 = tn = 0.0
+    nbytes = 0
+    batches = 0
+    while t1 < seconds:
+        pairs = [(int(r.choice(live)), int(r.integers(0, s.kv_heads))) for _ in range(n_pairs)]
+        m = synth.pair_batch_numpy(s, pairs, int(r.integers(1 << 30)), kv)
+        hp = [(i, h) for i in range(n_pairs) for h in range(G)]
         if kv == "int8":
-            codes = r.integers(-127, 128, size=(2,) + kmini.shape, dtype=np.int8)
-            sc = (r.uniform(1.5, 2.5, size=(2,) + kmini.shape[:-1]) / 127.0).astype(np.float32)
-            t0 = time.perf_counter()
-            oracle.decode_attention_i8_pairs(q, codes[0], codes[1], sc[0], sc[1], table, cl, scale, s.dtype, pairs)
-            total_t += time.perf_counter() - t0
-            total_bytes += int(cl[0]) * 2 * (s.head_dim + 4)
-            n += 1
-            continue
+            args = (m["q"], m["k_codes"], m["v_codes"], m["k_scales"], m["v_scales"], m["block_tables"],
+                    m["context_lens"], scale, s.dtype, hp)
+            fn = oracle.decode_attention_i8_pairs
+        else:
+            args = (m["q"], m["k"], m["v"], m["block_tables"], m["context_lens"], scale, s.dtype, hp)
+            fn = oracle.decode_attention_pairs
         t0 = time.perf_counter()
-        oracle.decode_attention_pairs(q, kmini, vmini, table, cl, scale, s.dtype, pairs)
-        total_t += time.perf_counter() - t0
-        total_bytes += int(cl[0]) * 2 * s.head_dim * s.elt_bytes
-        n += 1
-    gbs = total_bytes / total_t / 1e9
-    return gbs, "%d random (sequence, kv head) pairs of one %s layer (%d query heads each%s), %.1f s" % (
-        n, s.name, G, ", int8 pages" if kv == "int8" else "", total_t)
+        fn(*args)
+        t1 += time.perf_counter() - t0
+        if all_cores:
+            t0 = time.perf_counter()
+            fn(*args, omp=True)
+            tn += time.perf_counter() - t0
+        nbytes += int(m["context_lens"].astype(np.int64).sum()) * row_bytes
+        batches += 1
+    desc = "%d batches of %d random (sequence, kv head) pairs of one %s layer (%d query heads each%s); " \
+           "one thread: %.1f s" % (batches, n_pairs, s.name, G, ", int8 pages" if kv == "int8" else "", t1)
+    res = {"single": nbytes / t1 / 1e9, "cores_available": cores, "cpu_model": model, "sample": desc}
+    if all_cores:
+        res["all"] = nbytes / tn / 1e9
+        res["threads"] = threads
+        res["sample"] += "; %d threads: %.1f s" % (threads, tn)
+    return res
+
+
+def cpu_baseline_entry(res, unit):
+    """The bench line's cpu_baseline: the all-core leg, the single-thread leg beside it."""
+    return {"value": res.get("all", res["single"]), "unit": unit, "cores": res.get("threads", 1), "kind": "oracle",
+            "sample": res["sample"], "cpu_model": res["cpu_model"], "cores_available": res["cores_available"],
+            "single_thread": {"value": res["single"], "unit": unit, "cores": 1}}
 
 
 def run_reference(args):
@@ -238,25 +279,25 @@ def run_reference(args):
     if rank != 0:
         return 0
     s = synth.spec(args.workload, num_layers=args.layers)
-    per_step = max(0.02, min(2.0, 150.0 / max(1, args.steps + args.warmup)))
+    per_step = max(0.05, min(2.0, 150.0 / max(1, args.steps + args.warmup)))
     for i in range(args.warmup):
-        time_oracle_sample(s, per_step, seed=i, kv=args.kv)
-    vals, t_all = [], 0.0
-    import oracle  # noqa: F401
+        time_oracle_sample(s, per_step, seed=i, kv=args.kv, all_cores=False)
+    vals, t_all, last = [], 0.0, None
     for i in range(args.steps):
         t0 = time.perf_counter()
-        g, _ = time_oracle_sample(s, per_step, seed=1000 + i, kv=args.kv)
+        last = time_oracle_sample(s, per_step, seed=1000 + i, kv=args.kv)
         t_all += time.perf_counter() - t0
-        vals.append(g)
+        vals.append(last["all"])
     value = float(np.mean(vals))
+    cpu = cpu_baseline_entry(last, UNIT)
+    cpu["value"] = value
+    cpu["sample"] = "each step: " + cpu["sample"]
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * t_all / max(1, args.steps),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(s, args),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": "each step: ~%.2f s of single-thread fp64 oracle on random (sequence, kv head) "
-                                   "pairs of the workload" % per_step},
+        "cpu_baseline": cpu,
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -311,7 +352,7 @@ def run_ours(args):
     for j in range(INPUT_SETS):
         st = DecodeStep(pool, s.batch, s.q_heads, s.max_pages, theta=s.theta, num_splits=args.splits, device=dev,
                         fused=fused)
-        st.set_metadata(s.block_tables, s.context_lens, s.positions, non_blocking=False)
+        st.set_metadata(s.block_tables, s.context_lens, non_blocking=False)
         st.q.copy_(qs[j])
         st.k.copy_(ks[j])
         st.v.copy_(vs[j])
@@ -397,17 +438,16 @@ def run_ours(args):
         hout = torch.empty(st.out.shape, dtype=tdt).pin_memory()
         hbt = torch.from_numpy(s.block_tables).pin_memory()
         hcl = torch.from_numpy(s.context_lens).pin_memory()
-        hpos = torch.from_numpy(s.positions).pin_memory()
-        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hbt, hcl, hpos)) + 8 * s.batch
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hbt, hcl))
         d2h = hout.numel() * hout.element_size()
         for _ in range(max(1, args.warmup)):
-            st.set_metadata(hbt, hcl, hpos)
+            st.set_metadata(hbt, hcl)
             st.run(hq, hk, hv, hout)
         sync_all()
         n_e2e = max(1, args.steps // 2)
 
         def e2e_step(i):
-            st.set_metadata(hbt, hcl, hpos)
+            st.set_metadata(hbt, hcl)
             st.run(hq, hk, hv, hout)
 
         saved, args.steps = args.steps, n_e2e
@@ -427,8 +467,7 @@ def run_ours(args):
         achieved = layer_bytes / (attn_ms_mean * 1e-3) / 1e9
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
-            gbs, desc = time_oracle_sample(s, args.cpu_seconds, kv=args.kv)
-            cpu = {"value": gbs, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc}
+            cpu = cpu_baseline_entry(time_oracle_sample(s, args.cpu_seconds, kv=args.kv), UNIT)
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": per_step_ms, "higher_is_better": True, "scaling": "weak",

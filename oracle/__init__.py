@@ -25,13 +25,13 @@ from . import build as _build
 
 _DT = {"f16": 0, "bf16": 1}
 
-_lib = None
+_libs = {}
 
 
-def _load():
-    global _lib
-    if _lib is None:
-        path = _build.build()
+def _load(omp=False):
+    """The plain build, or (omp=True) the OpenMP build whose pair routines use every core."""
+    if omp not in _libs:
+        path = _build.build(omp=omp)
         lib = ctypes.CDLL(path)
         P = ctypes.c_void_p
         I = ctypes.c_int
@@ -61,8 +61,15 @@ def _load():
         lib.ora_decode_attention_i8_pairs.argtypes = [P, P, P, P, P, P, I, P, I, I, I, I, D, I, P, P, I, P]
         lib.ora_kv_cache_bytes.argtypes = [I, I, I, I64, I]
         lib.ora_kv_cache_bytes.restype = I64
-        _lib = lib
-    return _lib
+        lib.ora_set_threads.argtypes = [I]
+        lib.ora_set_threads.restype = I
+        _libs[omp] = lib
+    return _libs[omp]
+
+
+def set_threads(n):
+    """Threads of the OpenMP build's pair routines (n >= 1); returns the count in force."""
+    return int(_load(omp=True).ora_set_threads(int(n)))
 
 
 def _p(a):
@@ -160,8 +167,9 @@ def decode_attention(q, k_pool, v_pool, block_tables, context_lens, scale, dtype
     return out
 
 
-def decode_attention_pairs(q, k_pool, v_pool, block_tables, context_lens, scale, dtype, pairs):
-    """Same arithmetic for selected (b, h) pairs only; returns float64 [n_pairs, d]."""
+def decode_attention_pairs(q, k_pool, v_pool, block_tables, context_lens, scale, dtype, pairs, omp=False):
+    """Same arithmetic for selected (b, h) pairs only; returns float64 [n_pairs, d].
+    omp=True runs the pairs on all cores (OpenMP build; each pair's arithmetic unchanged)."""
     q = _c(q, np.uint16)
     kp = _c(k_pool, np.uint16)
     vp = _c(v_pool, np.uint16)
@@ -173,7 +181,7 @@ def decode_attention_pairs(q, k_pool, v_pool, block_tables, context_lens, scale,
     pb = _c(pairs[:, 0], np.int32)
     ph = _c(pairs[:, 1], np.int32)
     out = np.empty((pairs.shape[0], d), np.float64)
-    _load().ora_decode_attention_pairs(_p(q), _p(kp), _p(vp), _p(bt), bt.shape[1], _p(cl), Hq, Hkv,
+    _load(omp).ora_decode_attention_pairs(_p(q), _p(kp), _p(vp), _p(bt), bt.shape[1], _p(cl), Hq, Hkv,
                                        d, P, float(scale), _DT[dtype], _p(pb), _p(ph),
                                        pairs.shape[0], _p(out))
     return out
@@ -261,7 +269,9 @@ def kv_append_i8(k_codes, v_codes, k_scales, v_scales, k, v, block_tables, posit
 
 
 def decode_attention_i8_pairs(q, k_codes, v_codes, k_scales, v_scales, block_tables, context_lens, scale, dtype,
-                              pairs):
+                              pairs, omp=False):
+    """Decode attention of selected (b, h) pairs over an int8 pool (k = code * scale exactly
+    in fp64); omp=True runs the pairs on all cores.  Returns float64 [n_pairs, d]."""
     q = _c(q, np.uint16)
     kc = _c(k_codes, np.int8)
     vc = _c(v_codes, np.int8)
@@ -275,7 +285,7 @@ def decode_attention_i8_pairs(q, k_codes, v_codes, k_scales, v_scales, block_tab
     pb = _c(pairs[:, 0], np.int32)
     ph = _c(pairs[:, 1], np.int32)
     out = np.empty((pairs.shape[0], d), np.float64)
-    _load().ora_decode_attention_i8_pairs(_p(q), _p(kc), _p(vc), _p(ks), _p(vs), _p(bt), bt.shape[1], _p(cl), Hq,
+    _load(omp).ora_decode_attention_i8_pairs(_p(q), _p(kc), _p(vc), _p(ks), _p(vs), _p(bt), bt.shape[1], _p(cl), Hq,
                                           Hkv, d, P, float(scale), _DT[dtype], _p(pb), _p(ph), pairs.shape[0],
                                           _p(out))
     return out

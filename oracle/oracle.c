@@ -337,6 +337,10 @@ void ora_decode_attention_pairs(const uint16_t* q, const uint16_t* k_pool, const
                                 double* out)
 {
     int group = q_heads / kv_heads;
+    /* Each pair is an independent output: the OpenMP build (liboracle_omp.so) hands pairs
+     * to threads; the plain build ignores the pragma.  The arithmetic of a pair is the
+     * same in both. */
+#pragma omp parallel for schedule(dynamic, 1)
     for (int p = 0; p < n_pairs; ++p) {
         int b = pair_b[p], h = pair_h[p], g = h / group;
         int len = context_lens[b];
@@ -597,6 +601,7 @@ void ora_decode_attention_i8_pairs(const uint16_t* q, const int8_t* k_codes, con
                                    const int32_t* pair_h, int n_pairs, double* out)
 {
     int group = q_heads / kv_heads;
+#pragma omp parallel for schedule(dynamic, 1)
     for (int p = 0; p < n_pairs; ++p) {
         int b = pair_b[p], h = pair_h[p], g = h / group;
         int len = context_lens[b];
@@ -630,3 +635,22 @@ void ora_decode_attention_i8_pairs(const uint16_t* q, const int8_t* k_codes, con
         free(s);
     }
 }
+
+/*
+ * Thread count of the pair routines: the OpenMP build uses n threads (n >= 1) and reports
+ * how many it will use; the plain build always reports 1.
+ */
+#ifdef _OPENMP
+#include <omp.h>
+int ora_set_threads(int n)
+{
+    if (n >= 1) omp_set_num_threads(n);
+    return omp_get_max_threads();
+}
+#else
+int ora_set_threads(int n)
+{
+    (void)n;
+    return 1;
+}
+#endif

@@ -297,6 +297,38 @@ def mini_pool_numpy(s, b, g, seed):
     return k, v
 
 
+def pair_batch_numpy(s, pairs, seed, kv="native"):
+    """A standalone batch of (sequence, kv head) pairs of workload `s` for host-only runs:
+    pair i becomes sequence i with one kv head and the group's q heads, its own pages
+    (identity-ordered, numpy PCG64) and the workload's length of its sequence.
+    Returns dict(q [n, G, d] storage bits, block_tables [n, max_pages], context_lens [n],
+    k, v [pages, 1, P, d] storage bits -- or, kv="int8", k_codes, v_codes int8 and k_scales,
+    v_scales fp32 [pages, 1, P] drawn as pool_values_i8_numpy draws them)."""
+    rng = _rng(seed)
+    G = s.q_heads // s.kv_heads
+    lens = np.array([int(s.context_lens[b]) for b, _ in pairs], np.int32)
+    npages = (lens.astype(np.int64) + s.page_size - 1) // s.page_size
+    total = int(npages.sum())
+    width = max(1, int(npages.max()) if len(pairs) else 1)
+    table = np.full((len(pairs), width), -1, np.int32)
+    off = 0
+    for i, n in enumerate(npages):
+        table[i, :n] = np.arange(off, off + n, dtype=np.int32)
+        off += int(n)
+    shape = (total, 1, s.page_size, s.head_dim)
+    out = dict(block_tables=table, context_lens=lens,
+               q=round_f32(rng.standard_normal((len(pairs), G, s.head_dim), dtype=np.float32), s.dtype))
+    if kv == "int8":
+        out["k_codes"] = rng.integers(-127, 128, size=shape, dtype=np.int8)
+        out["v_codes"] = rng.integers(-127, 128, size=shape, dtype=np.int8)
+        out["k_scales"] = (rng.uniform(1.5, 2.5, size=shape[:-1]) / 127.0).astype(np.float32)
+        out["v_scales"] = (rng.uniform(1.5, 2.5, size=shape[:-1]) / 127.0).astype(np.float32)
+    else:
+        out["k"] = round_f32(rng.standard_normal(shape, dtype=np.float32), s.dtype)
+        out["v"] = round_f32(rng.standard_normal(shape, dtype=np.float32), s.dtype)
+    return out
+
+
 # ----------------------------------------------------------------- int8 pages
 # Stored int8 pages are drawn directly: codes uniform in [-127, 127], per-row fp32 scales
 # uniform in [1.5, 2.5] / 127 (values within about +-2, like the fp16 pools' N(0, 1)), the

@@ -48,3 +48,24 @@ def test_committed_decode_summaries_carry_digest_and_traffic():
             text = f.read()
         assert "- kernel_source_digest: `" in text, n
         assert "- dram_bytes_per_attention_call: " in text, n
+
+
+def test_cpu_baseline_times_both_legs_on_the_same_pairs():
+    import synth
+    s = synth.spec("tiny")
+    res = bench.time_oracle_sample(s, 0.05, seed=3)
+    assert res["single"] > 0 and res["all"] > 0
+    assert res["threads"] >= 1 and res["cores_available"] >= 1 and res["cpu_model"]
+    entry = bench.cpu_baseline_entry(res, "GB/s")
+    assert entry["kind"] == "oracle" and entry["cores"] == res["threads"]
+    assert entry["value"] == res["all"] and entry["single_thread"]["cores"] == 1
+
+
+def test_reference_arm_prints_one_line(capsys):
+    import json
+    assert bench.main(["--impl", "reference", "--workload", "tiny", "--steps", "1", "--warmup", "0"]) == 0
+    lines = [l for l in capsys.readouterr().out.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["value"] > 0 and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]

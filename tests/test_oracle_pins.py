@@ -514,3 +514,26 @@ def test_int8_append_lands_where_the_fp16_append_does():
     assert np.array_equal(vc2, vc_ref) and np.array_equal(vs2, vs_ref)
     assert not np.array_equal(kc2, kc)                  # something was written
     assert np.array_equal(kc2[2, :, 2], kc_ref[2, :, 2])  # page 2 row 2 (token 6 of seq 0)
+
+
+def test_openmp_build_gives_the_same_bits_as_the_plain_build():
+    """The all-core build of the pair routines only spreads independent pairs over threads:
+    every output bit equals the single-thread build's."""
+    sp = synth.random_spec(88, 5, 8, 2, 64, 16, [300, 1, 47, 0, 129], dtype="bf16")
+    pairs = [(b, h) for b in range(sp.batch) for h in range(sp.q_heads)]
+    m = synth.pair_batch_numpy(sp, [(b, g) for b in range(sp.batch) for g in range(sp.kv_heads)], 9)
+    G = sp.q_heads // sp.kv_heads
+    hp = [(i, h) for i in range(m["q"].shape[0]) for h in range(G)]
+    oracle.set_threads(4)
+    a = oracle.decode_attention_pairs(m["q"], m["k"], m["v"], m["block_tables"], m["context_lens"], 0.125, "bf16", hp)
+    b = oracle.decode_attention_pairs(m["q"], m["k"], m["v"], m["block_tables"], m["context_lens"], 0.125, "bf16", hp,
+                                      omp=True)
+    assert np.array_equal(a.view(np.uint64), b.view(np.uint64))
+    m8 = synth.pair_batch_numpy(sp, [(b, g) for b in range(sp.batch) for g in range(sp.kv_heads)], 10, kv="int8")
+    args = (m8["q"], m8["k_codes"], m8["v_codes"], m8["k_scales"], m8["v_scales"], m8["block_tables"],
+            m8["context_lens"], 0.125, "bf16", hp)
+    a8 = oracle.decode_attention_i8_pairs(*args)
+    b8 = oracle.decode_attention_i8_pairs(*args, omp=True)
+    assert np.array_equal(a8.view(np.uint64), b8.view(np.uint64))
+    assert len(pairs) == sp.batch * sp.q_heads
+
