@@ -31,10 +31,11 @@
  *     library kernel before it on the same stream.  The decode calls read cached pages
  *     in that prologue, all but the page of each sequence's newest token; so the calls
  *     that write pages (paged_kv_append, rope_append) let the next kernel start only once
- *     their rows are written, whatever tokens and slots they are given, and
- *     paged_decode_layer, which lets it start earlier, writes only the newest token of
- *     each sequence (position context_lens[b] - 1).  A decode call that directly follows
- *     paged_decode_layer on the same layer must be given the same context_lens.
+ *     their rows are written, whatever tokens and slots they are given, while
+ *     rope_append_step and paged_decode_layer, which let it start earlier, write only the
+ *     newest token of each sequence (position context_lens[b] - 1).  A decode call that
+ *     directly follows one of these two on the same layer must be given the same
+ *     context_lens and block tables.
  *   - Layouts are row-major, innermost index last.  Element type: PKV_F16 (IEEE
  *     binary16) or PKV_BF16 (bfloat16), the same for q, k, v, the pool and the output.
  *   - Device-side index checks: an out-of-range page id or slot is never dereferenced;
@@ -207,6 +208,26 @@ int paged_kv_append(const pkv_pool* pool, int layer, const void* k, const void* 
 int rope_append(const pkv_pool* pool, int layer, void* q, void* k, const void* v,
                 const int32_t* positions, const int64_t* slot_mapping, int n_tokens, int q_heads,
                 double theta, pkv_stream_t stream);
+
+/*
+ * rope_append in the decode step's form ([ENGINE] s4.3 rotate the new token, append it):
+ * one new token per sequence, sequence b's at position L - 1 with L = context_lens[b] (the
+ * new token counted); q[b] [q_heads][head_dim] and k[b] [kv_heads][head_dim] are turned in
+ * place at that position (fp64, one rounding) and the turned k[b] and v[b] are copied bit
+ * for bit (int8 pool: quantised) into row (L - 1) % page_size of page
+ * block_tables[b][(L - 1) / page_size] of `layer`.  Results are identical to rope_append
+ * given positions L - 1 and the slots pkv_slot_mapping gives them; sequences with L <= 0 are
+ * left untouched.  A table entry outside [0, num_pages), or a position past
+ * max_pages_per_seq pages, is skipped and sets PKV_DEVERR_BAD_PAGE.
+ *   q, k, v: device, 16-byte aligned; block_tables [batch][max_pages_per_seq] and
+ *   context_lens [batch]: device int32, as for paged_decode_attention.
+ * Since it writes nothing but each sequence's newest token, it lets the next kernel on the
+ * stream start at once: a paged_decode_attention given the same context_lens and
+ * block_tables prefetches every other page while this call runs.
+ */
+int rope_append_step(const pkv_pool* pool, int layer, void* q, void* k, const void* v,
+                     const int32_t* block_tables, int max_pages_per_seq, const int32_t* context_lens,
+                     int batch, int q_heads, double theta, pkv_stream_t stream);
 
 /*
  * RMSNorm of each row of the decode hidden state ([ENGINE] s4.2: root mean square only,

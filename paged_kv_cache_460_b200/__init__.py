@@ -23,7 +23,7 @@ from ._lib import (PKV_BF16, PKV_DEVERR_BAD_PAGE, PKV_DEVERR_BAD_SLOT, PKV_DEVER
                    PKV_MAX_DECODE_SPLITS, PagedKVError, lib)
 
 __all__ = [
-    "KVPool", "rope_apply", "paged_kv_append", "rope_append", "paged_decode_attention", "rope_table",
+    "KVPool", "rope_apply", "paged_kv_append", "rope_append", "rope_append_step", "paged_decode_attention", "rope_table",
     "paged_decode_layer", "paged_prefill_attention", "rms_norm", "pkv_slot_mapping",
     "pkv_kv_cache_bytes", "pkv_decode_workspace_size", "pkv_decode_default_splits",
     "kv_get_device_error", "DecodeWorkspace", "PagedKVError", "PKV_F16", "PKV_BF16", "PKV_I8",
@@ -212,6 +212,24 @@ def rope_append(pool, layer, q, k, v, positions, slot_mapping, theta=10000.0, st
     st = lib().rope_append(pool.handle, layer, _ptr(q), _ptr(k), _ptr(v), _ptr(positions), _ptr(slot_mapping),
                            k.shape[0], q.shape[1], float(theta), _stream(stream))
     _lib.check("rope_append", st)
+
+
+def rope_append_step(pool, layer, q, k, v, block_tables, context_lens, theta=10000.0, stream=None):
+    """The decode step's RoPE + append: sequence b's new token sits at position
+    context_lens[b] - 1; q [B, q_heads, d] and k [B, kv_heads, d] are turned in place there
+    and k, v written into that position's slot of the page table -- the results of
+    rope_append with those positions and slots, in one launch that lets the next decode
+    call (same lengths and tables) start while it runs."""
+    torch = _torch()
+    _need(q, "q", pool.dtype)
+    _need(k, "k", pool.dtype)
+    _need(v, "v", pool.dtype)
+    _need(block_tables, "block_tables", torch.int32)
+    _need(context_lens, "context_lens", torch.int32)
+    st = lib().rope_append_step(pool.handle, layer, _ptr(q), _ptr(k), _ptr(v), _ptr(block_tables),
+                                block_tables.shape[1], _ptr(context_lens), k.shape[0], q.shape[1], float(theta),
+                                _stream(stream))
+    _lib.check("rope_append_step", st)
 
 
 def paged_prefill_attention(pool, layer, out, q, cu_q, block_tables, context_lens, scale, kv_heads=None,

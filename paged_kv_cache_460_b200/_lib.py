@@ -42,6 +42,7 @@ SIGNATURES = {
     "rope_apply": (_I, [_P, _P, _P, _I, _I, _I, _I, _D, _I, _P]),
     "paged_kv_append": (_I, [_P, _I, _P, _P, _P, _I, _P]),
     "rope_append": (_I, [_P, _I, _P, _P, _P, _P, _P, _I, _I, _D, _P]),
+    "rope_append_step": (_I, [_P, _I, _P, _P, _P, _P, _I, _P, _I, _I, _D, _P]),
     "rms_norm": (_I, [_P, _P, _P, _P, _I, _I, _F, _I, _P]),
     "paged_prefill_attention": (_I, [_P, _I, _P, _P, _P, _I, _P, _I, _P, _I, _I, _I, _F, _P]),
     "pkv_decode_default_splits": (_I, [_I, _I, _I, _I, _I, ctypes.POINTER(_I)]),

@@ -285,6 +285,30 @@ extern "C" int rope_append(const pkv_pool* pool, int layer, void* q, void* k, co
     return launch_rope_append(prm, n_tokens, pool->dtype, reinterpret_cast<cudaStream_t>(stream));
 }
 
+extern "C" int rope_append_step(const pkv_pool* pool, int layer, void* q, void* k, const void* v,
+                                const int32_t* block_tables, int max_pages_per_seq, const int32_t* context_lens,
+                                int batch, int q_heads, double theta, pkv_stream_t stream)
+{
+    if (!pool || layer < 0 || layer >= pool->num_layers || batch < 0 || q_heads < 0 || !(theta > 0.0))
+        return PKV_ERR_INVALID_ARG;
+    if (max_pages_per_seq <= 0) return PKV_ERR_INVALID_ARG;
+    if (batch == 0) return PKV_OK;
+    if (!k || !v || !block_tables || !context_lens || (q_heads > 0 && !q)) return PKV_ERR_INVALID_ARG;
+    if (misaligned16(q, k, v)) return PKV_ERR_INVALID_ARG;
+    RopeAppendParams prm = pool_params(pool, layer);
+    prm.q = q;
+    prm.k = k;
+    prm.v = v;
+    prm.context_lens = context_lens;
+    prm.block_tables = block_tables;
+    prm.max_pages = max_pages_per_seq;
+    prm.q_heads = q_heads;
+    prm.theta = theta;
+    // writes only each sequence's newest token: the next kernel may start at once
+    prm.mode |= kRopeRotate | kRopeAppend | kRopeFromLens | kRopeEarlyRelease;
+    return launch_rope_append(prm, batch, pool->dtype, reinterpret_cast<cudaStream_t>(stream));
+}
+
 extern "C" int rms_norm(void* out, const void* x, void* residual, const void* weight, int rows, int hidden,
                         float eps, int dtype, pkv_stream_t stream)
 {

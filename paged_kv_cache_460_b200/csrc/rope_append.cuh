@@ -18,6 +18,11 @@ constexpr int kRopeQuantI8 = 4;  // ... as int8 codes plus a per-row fp32 scale
 // for launches that write no pool page: the decode kernels read cached pages before their
 // own wait, so a launch that appends releases them only once its rows are written.
 constexpr int kRopeEarlyRelease = 8;
+// The decode step's form: token t is sequence t's newest token, at position
+// context_lens[t] - 1, in the slot its page table gives that position.  Such a launch writes
+// only pages that a decode kernel given the same lengths does not prefetch, so it may also
+// release its dependent early.
+constexpr int kRopeFromLens = 16;
 
 struct RopeAppendParams {
     void* q;                 // [n][q_heads][d]   (rotated in place)
@@ -25,6 +30,9 @@ struct RopeAppendParams {
     const void* v;           // [n][kv_heads][d]
     const int32_t* positions;
     const int64_t* slots;
+    const int32_t* context_lens;     // kRopeFromLens: [n] lengths (new token included)
+    const int32_t* block_tables;     //   and page tables [n][max_pages]
+    int max_pages;
     void* k_layer;           // this layer's K pool [pages][kv_heads][P][d]
     void* v_layer;
     float* ks_layer;         // int8 pools: this layer's row scales [pages][kv_heads][P]
@@ -97,7 +105,7 @@ __global__ void __launch_bounds__(256) rope_append_kernel(const RopeAppendParams
 {
     __shared__ double cs[64][2];
     const int t = blockIdx.x;
-    const int pos = (p.mode & kRopeRotate) ? p.positions[t] : -1;
+    const int pos = (p.mode & kRopeFromLens) ? p.context_lens[t] - 1 : ((p.mode & kRopeRotate) ? p.positions[t] : -1);
     const int half = p.head_dim >> 1;
     if (pos >= 0) {
         for (int i = threadIdx.x; i < half; i += blockDim.x) {
@@ -112,7 +120,16 @@ __global__ void __launch_bounds__(256) rope_append_kernel(const RopeAppendParams
     if (p.mode & kRopeEarlyRelease) pdl_launch_dependents();
     pdl_wait();
     int64_t slot = -1;
-    if (p.mode & kRopeAppend) {
+    if ((p.mode & kRopeAppend) && (p.mode & kRopeFromLens)) {
+        if (pos >= 0) {            // the slot of position pos through the sequence's page table
+            const int j = pos / p.page_size;
+            const int page = j < p.max_pages ? p.block_tables[(int64_t)t * p.max_pages + j] : -1;
+            if (page >= 0 && (int64_t)page * p.page_size < p.num_slots)
+                slot = (int64_t)page * p.page_size + (pos - j * p.page_size);
+            else if (blockIdx.y == 0 && threadIdx.x == 0)
+                atomicOr(&g_error_word, PKV_DEVERR_BAD_PAGE);
+        }
+    } else if (p.mode & kRopeAppend) {
         slot = p.slots[t];
         if (slot >= p.num_slots) {
             if (blockIdx.y == 0 && threadIdx.x == 0) atomicOr(&g_error_word, PKV_DEVERR_BAD_SLOT);

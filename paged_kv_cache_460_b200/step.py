@@ -13,8 +13,7 @@ import math
 
 import torch
 
-from . import (DecodeWorkspace, KVPool, paged_decode_attention, paged_decode_layer, pkv_slot_mapping, rope_append,
-               rope_table)
+from . import (DecodeWorkspace, KVPool, paged_decode_attention, paged_decode_layer, rope_append_step, rope_table)
 
 
 class DecodeStep:
@@ -24,8 +23,9 @@ class DecodeStep:
     batch, q_heads: the step's shape; the kv heads and head_dim are the pool's.
     Device buffers (fill them, or pass host tensors to ``run``):
       q [layers, batch, q_heads, d], k and v [layers, batch, kv_heads, d],
-      block_tables [batch, max_pages] int32, context_lens [batch] int32,
-      positions [batch] int32, slot_mapping [batch] int64, out [layers, batch, q_heads, d].
+      block_tables [batch, max_pages] int32, context_lens [batch] int32 (the new token
+      included: it sits at position context_lens[b] - 1, in the slot the page table gives
+      that position), out [layers, batch, q_heads, d].
     """
 
     def __init__(self, pool: KVPool, batch, q_heads, max_pages, scale=None, theta=10000.0, num_splits=0,
@@ -40,8 +40,6 @@ class DecodeStep:
         self.out = torch.empty((L, batch, q_heads, d), dtype=dt, device=dev)
         self.block_tables = torch.full((batch, max_pages), -1, dtype=torch.int32, device=dev)
         self.context_lens = torch.zeros(batch, dtype=torch.int32, device=dev)
-        self.positions = torch.full((batch,), -1, dtype=torch.int32, device=dev)
-        self.slot_mapping = torch.full((batch,), -1, dtype=torch.int64, device=dev)
         self.scale = 1.0 / math.sqrt(d) if scale is None else scale
         self.theta = theta
         self.workspace = DecodeWorkspace(batch, q_heads, Hkv, d, pool.page_size, dt, num_splits, device=dev,
@@ -55,15 +53,16 @@ class DecodeStep:
 
     def layer(self, i, stream=None):
         """Enqueue layer i of the step on the current stream: RoPE + KV append (one
-        kernel), then attention (one kernel); fused: the whole layer in one kernel (the
-        step's angle table must be current)."""
+        kernel, each sequence's new token at position context_lens[b] - 1 and its slot
+        taken from the page table), then attention (one kernel); fused: the whole layer in
+        one kernel (the step's angle table must be current)."""
         if self.fused:
             paged_decode_layer(self.pool, i, self.out[i], self.q[i], self.k[i], self.v[i], self.rope,
                                self.block_tables, self.context_lens, self.scale,
                                num_splits=self.workspace.num_splits, workspace=self.workspace, stream=stream)
             return
-        rope_append(self.pool, i, self.q[i], self.k[i], self.v[i], self.positions, self.slot_mapping, self.theta,
-                    stream)
+        rope_append_step(self.pool, i, self.q[i], self.k[i], self.v[i], self.block_tables, self.context_lens,
+                         self.theta, stream)
         paged_decode_attention(self.pool, i, self.out[i], self.q[i], self.block_tables, self.context_lens,
                                self.scale, num_splits=self.workspace.num_splits, workspace=self.workspace,
                                stream=stream)
@@ -93,17 +92,11 @@ class DecodeStep:
             self.capture()
         self.graph.replay()
 
-    def set_metadata(self, block_tables, context_lens, positions, non_blocking=True):
-        """Copy page tables, lengths and positions in (host or device tensors); the slot
-        mapping of the new tokens is derived on the host from the same tables."""
-        import numpy as np
-        bt = block_tables.cpu().numpy() if torch.is_tensor(block_tables) else np.asarray(block_tables)
-        pos = positions.cpu().numpy() if torch.is_tensor(positions) else np.asarray(positions)
-        slots = torch.from_numpy(pkv_slot_mapping(bt, pos, self.pool.page_size))
-        self.block_tables.copy_(torch.as_tensor(bt), non_blocking=non_blocking)
+    def set_metadata(self, block_tables, context_lens, non_blocking=True):
+        """Copy the page tables and lengths in (host or device tensors); each sequence's new
+        token position and its slot follow from them on the device."""
+        self.block_tables.copy_(torch.as_tensor(block_tables), non_blocking=non_blocking)
         self.context_lens.copy_(torch.as_tensor(context_lens), non_blocking=non_blocking)
-        self.positions.copy_(torch.as_tensor(pos), non_blocking=non_blocking)
-        self.slot_mapping.copy_(slots, non_blocking=non_blocking)
 
     def run(self, q, k, v, out_host=None):
         """Copy the step's q, k, v (host, ideally pinned) in, replay, copy out to out_host."""

@@ -242,6 +242,21 @@ def test_noalloc_checks_arguments_before_its_scratch_limit(L):
     L.kv_pool_destroy(h)
 
 
+def test_rope_append_step_validates(L):
+    h = _pool(L, num_pages=8, page_size=16, kv_heads=2, head_dim=64)
+    f = _fake_ptr
+    assert L.rope_append_step(None, 0, f(), f(), f(), f(), 4, f(), 1, 2, 10000.0, None) == _lib.PKV_ERR_INVALID_ARG
+    assert L.rope_append_step(h, 1, f(), f(), f(), f(), 4, f(), 1, 2, 10000.0, None) == _lib.PKV_ERR_INVALID_ARG
+    assert L.rope_append_step(h, 0, f(), f(), f(), f(), 0, f(), 1, 2, 10000.0, None) == _lib.PKV_ERR_INVALID_ARG
+    assert L.rope_append_step(h, 0, f(), f(), f(), f(), 4, f(), 1, 2, 0.0, None) == _lib.PKV_ERR_INVALID_ARG
+    assert L.rope_append_step(h, 0, f(), None, f(), f(), 4, f(), 1, 2, 10000.0, None) == _lib.PKV_ERR_INVALID_ARG
+    assert L.rope_append_step(h, 0, f(), f(), f(), None, 4, f(), 1, 2, 10000.0, None) == _lib.PKV_ERR_INVALID_ARG
+    assert L.rope_append_step(h, 0, f(0x10008), f(), f(), f(), 4, f(), 1, 2, 10000.0, None) \
+        == _lib.PKV_ERR_INVALID_ARG                                      # q misaligned
+    assert L.rope_append_step(h, 0, f(), f(), f(), f(), 4, f(), 0, 2, 10000.0, None) == 0
+    L.kv_pool_destroy(h)
+
+
 def test_rope_append_validates(L):
     h = _pool(L, num_pages=8, page_size=16, kv_heads=2, head_dim=64)
     f = _fake_ptr

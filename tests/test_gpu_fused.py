@@ -86,7 +86,7 @@ def test_fused_step_is_bit_identical_to_two_launch_step_at_full_size():
     outs = []
     for pool, fused in zip(pools, (False, True)):
         st = DecodeStep(pool, s.batch, s.q_heads, s.max_pages, theta=s.theta, fused=fused)
-        st.set_metadata(s.block_tables, s.context_lens, s.positions, non_blocking=False)
+        st.set_metadata(s.block_tables, s.context_lens, non_blocking=False)
         st.q.copy_(qs[0])
         st.k.copy_(ks[0])
         st.v.copy_(vs[0])
