@@ -381,10 +381,10 @@ def run_ours(args):
             if fused:                               # the angle table of st0 is current
                 pkv.paged_decode_layer(pool, layer, st0.out[layer], st0.q[layer], st0.k[layer], st0.v[layer],
                                        st0.rope, st0.block_tables, st0.context_lens, st0.scale,
-                                       num_splits=st0.workspace.num_splits, workspace=st0.workspace)
+                                       num_splits=st0.num_splits, workspace=st0.workspace)
             else:
                 pkv.paged_decode_attention(pool, layer, st0.out[layer], st0.q[layer], st0.block_tables,
-                                           st0.context_lens, st0.scale, num_splits=st0.workspace.num_splits,
+                                           st0.context_lens, st0.scale, num_splits=st0.num_splits,
                                            workspace=st0.workspace)
     torch.cuda.current_stream().wait_stream(cs)
     for i in range(args.warmup):
@@ -484,7 +484,7 @@ def run_ours(args):
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": args.steps * steps[0].kernels_per_step * world,
-            "num_splits": steps[0].workspace.num_splits,
+            "num_splits": args.splits or pkv.pkv_decode_auto_splits(pool, s.batch, s.max_pages, s.q_heads),
             "launch": "one CUDA graph per step (%d kernels%s)" % (
                 steps[0].kernels_per_step, ": an angle table, then one fused kernel per layer" if fused else ""),
             "clocks": clk,

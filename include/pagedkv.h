@@ -251,6 +251,19 @@ int pkv_decode_default_splits(int q_heads, int kv_heads, int head_dim, int page_
                               int* num_splits_out);
 
 /*
+ * The split count paged_decode_attention and paged_decode_layer use for num_splits = 0 on
+ * this pool and shape: pkv_decode_default_splits (a full wave of CTAs), or fewer when
+ * kv_heads x batch x the work units of max_pages_per_seq pages (a unit is a page for one
+ * query head per kv head, 16 tokens for grouped heads, 32 tokens on int8 pages) would leave
+ * a CTA fewer than 16 units: ceil(units / 16), at least 1.  Never above
+ * pkv_decode_default_splits, so a workspace sized for that serves every automatic call.
+ * Needs a CUDA device (PKV_ERR_CUDA without one); INVALID_ARG / UNSUPPORTED as for
+ * paged_decode_attention.
+ */
+int pkv_decode_auto_splits(const pkv_pool* pool, int batch, int max_pages_per_seq, int q_heads, int kv_heads,
+                           int* num_splits_out);
+
+/*
  * Workspace bytes paged_decode_attention needs for `num_splits` (1 .. PKV_MAX_DECODE_SPLITS)
  * partitions: a fixed region of PKV_MAX_DECODE_SPLITS int32 counters (16 KiB), then per
  * partition two fp32 partial results (running max, sum and the unnormalised output of every
@@ -277,7 +290,7 @@ size_t pkv_decode_workspace_size(int batch, int q_heads, int kv_heads, int head_
  *   kv_heads must equal the pool's; q_heads a multiple of it with q_heads / kv_heads in
  *   {1, 2, 4, 8}.
  *   num_splits: number of work partitions, at most PKV_MAX_DECODE_SPLITS
- *           (0 = pkv_decode_default_splits).  The batch's
+ *           (0 = pkv_decode_auto_splits for this shape).  The batch's
  *           pages x kv heads are laid end to end and cut into num_splits equal ranges, one
  *           per CTA; a (sequence, kv head) cut by a range boundary is finished by the CTA
  *           that delivers its last partial, which rescales the partial softmax sums

@@ -25,7 +25,7 @@ from ._lib import (PKV_BF16, PKV_DEVERR_BAD_PAGE, PKV_DEVERR_BAD_SLOT, PKV_DEVER
 __all__ = [
     "KVPool", "rope_apply", "paged_kv_append", "rope_append", "rope_append_step", "paged_decode_attention", "rope_table",
     "paged_decode_layer", "paged_prefill_attention", "rms_norm", "pkv_slot_mapping",
-    "pkv_kv_cache_bytes", "pkv_decode_workspace_size", "pkv_decode_default_splits",
+    "pkv_kv_cache_bytes", "pkv_decode_workspace_size", "pkv_decode_default_splits", "pkv_decode_auto_splits",
     "kv_get_device_error", "DecodeWorkspace", "PagedKVError", "PKV_F16", "PKV_BF16", "PKV_I8",
     "PKV_DEVERR_BAD_PAGE", "PKV_DEVERR_BAD_SLOT", "PKV_DEVERR_TIMEOUT", "PKV_MAX_DECODE_SPLITS",
 ]
@@ -163,6 +163,15 @@ def pkv_decode_default_splits(q_heads, kv_heads, head_dim, page_size, dtype=PKV_
     return n.value
 
 
+def pkv_decode_auto_splits(pool, batch, max_pages_per_seq, q_heads, kv_heads=None):
+    """The split count a decode call with num_splits = 0 uses on this pool and shape."""
+    n = ctypes.c_int()
+    _lib.check("pkv_decode_auto_splits",
+               lib().pkv_decode_auto_splits(pool.handle, batch, max_pages_per_seq, q_heads,
+                                            pool.kv_heads if kv_heads is None else kv_heads, ctypes.byref(n)))
+    return n.value
+
+
 def pkv_decode_workspace_size(batch, q_heads, kv_heads, head_dim, num_splits):
     return int(lib().pkv_decode_workspace_size(batch, q_heads, kv_heads, head_dim, num_splits))
 
@@ -273,6 +282,9 @@ class DecodeWorkspace:
     def __init__(self, batch, q_heads, kv_heads, head_dim, page_size, dtype, num_splits=0, device=None,
                  storage=None):
         torch = _torch()
+        # auto: sized for the full wave, which bounds every automatic split count, so calls
+        # may pass num_splits = 0 and let the library choose
+        self.auto = num_splits == 0
         if num_splits == 0:
             code = dtype_code(dtype) if storage is None else storage
             num_splits = pkv_decode_default_splits(q_heads, kv_heads, head_dim, page_size, code)
@@ -295,7 +307,7 @@ def paged_decode_attention(pool, layer, out, q, block_tables, context_lens, scal
     if workspace is None:
         workspace = DecodeWorkspace(B, Hq, kv_heads, pool.head_dim, pool.page_size, pool.dtype, num_splits,
                                     device=q.device, storage=pool.storage)
-    if num_splits == 0:
+    if num_splits == 0 and not workspace.auto:
         num_splits = workspace.num_splits
     st = lib().paged_decode_attention(pool.handle, layer, _ptr(out), _ptr(q), _ptr(block_tables),
                                       block_tables.shape[1], _ptr(context_lens), B, Hq, kv_heads, float(scale),
@@ -333,7 +345,7 @@ def paged_decode_layer(pool, layer, out, q, k, v, rope, block_tables, context_le
     if workspace is None:
         workspace = DecodeWorkspace(B, Hq, pool.kv_heads, pool.head_dim, pool.page_size, pool.dtype, num_splits,
                                     device=q.device, storage=pool.storage)
-    if num_splits == 0:
+    if num_splits == 0 and not workspace.auto:
         num_splits = workspace.num_splits
     st = lib().paged_decode_layer(pool.handle, layer, _ptr(out), _ptr(q), _ptr(k), _ptr(v), _ptr(rope),
                                   _ptr(block_tables), block_tables.shape[1], _ptr(context_lens), B, Hq, pool.kv_heads,

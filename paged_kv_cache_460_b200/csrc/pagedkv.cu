@@ -66,7 +66,27 @@ struct DecodeOps {
     int (*launch)(const DecodeParams&, cudaStream_t);
     int (*splits)(int*);
     int group;
+    int unit_tokens;    // tokens of one work unit: a page (CUDA cores), 16 (MMA), 32 (int8)
 };
+
+// The automatic split count: the device's full wave (SMs x resident CTAs), unless the
+// batch's work is too small to give every CTA at least kMinUnitsPerCta units; then fewer,
+// fuller CTAs -- each CTA pays a fixed cost (lengths scan, first page-table window, ring
+// fill, merge of its cut segments) that a few units do not amortise.  The host knows only
+// an upper bound of the work: kv_heads x batch x the units of max_pages_per_seq pages.
+constexpr long long kMinUnitsPerCta = 16;
+
+int auto_splits(int full_wave, long long max_units)
+{
+    const long long n = (max_units + kMinUnitsPerCta - 1) / kMinUnitsPerCta;
+    return n < 1 ? 1 : (n < full_wave ? (int)n : full_wave);
+}
+
+long long max_decode_units(int kv_heads, int batch, int max_pages, int page_size, int unit_tokens)
+{
+    const long long per_seq = ((long long)max_pages * page_size + unit_tokens - 1) / unit_tokens;
+    return (long long)kv_heads * batch * per_seq;
+}
 
 // One query head per kv head: the CUDA-core kernel; 2 to 8 heads sharing a kv head: the
 // tensor-core kernel.  Int8 pages (I8): the int8 tensor-core kernel for every group size.
@@ -124,11 +144,12 @@ int DecodeImpl<D, P, G, T, I8>::configured[kMaxDevices] = {0};
 template <int D, int P, typename T, bool I8>
 bool pick_group(int group, DecodeOps& ops)
 {
+    const int ut = I8 ? 32 : (group == 1 ? P : 16);
     switch (group) {
-    case 1: ops = {DecodeImpl<D, P, 1, T, I8>::launch, DecodeImpl<D, P, 1, T, I8>::splits, 1}; return true;
-    case 2: ops = {DecodeImpl<D, P, 2, T, I8>::launch, DecodeImpl<D, P, 2, T, I8>::splits, 2}; return true;
-    case 4: ops = {DecodeImpl<D, P, 4, T, I8>::launch, DecodeImpl<D, P, 4, T, I8>::splits, 4}; return true;
-    case 8: ops = {DecodeImpl<D, P, 8, T, I8>::launch, DecodeImpl<D, P, 8, T, I8>::splits, 8}; return true;
+    case 1: ops = {DecodeImpl<D, P, 1, T, I8>::launch, DecodeImpl<D, P, 1, T, I8>::splits, 1, ut}; return true;
+    case 2: ops = {DecodeImpl<D, P, 2, T, I8>::launch, DecodeImpl<D, P, 2, T, I8>::splits, 2, ut}; return true;
+    case 4: ops = {DecodeImpl<D, P, 4, T, I8>::launch, DecodeImpl<D, P, 4, T, I8>::splits, 4, ut}; return true;
+    case 8: ops = {DecodeImpl<D, P, 8, T, I8>::launch, DecodeImpl<D, P, 8, T, I8>::splits, 8, ut}; return true;
     default: return false;
     }
 }
@@ -341,6 +362,23 @@ extern "C" int pkv_decode_default_splits(int q_heads, int kv_heads, int head_dim
     return ops.splits(num_splits_out);
 }
 
+extern "C" int pkv_decode_auto_splits(const pkv_pool* pool, int batch, int max_pages_per_seq, int q_heads,
+                                      int kv_heads, int* num_splits_out)
+{
+    if (!pool || !num_splits_out || batch < 0 || max_pages_per_seq <= 0 || q_heads <= 0 || kv_heads != pool->kv_heads ||
+        q_heads % kv_heads)
+        return PKV_ERR_INVALID_ARG;
+    DecodeOps ops;
+    if (!pick_decode(pool->head_dim, pool->page_size, q_heads / kv_heads, pool->dtype, pool->storage, ops))
+        return PKV_ERR_UNSUPPORTED;
+    int full = 0;
+    const int st = ops.splits(&full);
+    if (st != PKV_OK) return st;
+    *num_splits_out = auto_splits(full, max_decode_units(kv_heads, batch, max_pages_per_seq, pool->page_size,
+                                                         ops.unit_tokens));
+    return PKV_OK;
+}
+
 extern "C" size_t pkv_decode_workspace_size(int batch, int q_heads, int kv_heads, int head_dim, int num_splits)
 {
     if (batch < 0 || q_heads <= 0 || kv_heads <= 0 || q_heads % kv_heads || head_dim <= 0 || num_splits <= 0 ||
@@ -368,6 +406,8 @@ extern "C" int paged_decode_attention(const pkv_pool* pool, int layer, void* out
     if (num_splits == 0) {
         const int st = ops.splits(&num_splits);
         if (st != PKV_OK) return st;
+        num_splits = auto_splits(num_splits, max_decode_units(kv_heads, batch, max_pages_per_seq, pool->page_size,
+                                                              ops.unit_tokens));
     }
     const WorkspaceLayout wl = workspace_layout(batch, ops.group, pool->head_dim, num_splits);
     if (workspace_bytes < wl.total) return PKV_ERR_NO_SPACE;
@@ -405,11 +445,22 @@ namespace {
 // the CUDA-core kernel for 16-bit pages with one query head per kv head, the int8 kernel
 // for int8 pages with any group size.
 template <int D, int P, int G, typename T, bool I8>
+struct FusedKernel {      // 16-bit pages: the CUDA-core kernel (one query head per kv head)
+    static constexpr auto fn = decode_pass1_kernel<D, P, G, T, true>;
+    static int smem(int batch) { return DecodeShape<D, P, G>::smem_bytes(batch); }
+};
+template <int D, int P, int G, typename T>
+struct FusedKernel<D, P, G, T, true> {
+    static constexpr auto fn = decode_i8_kernel<D, P, G, T, true>;
+    static int smem(int batch) { return I8Shape<D, G>::smem_bytes(batch); }
+};
+
+template <int D, int P, int G, typename T, bool I8>
 int launch_fused(const DecodeParams& prm, cudaStream_t st)
 {
     static int configured[kMaxDevices] = {0};
-    constexpr auto fn = I8 ? decode_i8_kernel<D, P, G, T, true> : decode_pass1_kernel<D, P, G, T, true>;
-    const int smem = I8 ? I8Shape<D, G>::smem_bytes(prm.batch) : DecodeShape<D, P, G>::smem_bytes(prm.batch);
+    constexpr auto fn = FusedKernel<D, P, G, T, I8>::fn;
+    const int smem = FusedKernel<D, P, G, T, I8>::smem(prm.batch);
     if (smem > kMaxSmemPerCta) return PKV_ERR_UNSUPPORTED;
     if (ensure_smem(fn, smem, configured) != cudaSuccess) return PKV_ERR_CUDA;
     return status_of(launch_pdl(fn, dim3(prm.num_splits), dim3(kDecodeThreads), smem, st, prm));
@@ -474,6 +525,8 @@ extern "C" int paged_decode_layer(const pkv_pool* pool, int layer, void* out, co
     if (num_splits == 0) {
         const int st = ops.splits(&num_splits);
         if (st != PKV_OK) return st;
+        num_splits = auto_splits(num_splits, max_decode_units(kv_heads, batch, max_pages_per_seq, pool->page_size,
+                                                              ops.unit_tokens));
     }
     const WorkspaceLayout wl = workspace_layout(batch, group, pool->head_dim, num_splits);
     if (workspace_bytes < wl.total) return PKV_ERR_NO_SPACE;

@@ -42,6 +42,7 @@ class DecodeStep:
         self.context_lens = torch.zeros(batch, dtype=torch.int32, device=dev)
         self.scale = 1.0 / math.sqrt(d) if scale is None else scale
         self.theta = theta
+        self.num_splits = num_splits          # 0: the library's automatic choice for the shape
         self.workspace = DecodeWorkspace(batch, q_heads, Hkv, d, pool.page_size, dt, num_splits, device=dev,
                                          storage=pool.storage)
         self.graph = None
@@ -59,12 +60,12 @@ class DecodeStep:
         if self.fused:
             paged_decode_layer(self.pool, i, self.out[i], self.q[i], self.k[i], self.v[i], self.rope,
                                self.block_tables, self.context_lens, self.scale,
-                               num_splits=self.workspace.num_splits, workspace=self.workspace, stream=stream)
+                               num_splits=self.num_splits, workspace=self.workspace, stream=stream)
             return
         rope_append_step(self.pool, i, self.q[i], self.k[i], self.v[i], self.block_tables, self.context_lens,
                          self.theta, stream)
         paged_decode_attention(self.pool, i, self.out[i], self.q[i], self.block_tables, self.context_lens,
-                               self.scale, num_splits=self.workspace.num_splits, workspace=self.workspace,
+                               self.scale, num_splits=self.num_splits, workspace=self.workspace,
                                stream=stream)
 
     def eager(self):
