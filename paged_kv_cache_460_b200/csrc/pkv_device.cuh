@@ -19,6 +19,21 @@ __device__ unsigned int g_error_word = 0;
 // B200's clocks); a healthy wait ends within microseconds.
 constexpr long long kWaitLimitCycles = 2000000000LL;
 
+// The limit of the waits through which a warp consumes another's work (mbar_wait_bounded).
+// A test build may shorten it (-DPKV_CONSUMER_WAIT_LIMIT_CYCLES=...) to drive the abort
+// path, and poll the barrier with the non-blocking test_wait, checking the limit at every
+// probe (-DPKV_CONSUMER_WAIT_POLL=1): try_wait may suspend the thread until the phase
+// completes, so a healthy wait would never see a short limit run out.  The drain waits for
+// copies and MMAs already in flight keep try_wait and kWaitLimitCycles, so no CTA exits, or
+// frees tensor memory, with asynchronous writes outstanding.
+#ifndef PKV_CONSUMER_WAIT_LIMIT_CYCLES
+#define PKV_CONSUMER_WAIT_LIMIT_CYCLES 2000000000LL
+#endif
+#ifndef PKV_CONSUMER_WAIT_POLL
+#define PKV_CONSUMER_WAIT_POLL 0
+#endif
+constexpr long long kConsumerWaitLimitCycles = PKV_CONSUMER_WAIT_LIMIT_CYCLES;
+
 __device__ __forceinline__ uint32_t smem_addr(const void* p)
 {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -65,18 +80,43 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity)
     return done != 0;
 }
 
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity)
+{
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
 // Wait until the phase with the given parity has completed.  Gives up (returns
-// false) when *abort is set by another warp, or after kWaitLimitCycles, in which
-// case it sets *abort and PKV_DEVERR_TIMEOUT.
+// false) when *abort is set by another warp, or after kConsumerWaitLimitCycles, in
+// which case it sets *abort and PKV_DEVERR_TIMEOUT.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort)
 {
+#if PKV_CONSUMER_WAIT_POLL
+    const long long t_poll = clock64();
+    for (;;) {
+        if (mbar_test_wait(bar, parity)) return true;
+        if (*abort) return false;
+        if (clock64() - t_poll > kConsumerWaitLimitCycles) {
+            *abort = 1;
+            atomicOr(&g_error_word, PKV_DEVERR_TIMEOUT);
+            return false;
+        }
+    }
+#endif
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     for (uint32_t n = 1;; ++n) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((n & 31u) == 0) {
             if (*abort) return false;
-            if (clock64() - t0 > kWaitLimitCycles) {
+            if (clock64() - t0 > kConsumerWaitLimitCycles) {
                 *abort = 1;
                 atomicOr(&g_error_word, PKV_DEVERR_TIMEOUT);
                 return false;
