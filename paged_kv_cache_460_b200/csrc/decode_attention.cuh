@@ -46,7 +46,9 @@ constexpr int kDecodeThreads = kDecodeWarps * 32;
 // is held to 128 registers so that a RoPE/append CTA still fits beside them).  Deeper
 // rings (3-5 slots) measured slower on the 10-request, 32-layer decode workload.
 constexpr int kRingBudgetBytes = 68 * 1024;
-constexpr int kMaxMergeParts = 4;   // partials loaded per merge round
+// Partials loaded per merge round.  Eight per round measured slower on every workload: the
+// merge is inlined in the segment loop and its registers cost the hot loop spills.
+constexpr int kMaxMergeParts = 4;
 
 struct DecodeParams {
     const void* k;              // this layer's K pool  [pages][kv_heads][P][D]
@@ -74,7 +76,12 @@ struct DecodeParams {
 
 __host__ __device__ constexpr int align_up(int x, int a) { return (x + a - 1) / a * a; }
 
-template <int D, int P, int G>
+// kFused: the fused layer also keeps, per CTA, the angle-table rows of the first two
+// sequences its range touches and the new k and v rows of the first two sequence ends in its
+// range (kNewRows rows of D elements), so that turning q at a segment's start and the append
+// at a sequence's end read shared memory instead of waiting on global loads; the ids of those
+// rows follow (kFusedIds ints).
+template <int D, int P, int G, bool kFused = false>
 struct DecodeShape {
     static constexpr int kChunk = P * D * 2;                 // bytes of one (page, head)
     static constexpr int kQBytes = G * D * 2;
@@ -86,7 +93,12 @@ struct DecodeShape {
     static constexpr int kCmbFloats = kDecodeWarps * G * (D + 2);
     static constexpr int kPbufOffset = kCmbOffset + 2 * kCmbFloats * 4;     // [warps][G][P] floats
     static constexpr int kWarpTotOffset = kPbufOffset + kDecodeWarps * G * P * 4;
-    static constexpr int kScanOffset = kWarpTotOffset + 64;
+    static constexpr int kRopeRows = kFused ? 2 : 0;
+    static constexpr int kRopeOffset = kWarpTotOffset + 64;                 // [kRopeRows][D/2][2] doubles
+    static constexpr int kNewOffset = kRopeOffset + kRopeRows * D * 8;      // [2][k, v][D] of T
+    static constexpr int kNewRows = kFused ? 4 : 0;
+    static constexpr int kIdsOffset = kNewOffset + kNewRows * D * 2;        // rope b[2], append (b*Hkv+g)[2]
+    static constexpr int kScanOffset = kIdsOffset + (kFused ? 16 : 0);
     // prefix[batch+1] and lens[batch] follow
     static int smem_bytes(int batch) { return kScanOffset + 4 * (2 * batch + 1); }
 };
@@ -153,6 +165,50 @@ __device__ __forceinline__ void next_unit(int& b, int& g, int& j, int& np, const
     } while (np == 0);
 }
 
+// A release/acquire fence at gpu scope: with the CTA barrier before it, the partials that
+// the CTA's threads wrote are visible to whichever CTA reads the delivery counter after it.
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+
+// Before the PDL wait, pull into L2 the q rows of (b, g)'s query heads (G x D elements of T,
+// one 128-byte line per lane), which the kernel reads right after the wait, so that read
+// finds them in L2 instead of DRAM.  If the kernel ahead is still writing q, the prefetched
+// lines are only an older copy in L2, which its writes update (L2 is the coherence point);
+// nothing is read into registers or shared memory before the wait.
+template <int D, int G, typename T>
+__device__ __forceinline__ void prefetch_q_rows(const DecodeParams& p, int b, int g, int lane)
+{
+    constexpr int kLines = (G * D * (int)sizeof(T) + 127) / 128;
+    const unsigned char* q = reinterpret_cast<const unsigned char*>(static_cast<const T*>(p.q) +
+                                                                    ((long long)b * p.q_heads + (long long)g * G) * D);
+    if (lane < kLines) prefetch_l2(q + lane * 128);
+}
+
+// Before the PDL wait, pull into L2 with the evict-last priority the workspace lines this
+// CTA writes at its segment ends -- its two partial slots, and the delivery counters of the
+// segments its range cuts (its own index and its first segment's first CTA).  The workspace
+// is touched once per call, so the KV stream of a call would otherwise push those lines out
+// and the partial stores and counter atomics at the CTA's end, on the kernel's critical path,
+// would go to DRAM.  Only L2 lines move; nothing is read or written before the wait.
+template <int D, int G>
+__device__ __forceinline__ void prefetch_epilogue_lines(const DecodeParams& p, long long r0, long long chunk,
+                                                        const int* prefix, int tid)
+{
+    constexpr int kSlotBytes = 2 * G * D * 4;                       // both partial slots of this CTA
+    if (tid < kSlotBytes / 128) {
+        prefetch_l2_evict_last(reinterpret_cast<const unsigned char*>(p.part_o + (long long)blockIdx.x * 2 * G * D) +
+                               tid * 128);
+    } else if (tid == kSlotBytes / 128) {
+        prefetch_l2_evict_last(p.part_ml + (long long)blockIdx.x * 2 * G * 2);
+    } else if (tid == kSlotBytes / 128 + 1) {
+        prefetch_l2_evict_last(p.counters + blockIdx.x);
+    } else if (tid == kSlotBytes / 128 + 2) {
+        int b, g, j;                                                // the first segment's first CTA
+        locate_unit(r0, prefix, p.batch, p.kv_heads, b, g, j);
+        const long long seg0 = (long long)p.kv_heads * prefix[b] + (long long)g * (prefix[b + 1] - prefix[b]);
+        prefetch_l2_evict_last(p.counters + seg0 / chunk);
+    }
+}
+
 // End of a segment, after every warp has published its (m, l, o) of it in `buf`
 // ([warps][G][D + 2]: o, then m and l): combine the warps; a segment wholly inside the
 // CTA's range [r0, r1) is normalised and written as the output, a cut one leaves a
@@ -160,8 +216,9 @@ __device__ __forceinline__ void next_unit(int& b, int& g, int& j, int& np, const
 // after it), and the CTA that delivers the last partial of a segment merges them:
 // M = max m_k, out = sum_k 2^(m_k - M) o_k / sum_k 2^(m_k - M) l_k.  The delivery is
 // counted with an atomic in the workspace (indexed by the segment's first CTA); one
-// thread publishes the CTA's writes with a gpu-scope fence (cumulative over the barrier)
-// and the merging CTA reads the other partials through L2, then resets the counter.
+// thread publishes the CTA's writes with a gpu-scope release fence (cumulative over the
+// barrier) and the merging CTA, after an acquire fence, reads the other partials through
+// L2, then resets the counter.
 template <int D, int G, typename T>
 __device__ __forceinline__ void segment_epilogue(const DecodeParams& p, const float* buf, int b, int g, int np,
                                                  const int* prefix, long long r0, long long r1, long long chunk,
@@ -199,15 +256,15 @@ __device__ __forceinline__ void segment_epilogue(const DecodeParams& p, const fl
     }
     if (!complete) {
         // Deliver this partial; the CTA that delivers the last one merges the segment.
-        // One thread publishes the CTA's writes (a gpu-scope fence is cumulative over
-        // the barrier) and counts them in; the merging CTA reads the other partials
+        // One thread publishes the CTA's writes (a gpu-scope release fence is cumulative
+        // over the barrier) and counts them in; the merging CTA reads the other partials
         // through L2.
         const int c0 = (int)(seg0 / chunk), c1 = (int)((seg0 + np - 1) / chunk);
         named_barrier(1, kDecodeThreads);
         if (tid == 0) {
-            __threadfence();
+            fence_acq_rel_gpu();          // release: the CTA's partial (ordered by the barrier)
             const bool last = atomicAdd(&p.counters[c0], 1) == c1 - c0;
-            if (last) __threadfence();
+            if (last) fence_acq_rel_gpu();   // acquire: the other CTAs' partials
             *last_flag = last;
         }
         named_barrier(1, kDecodeThreads);
@@ -256,7 +313,7 @@ __device__ __forceinline__ void segment_epilogue(const DecodeParams& p, const fl
 template <int D, int P, int G, typename T, bool kFused = false>
 __global__ void __launch_bounds__(kDecodeThreads, G == 1 ? 4 : 1) decode_pass1_kernel(const DecodeParams p)
 {
-    using S = DecodeShape<D, P, G>;
+    using S = DecodeShape<D, P, G, kFused>;
     constexpr int NW = kDecodeWarps;
     constexpr int DEPTH = S::kDepth;
     constexpr int CPR = D / 8;            // 16-byte chunks per K/V row
@@ -361,9 +418,62 @@ __global__ void __launch_bounds__(kDecodeThreads, G == 1 ? 4 : 1) decode_pass1_k
         }
         advance();
     };
+    // Fused layer: which angle-table rows and new k, v rows this CTA keeps (see DecodeShape),
+    // and the angle rows themselves, fetched before the PDL wait -- the table is written once
+    // per step by rope_table, which releases its successor only after writing it.
+    int* fids = reinterpret_cast<int*>(smem + S::kIdsOffset);
+    double* rope_c = reinterpret_cast<double*>(smem + S::kRopeOffset);
+    T* new_c = reinterpret_cast<T*>(smem + S::kNewOffset);
+    if constexpr (kFused) {
+        if (tid == 0) {
+            int nr = 0, na = 0;
+            fids[0] = fids[1] = fids[2] = fids[3] = -1;
+            if (r0 < r1) {
+                int sb, sg, sj;
+                locate_unit(r0, prefix, p.batch, Hkv, sb, sg, sj);
+                int snp = prefix[sb + 1] - prefix[sb];
+                for (long long su = r0; su < r1 && (nr < 2 || na < 2);) {
+                    const long long s_end = (long long)Hkv * prefix[sb] + (long long)(sg + 1) * snp;
+                    if (nr < 2 && (nr == 0 || fids[nr - 1] != sb)) fids[nr++] = sb;
+                    if (na < 2 && s_end <= r1) fids[2 + na++] = sb * Hkv + sg;
+                    su = s_end;
+                    if (++sg == Hkv) {
+                        sg = 0;
+                        do {
+                            ++sb;
+                            snp = sb < p.batch ? prefix[sb + 1] - prefix[sb] : 1;
+                        } while (snp == 0);
+                    }
+                }
+            }
+        }
+        __syncthreads();
+        constexpr int RV = D * 8 / 16;                       // 16-byte pieces of one angle row
+        for (int i = tid; i < 2 * RV; i += kDecodeThreads)
+            if (fids[i / RV] >= 0)
+                cp_async16(reinterpret_cast<unsigned char*>(rope_c) + i * 16,
+                           reinterpret_cast<const unsigned char*>(p.rope + (long long)fids[i / RV] * D) + (i % RV) * 16);
+    }
+    auto rope_row = [&](int bb) -> const double* {
+        if constexpr (kFused) {
+            if (fids[0] == bb) return rope_c;
+            if (fids[1] == bb) return rope_c + D;
+        }
+        return p.rope + (long long)bb * D;
+    };
     // Before waiting on the previous kernel: prefetch this warp's first pages, except a
     // page holding a sequence's newest token (a fused layer before this kernel may still
     // be writing it) and the q rows (the kernel before may still be producing them).
+    if (n_mine > 0) prefetch_q_rows<D, G, T>(p, ib, ig, lane);     // this warp's first segment
+    if (r0 < r1) prefetch_epilogue_lines<D, G>(p, r0, chunk, prefix, tid);
+    if constexpr (kFused) {                   // the new k, v rows of the kept sequence ends
+        constexpr int kRowLines = (D * (int)sizeof(T) + 127) / 128;
+        if (warp == 0 && lane < 4 * kRowLines && fids[2 + lane / (2 * kRowLines)] >= 0) {
+            const int a = lane / (2 * kRowLines), kv = (lane / kRowLines) & 1;
+            prefetch_l2(reinterpret_cast<const unsigned char*>(static_cast<const T*>(kv ? p.v_new : p.k_new) +
+                                                               (long long)fids[2 + a] * D) + (lane % kRowLines) * 128);
+        }
+    }
     int m_pre = 0, pre_qb[DEPTH], pre_qg[DEPTH];
     for (; m_pre < DEPTH && m_pre < n_mine; ++m_pre) {
         if (!kFused && ij == inp - 1) break;
@@ -393,12 +503,23 @@ __global__ void __launch_bounds__(kDecodeThreads, G == 1 ? 4 : 1) decode_pass1_k
     float* pbuf = pbuf_all + warp * G * P;
     for (int k = 0; k < m_pre; ++k)
         if (pre_qb[k] >= 0) issue_q(k, pre_qb[k], pre_qg[k]);
+    if constexpr (kFused) {                   // the new k, v rows of the kept sequence ends
+        constexpr int NV = D * 2 / 16;        // 16-byte pieces of one row
+        for (int i = tid; i < 4 * NV; i += kDecodeThreads) {
+            const int a = i / (2 * NV), kv = (i / NV) & 1;
+            if (fids[2 + a] >= 0)
+                cp_async16(reinterpret_cast<unsigned char*>(new_c) + i * 16,
+                           reinterpret_cast<const unsigned char*>(static_cast<const T*>(kv ? p.v_new : p.k_new) +
+                                                                  (long long)fids[2 + a] * D) + (i % NV) * 16);
+        }
+    }
     if (m_pre == DEPTH) cp_async_commit();
     for (int k = m_pre; k < DEPTH; ++k) {
         if (k < n_mine) issue(k);
         cp_async_commit();
     }
     cp_async_wait<0>();
+    if constexpr (kFused) __syncthreads();   // the CTA's kept rows, copied by all threads
 
     // ---- compute side.  q.k: lane (t, h) = (lane / 2, lane % 2) dots rows t (and t + 16
     // at P = 32) over chunks h*CPL .. h*CPL+CPL-1; p.V: lane owns output columns
@@ -437,9 +558,14 @@ __global__ void __launch_bounds__(kDecodeThreads, G == 1 ? 4 : 1) decode_pass1_k
                     if (lane < 2 * CPR) {
                         const bool is_v = lane >= CPR;
                         const int c = is_v ? lane - CPR : lane;
-                        uint4 w = reinterpret_cast<const uint4*>(static_cast<const T*>(is_v ? p.v_new : p.k_new) +
-                                                                 ((long long)b * Hkv + g) * D)[c];
-                        if (!is_v) rope_rotate8<T>(w, p.rope + (long long)b * D, 4 * c);
+                        const int bg = b * Hkv + g;
+                        const T* src = fids[2] == bg ? new_c : fids[3] == bg ? new_c + 2 * D
+                                                                              : static_cast<const T*>(p.k_new) + (long long)bg * D;
+                        if (is_v)
+                            src = fids[2] == bg ? new_c + D : fids[3] == bg ? new_c + 3 * D
+                                                                             : static_cast<const T*>(p.v_new) + (long long)bg * D;
+                        uint4 w = reinterpret_cast<const uint4*>(src)[c];
+                        if (!is_v) rope_rotate8<T>(w, rope_row(b), 4 * c);
                         if (is_v)
                             *reinterpret_cast<uint4*>(s + S::kChunk + tn * (2 * D) + c * 16) = w;
                         else
@@ -457,7 +583,7 @@ __global__ void __launch_bounds__(kDecodeThreads, G == 1 ? 4 : 1) decode_pass1_k
                     for (int n = lane; n < G * CPR; n += 32) {
                         uint4* qv = reinterpret_cast<uint4*>(s + 2 * S::kChunk) + n;
                         uint4 w = *qv;
-                        rope_rotate8<T>(w, p.rope + (long long)b * D, 4 * (n % CPR));
+                        rope_rotate8<T>(w, rope_row(b), 4 * (n % CPR));
                         *qv = w;
                     }
                     __syncwarp();

@@ -235,6 +235,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_i8_kernel(const Deco
         }
         advance();
     };
+    if (n_mine > 0) prefetch_q_rows<D, G, T>(p, ib, ig, lane);     // this warp's first segment
+    if (r0 < r1) prefetch_epilogue_lines<D, G>(p, r0, chunk, prefix, tid);
     int m_pre = 0, pre_qb[DEPTH], pre_qg[DEPTH];
     for (; m_pre < DEPTH && m_pre < n_mine; ++m_pre) {
         if (!kFused && ij == inp - 1) break;

@@ -141,10 +141,13 @@ struct DecodeImpl {
 template <int D, int P, int G, typename T, bool I8>
 int DecodeImpl<D, P, G, T, I8>::configured[kMaxDevices] = {0};
 
+// Tokens of one work unit of the decode kernel for this page size, group and storage.
+constexpr int unit_tokens(int P, int group, bool i8) { return i8 ? 32 : (group == 1 ? P : 16); }
+
 template <int D, int P, typename T, bool I8>
 bool pick_group(int group, DecodeOps& ops)
 {
-    const int ut = I8 ? 32 : (group == 1 ? P : 16);
+    const int ut = unit_tokens(P, group, I8);
     switch (group) {
     case 1: ops = {DecodeImpl<D, P, 1, T, I8>::launch, DecodeImpl<D, P, 1, T, I8>::splits, 1, ut}; return true;
     case 2: ops = {DecodeImpl<D, P, 2, T, I8>::launch, DecodeImpl<D, P, 2, T, I8>::splits, 2, ut}; return true;
@@ -447,7 +450,7 @@ namespace {
 template <int D, int P, int G, typename T, bool I8>
 struct FusedKernel {      // 16-bit pages: the CUDA-core kernel (one query head per kv head)
     static constexpr auto fn = decode_pass1_kernel<D, P, G, T, true>;
-    static int smem(int batch) { return DecodeShape<D, P, G>::smem_bytes(batch); }
+    static int smem(int batch) { return DecodeShape<D, P, G, true>::smem_bytes(batch); }
 };
 template <int D, int P, int G, typename T>
 struct FusedKernel<D, P, G, T, true> {

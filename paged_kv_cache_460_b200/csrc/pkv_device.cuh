@@ -152,6 +152,19 @@ __device__ __forceinline__ void cp_async16(void* dst, const void* src)
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
 }
 
+// Pull the 128-byte line holding `p` into L2 (no register result, no L1 fill).
+__device__ __forceinline__ void prefetch_l2(const void* p)
+{
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
+// Pull the line holding `p` into L2 with the evict-last priority, so that a stream of
+// normal-priority lines passing through L2 does not push it out before it is used.
+__device__ __forceinline__ void prefetch_l2_evict_last(const void* p)
+{
+    asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(p));
+}
+
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 
 // Wait until at most N of this thread's committed cp.async groups are still in flight.

@@ -66,12 +66,12 @@ __device__ __forceinline__ void rope_rotate8(uint4& u, const double* cs, int i0)
 // Angles of the decode step's new tokens, shared by every layer of the step: for sequence b
 // with L = context_lens[b] cached tokens (the new one included), position L - 1, and pair i,
 // table[b][i] = (cos, sin)(pos * theta^(-2i/d)), evaluated in fp64 exactly as the RoPE
-// kernel does.  Sequences with no token get zeros.
+// kernel does.  Sequences with no token get zeros.  The kernel lets its successor start only
+// after its rows are written and fenced: the fused layer reads the table before its own wait.
 __global__ void __launch_bounds__(64) rope_table_kernel(const int32_t* __restrict__ context_lens, int head_dim,
                                                         double theta, double* __restrict__ table)
 {
     pdl_wait();
-    pdl_launch_dependents();
     const int b = blockIdx.x, half = head_dim >> 1;
     const int pos = context_lens[b] - 1;
     for (int i = threadIdx.x; i < half; i += blockDim.x) {
@@ -83,6 +83,9 @@ __global__ void __launch_bounds__(64) rope_table_kernel(const int32_t* __restric
         table[((long long)b * half + i) * 2] = cn;
         table[((long long)b * half + i) * 2 + 1] = sn;
     }
+    __threadfence();
+    __syncthreads();
+    pdl_launch_dependents();
 }
 
 // Grid: (token, part).  Each thread handles one 16-byte vector (8 elements, 4 pairs)
