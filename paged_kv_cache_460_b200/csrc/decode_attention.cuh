@@ -76,6 +76,13 @@ struct DecodeParams {
 
 __host__ __device__ constexpr int align_up(int x, int a) { return (x + a - 1) / a * a; }
 
+// CTAs of `smem` dynamic shared-memory bytes that fit on one SM (228 KB, 1 KB reserved per
+// CTA), between 1 and 3 (three is the most the decode kernels are tuned for).
+__host__ __device__ constexpr int ctas_per_sm(int smem)
+{
+    return (228 * 1024) / (smem + 1024) >= 3 ? 3 : ((228 * 1024) / (smem + 1024) < 1 ? 1 : (228 * 1024) / (smem + 1024));
+}
+
 // kFused: the fused layer also keeps, per CTA, the angle-table rows of the first two
 // sequences its range touches and the new k and v rows of the first two sequence ends in its
 // range (kNewRows rows of D elements), so that turning q at a segment's start and the append

@@ -50,6 +50,7 @@ struct I8Shape {
     static constexpr int kWarpTotOffset = kCmbOffset + 2 * kCmbFloats * 4;
     static constexpr int kScanOffset = kWarpTotOffset + 64;
     static int smem_bytes(int batch) { return kScanOffset + 4 * (2 * batch + 1); }
+    static constexpr int kCtasPerSm = ctas_per_sm(kScanOffset + 4 * (2 * 64 + 1));
 };
 
 // Position of 16-byte chunk c of token row t in shared memory: c ^ swizzle(t), so that the
@@ -122,8 +123,11 @@ __device__ __forceinline__ uint2 i8_quantise_vec(const uint4& u, int vpr, bool a
 // in shared memory from the step's angle table at each segment's first unit; the warp that
 // owns a sequence's last unit turns the new k, quantises k and v, appends codes and scales to
 // the pool and patches its staged copy; every unit may be prefetched before the PDL wait.
+// Register cap from the CTAs per SM that shared memory admits (kCtasPerSm: three with one query
+// head per kv head at head_dim 128, two with two or four, one with eight): a tighter cap would
+// only cost registers, not add residency.
 template <int D, int P, int G, typename T, bool kFused = false>
-__global__ void __launch_bounds__(kDecodeThreads, 3) decode_i8_kernel(const DecodeParams p)
+__global__ void __launch_bounds__(kDecodeThreads, I8Shape<D, G>::kCtasPerSm) decode_i8_kernel(const DecodeParams p)
 {
     using S = I8Shape<D, G>;
     using Mma = MmaOps<__half>;

@@ -41,6 +41,7 @@ struct MmaShape {
     static constexpr int kWarpTotOffset = kCmbOffset + 2 * kCmbFloats * 4;
     static constexpr int kScanOffset = kWarpTotOffset + 64;
     static int smem_bytes(int batch) { return kScanOffset + 4 * (2 * batch + 1); }
+    static constexpr int kCtasPerSm = ctas_per_sm(kScanOffset + 4 * (2 * 64 + 1));
 };
 
 template <typename T> struct MmaOps;
@@ -96,8 +97,10 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x)
     return y;
 }
 
+// Register cap from the CTAs per SM that shared memory admits (kCtasPerSm: two with two or four
+// query heads per kv head at head_dim 128, one with eight).
 template <int D, int P, int G, typename T>
-__global__ void __launch_bounds__(kDecodeThreads, 3) decode_pass1_mma_kernel(const DecodeParams p)
+__global__ void __launch_bounds__(kDecodeThreads, MmaShape<D, G>::kCtasPerSm) decode_pass1_mma_kernel(const DecodeParams p)
 {
     using S = MmaShape<D, G>;
     constexpr int NW = kDecodeWarps;
