@@ -317,8 +317,10 @@ __device__ __forceinline__ void segment_epilogue(const DecodeParams& p, const fl
 // new token at position L - 1) turns the new k, writes k and v into the pool (the append)
 // and into its staged copy of the page.  No other kernel writes the pool meanwhile, so every
 // page may be prefetched before the PDL wait.
+// Register cap: 128 for the attention kernel alone (three of its CTAs and a RoPE/append CTA fit
+// on one SM); the fused layer has no such neighbour and takes the cap of three CTAs per SM.
 template <int D, int P, int G, typename T, bool kFused = false>
-__global__ void __launch_bounds__(kDecodeThreads, G == 1 ? 4 : 1) decode_pass1_kernel(const DecodeParams p)
+__global__ void __launch_bounds__(kDecodeThreads, G == 1 ? (kFused ? 3 : 4) : 1) decode_pass1_kernel(const DecodeParams p)
 {
     using S = DecodeShape<D, P, G, kFused>;
     constexpr int NW = kDecodeWarps;
