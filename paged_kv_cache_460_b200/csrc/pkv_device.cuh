@@ -1,5 +1,6 @@
 // Device-side building blocks for sm_100a: shared-memory barriers with bounded
-// waits, 1-D bulk (TMA) copies, programmatic dependent launch, element types.
+// waits, asynchronous copies and L2 prefetches, programmatic dependent launch,
+// element types.
 #ifndef PKV_DEVICE_CUH_
 #define PKV_DEVICE_CUH_
 
@@ -125,27 +126,6 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     }
 }
 
-// 1-D bulk copy global -> shared through the TMA unit; completion is counted in
-// bytes on `bar`.  Addresses 16-byte aligned, size a multiple of 16.  The KV
-// stream is read exactly once, so it is marked evict-first in L2.
-__device__ __forceinline__ void bulk_load_evict_first(void* dst, const void* src, uint32_t bytes,
-                                                      uint64_t* bar, uint64_t policy)
-{
-    asm volatile(
-        "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
-            smem_addr(dst)),
-        "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(policy)
-        : "memory");
-}
-
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar)
-{
-    asm volatile("cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                     smem_addr(dst)),
-                 "l"(src), "r"(bytes), "r"(smem_addr(bar))
-                 : "memory");
-}
-
 // 16-byte asynchronous global -> shared copy (cp.async, cached in L2 only).
 __device__ __forceinline__ void cp_async16(void* dst, const void* src)
 {
@@ -170,13 +150,6 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 // Wait until at most N of this thread's committed cp.async groups are still in flight.
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-
-__device__ __forceinline__ uint64_t l2_policy_evict_first()
-{
-    uint64_t pol;
-    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
-    return pol;
-}
 
 // Programmatic dependent launch: wait for the preceding kernel of the stream to
 // finish (and its writes to be visible); allow the next kernel to start its prologue.
