@@ -485,6 +485,7 @@ def run_ours(args):
             "e2e": e2e,
             "gpu_launches": args.steps * steps[0].kernels_per_step * world,
             "num_splits": args.splits or pkv.pkv_decode_auto_splits(pool, s.batch, s.max_pages, s.q_heads),
+            "cluster": 0 if args.splits else pkv.pkv_decode_cluster_size(pool, s.batch, s.max_pages, s.q_heads),
             "launch": "one CUDA graph per step (%d kernels%s)" % (
                 steps[0].kernels_per_step, ": an angle table, then one fused kernel per layer" if fused else ""),
             "clocks": clk,

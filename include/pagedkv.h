@@ -264,6 +264,19 @@ int pkv_decode_auto_splits(const pkv_pool* pool, int batch, int max_pages_per_se
                            int* num_splits_out);
 
 /*
+ * Whether num_splits = 0 runs the cluster variant on this pool and shape, and its cluster
+ * size: *cluster_out = C >= 2, or 0 for the partitioned kernel.  The cluster variant serves
+ * 16-bit pools with one query head per kv head when batch x kv_heads is at most half of
+ * pkv_decode_default_splits: one thread-block cluster of C = min(8, default_splits /
+ * (batch x kv_heads), max_pages_per_seq) CTAs per (sequence, kv head), each CTA taking an
+ * equal share of that pair's pages, the shares merged through distributed shared memory
+ * (no workspace is touched).  Needs a CUDA device (PKV_ERR_CUDA without one); INVALID_ARG /
+ * UNSUPPORTED as for paged_decode_attention.
+ */
+int pkv_decode_cluster_size(const pkv_pool* pool, int batch, int max_pages_per_seq, int q_heads, int kv_heads,
+                            int* cluster_out);
+
+/*
  * Workspace bytes paged_decode_attention needs for `num_splits` (1 .. PKV_MAX_DECODE_SPLITS)
  * partitions: a fixed region of PKV_MAX_DECODE_SPLITS int32 counters (16 KiB), then per
  * partition two fp32 partial results (running max, sum and the unnormalised output of every
@@ -290,7 +303,8 @@ size_t pkv_decode_workspace_size(int batch, int q_heads, int kv_heads, int head_
  *   kv_heads must equal the pool's; q_heads a multiple of it with q_heads / kv_heads in
  *   {1, 2, 4, 8}.
  *   num_splits: number of work partitions, at most PKV_MAX_DECODE_SPLITS
- *           (0 = pkv_decode_auto_splits for this shape).  The batch's
+ *           (0 = pkv_decode_auto_splits for this shape, or the cluster variant where
+ *           pkv_decode_cluster_size gives one).  The batch's
  *           pages x kv heads are laid end to end and cut into num_splits equal ranges, one
  *           per CTA; a (sequence, kv head) cut by a range boundary is finished by the CTA
  *           that delivers its last partial, which rescales the partial softmax sums

@@ -26,6 +26,7 @@ __all__ = [
     "KVPool", "rope_apply", "paged_kv_append", "rope_append", "rope_append_step", "paged_decode_attention", "rope_table",
     "paged_decode_layer", "paged_prefill_attention", "rms_norm", "pkv_slot_mapping",
     "pkv_kv_cache_bytes", "pkv_decode_workspace_size", "pkv_decode_default_splits", "pkv_decode_auto_splits",
+    "pkv_decode_cluster_size",
     "kv_get_device_error", "DecodeWorkspace", "PagedKVError", "PKV_F16", "PKV_BF16", "PKV_I8",
     "PKV_DEVERR_BAD_PAGE", "PKV_DEVERR_BAD_SLOT", "PKV_DEVERR_TIMEOUT", "PKV_MAX_DECODE_SPLITS",
 ]
@@ -169,6 +170,16 @@ def pkv_decode_auto_splits(pool, batch, max_pages_per_seq, q_heads, kv_heads=Non
     _lib.check("pkv_decode_auto_splits",
                lib().pkv_decode_auto_splits(pool.handle, batch, max_pages_per_seq, q_heads,
                                             pool.kv_heads if kv_heads is None else kv_heads, ctypes.byref(n)))
+    return n.value
+
+
+def pkv_decode_cluster_size(pool, batch, max_pages_per_seq, q_heads, kv_heads=None):
+    """Cluster size of the cluster variant that num_splits = 0 runs on this pool and shape
+    (0: the partitioned kernel)."""
+    n = ctypes.c_int()
+    _lib.check("pkv_decode_cluster_size",
+               lib().pkv_decode_cluster_size(pool.handle, batch, max_pages_per_seq, q_heads,
+                                             pool.kv_heads if kv_heads is None else kv_heads, ctypes.byref(n)))
     return n.value
 
 

@@ -47,6 +47,7 @@ SIGNATURES = {
     "paged_prefill_attention": (_I, [_P, _I, _P, _P, _P, _I, _P, _I, _P, _I, _I, _I, _F, _P]),
     "pkv_decode_default_splits": (_I, [_I, _I, _I, _I, _I, ctypes.POINTER(_I)]),
     "pkv_decode_auto_splits": (_I, [_P, _I, _I, _I, _I, ctypes.POINTER(_I)]),
+    "pkv_decode_cluster_size": (_I, [_P, _I, _I, _I, _I, ctypes.POINTER(_I)]),
     "pkv_decode_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
     "pkv_decode_workspace_clear": (_I, [_P, _SZ, _P]),
     "rope_table": (_I, [_P, _I, _I, _D, _P, _P]),

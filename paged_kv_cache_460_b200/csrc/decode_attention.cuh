@@ -71,6 +71,7 @@ struct DecodeParams {
     int kv_heads;
     int num_pages;
     int num_splits;
+    int cluster;                // cluster variant: CTAs per (sequence, kv head) cluster
     float scale_log2;           // scale * log2(e)
 };
 
@@ -88,7 +89,10 @@ __host__ __device__ constexpr int ctas_per_sm(int smem)
 // range (kNewRows rows of D elements), so that turning q at a segment's start and the append
 // at a sequence's end read shared memory instead of waiting on global loads; the ids of those
 // rows follow (kFusedIds ints).
-template <int D, int P, int G, bool kFused = false>
+// kCluster: the cluster variant also keeps the CTA's combined state of its piece of the
+// segment ([G][D + 2] floats: o, m, l), which the cluster's first CTA reads through
+// distributed shared memory.
+template <int D, int P, int G, bool kFused = false, bool kCluster = false>
 struct DecodeShape {
     static constexpr int kChunk = P * D * 2;                 // bytes of one (page, head)
     static constexpr int kQBytes = G * D * 2;
@@ -105,7 +109,8 @@ struct DecodeShape {
     static constexpr int kNewOffset = kRopeOffset + kRopeRows * D * 8;      // [2][k, v][D] of T
     static constexpr int kNewRows = kFused ? 4 : 0;
     static constexpr int kIdsOffset = kNewOffset + kNewRows * D * 2;        // rope b[2], append (b*Hkv+g)[2]
-    static constexpr int kScanOffset = kIdsOffset + (kFused ? 16 : 0);
+    static constexpr int kPartOffset = kIdsOffset + (kFused ? 16 : 0);     // [G][D + 2] floats (kCluster)
+    static constexpr int kScanOffset = kPartOffset + (kCluster ? G * (D + 2) * 4 : 0);
     // prefix[batch+1] and lens[batch] follow
     static int smem_bytes(int batch) { return kScanOffset + 4 * (2 * batch + 1); }
 };
@@ -226,10 +231,12 @@ __device__ __forceinline__ void prefetch_epilogue_lines(const DecodeParams& p, l
 // thread publishes the CTA's writes with a gpu-scope release fence (cumulative over the
 // barrier) and the merging CTA, after an acquire fence, reads the other partials through
 // L2, then resets the counter.
-template <int D, int G, typename T>
+// kCluster: a cut segment's combined state goes to `cpart` ([G][D + 2] in this CTA's shared
+// memory) for the cluster's merge (cluster_merge) instead of the workspace.
+template <int D, int G, typename T, bool kCluster = false>
 __device__ __forceinline__ void segment_epilogue(const DecodeParams& p, const float* buf, int b, int g, int np,
                                                  const int* prefix, long long r0, long long r1, long long chunk,
-                                                 volatile int* last_flag)
+                                                 volatile int* last_flag, float* cpart = nullptr)
 {
     constexpr int NW = kDecodeWarps;
     const int tid = threadIdx.x;
@@ -253,6 +260,12 @@ __device__ __forceinline__ void segment_epilogue(const DecodeParams& p, const fl
         if (complete) {
             T* dst = static_cast<T*>(p.out) + ((long long)b * p.q_heads + (long long)g * G + gi) * D + dd;
             *dst = Elt<T>::from_float(num / den);
+        } else if constexpr (kCluster) {
+            cpart[gi * (D + 2) + dd] = num;
+            if (dd == 0) {
+                cpart[gi * (D + 2) + D] = M;
+                cpart[gi * (D + 2) + D + 1] = den;
+            }
         } else {
             p.part_o[((long long)pslot * G + gi) * D + dd] = num;
             if (dd == 0) {
@@ -261,7 +274,7 @@ __device__ __forceinline__ void segment_epilogue(const DecodeParams& p, const fl
             }
         }
     }
-    if (!complete) {
+    if (!kCluster && !complete) {
         // Deliver this partial; the CTA that delivers the last one merges the segment.
         // One thread publishes the CTA's writes (a gpu-scope release fence is cumulative
         // over the barrier) and counts them in; the merging CTA reads the other partials
@@ -310,6 +323,51 @@ __device__ __forceinline__ void segment_epilogue(const DecodeParams& p, const fl
     }
 }
 
+// Thread-block cluster helpers (sm_90+): a barrier over all threads of the cluster with
+// release/acquire semantics, and loads from another CTA's shared memory.
+__device__ __forceinline__ void cluster_sync_all()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ float ld_dsmem_f32(const float* local, uint32_t rank)
+{
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_addr(local)), "r"(rank));
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+    return v;
+}
+
+// The cluster variant's merge, after every CTA of the cluster has stored its piece's state in
+// `cpart` (empty pieces: m = -inf, l = 0): the cluster's first CTA combines the C states,
+// M = max m_k, out = sum_k 2^(m_k - M) o_k / sum_k 2^(m_k - M) l_k, and writes the output;
+// every CTA then waits for it, so that no CTA leaves while its state is still being read.
+template <int D, int G, typename T>
+__device__ __forceinline__ void cluster_merge(const DecodeParams& p, const float* cpart, int b, int g, bool cut,
+                                              int rank, int C)
+{
+    cluster_sync_all();
+    if (rank == 0 && cut) {
+        for (int idx = threadIdx.x; idx < G * D; idx += kDecodeThreads) {
+            const int gi = idx / D, dd = idx - gi * D;
+            float M = -INFINITY;
+            for (int r = 0; r < C; ++r) M = fmaxf(M, ld_dsmem_f32(cpart + gi * (D + 2) + D, r));
+            float num = 0.f, den = 0.f;
+            for (int r = 0; r < C; ++r) {
+                const float m = ld_dsmem_f32(cpart + gi * (D + 2) + D, r);
+                if (m == -INFINITY) continue;                     // an empty piece
+                const float w = fast_exp2(m - M);
+                num = fmaf(w, ld_dsmem_f32(cpart + gi * (D + 2) + dd, r), num);
+                den = fmaf(w, ld_dsmem_f32(cpart + gi * (D + 2) + D + 1, r), den);
+            }
+            T* dst = static_cast<T*>(p.out) + ((long long)b * p.q_heads + (long long)g * G + gi) * D + dd;
+            *dst = Elt<T>::from_float(num / den);
+        }
+    }
+    cluster_sync_all();
+}
+
 // kFused: the whole decode layer in one kernel ("为什么要自己动手写一个LLM推理引擎"
 // (wzjinhao.cn/news/61427) s4.3 rotate q and k, append k and v, attend; s5.3 fuse small
 // kernels).  q arrives unturned and each warp turns its segment's q rows in shared memory
@@ -319,10 +377,15 @@ __device__ __forceinline__ void segment_epilogue(const DecodeParams& p, const fl
 // page may be prefetched before the PDL wait.
 // Register cap: 128 for the attention kernel alone (three of its CTAs and a RoPE/append CTA fit
 // on one SM); the fused layer has no such neighbour and takes the cap of three CTAs per SM.
-template <int D, int P, int G, typename T, bool kFused = false>
+//
+// kCluster: one cluster of p.cluster CTAs per (sequence, kv head) -- for batches whose
+// (sequence, kv head) pairs are too few to fill the GPU -- each CTA taking an equal share
+// of its pages; the pieces are merged through distributed shared memory (cluster_merge)
+// instead of the workspace, so no CTA waits on global fences, atomics or loads at its end.
+template <int D, int P, int G, typename T, bool kFused = false, bool kCluster = false>
 __global__ void __launch_bounds__(kDecodeThreads, G == 1 ? (kFused ? 3 : 4) : 1) decode_pass1_kernel(const DecodeParams p)
 {
-    using S = DecodeShape<D, P, G, kFused>;
+    using S = DecodeShape<D, P, G, kFused, kCluster>;
     constexpr int NW = kDecodeWarps;
     constexpr int DEPTH = S::kDepth;
     constexpr int CPR = D / 8;            // 16-byte chunks per K/V row
@@ -354,8 +417,23 @@ __global__ void __launch_bounds__(kDecodeThreads, G == 1 ? (kFused ? 3 : 4) : 1)
     const int Hkv = p.kv_heads;
     const long long W = (long long)Hkv * prefix[p.batch];
     const long long chunk = W > 0 ? (W + p.num_splits - 1) / p.num_splits : 1;
-    const long long r0 = (long long)blockIdx.x * chunk;
-    const long long r1 = min(W, r0 + chunk);
+    long long r0 = (long long)blockIdx.x * chunk;
+    long long r1 = min(W, r0 + chunk);
+    // cluster variant: this CTA's share of its cluster's (sequence, kv head)
+    const int c_rank = kCluster ? (int)(blockIdx.x % p.cluster) : 0;
+    const int c_b = kCluster ? (int)(blockIdx.x / p.cluster) / Hkv : 0;
+    const int c_g = kCluster ? (int)(blockIdx.x / p.cluster) % Hkv : 0;
+    const int c_np = kCluster ? prefix[c_b + 1] - prefix[c_b] : 0;
+    float* cpart = reinterpret_cast<float*>(smem + S::kPartOffset);
+    if constexpr (kCluster) {
+        const long long seg0 = (long long)Hkv * prefix[c_b] + (long long)c_g * c_np;
+        r0 = seg0 + (long long)c_rank * c_np / p.cluster;
+        r1 = seg0 + (long long)(c_rank + 1) * c_np / p.cluster;
+        for (int i = tid; i < G; i += kDecodeThreads) {      // an empty piece's state
+            cpart[i * (D + 2) + D] = -INFINITY;
+            cpart[i * (D + 2) + D + 1] = 0.f;
+        }
+    }
     const long long n_mine = r1 - r0 > warp ? (r1 - r0 - warp + NW - 1) / NW : 0;   // this warp's pages
 
     // lane l holds the page id of this warp's page win0 + l (-1: outside the table)
@@ -474,7 +552,7 @@ __global__ void __launch_bounds__(kDecodeThreads, G == 1 ? (kFused ? 3 : 4) : 1)
     // page holding a sequence's newest token (a fused layer before this kernel may still
     // be writing it) and the q rows (the kernel before may still be producing them).
     if (n_mine > 0) prefetch_q_rows<D, G, T>(p, ib, ig, lane);     // this warp's first segment
-    if (r0 < r1) prefetch_epilogue_lines<D, G>(p, r0, chunk, prefix, tid);
+    if (!kCluster && r0 < r1) prefetch_epilogue_lines<D, G>(p, r0, chunk, prefix, tid);
     if constexpr (kFused) {                   // the new k, v rows of the kept sequence ends
         constexpr int kRowLines = (D * (int)sizeof(T) + 127) / 128;
         if (warp == 0 && lane < 4 * kRowLines && fids[2 + lane / (2 * kRowLines)] >= 0) {
@@ -506,7 +584,7 @@ __global__ void __launch_bounds__(kDecodeThreads, G == 1 ? (kFused ? 3 : 4) : 1)
         T* row = static_cast<T*>(p.out) + (long long)b * p.q_heads * D;
         for (int idx = tid; idx < p.q_heads * D; idx += blockDim.x) row[idx] = Elt<T>::from_float(0.f);
     }
-    if (r0 >= r1) return;
+    if (!kCluster && r0 >= r1) return;       // (a cluster's CTAs all reach its merge)
 
     unsigned char* ring = smem + ring_off;
     float* pbuf = pbuf_all + warp * G * P;
@@ -545,9 +623,11 @@ __global__ void __launch_bounds__(kDecodeThreads, G == 1 ? (kFused ? 3 : 4) : 1)
         for (int e = 0; e < EPL; ++e) o[gi][e] = 0.f;
     }
     long long kc = 0;                         // this warp's pages consumed
-    int b, g, j;
-    locate_unit(r0, prefix, p.batch, Hkv, b, g, j);
-    int np = prefix[b + 1] - prefix[b];
+    int b = 0, g = 0, j = 0, np = 1;
+    if (r0 < r1) {
+        locate_unit(r0, prefix, p.batch, Hkv, b, g, j);
+        np = prefix[b + 1] - prefix[b];
+    }
     int seg = 0;
     // One pass per segment (the range's part of one (sequence, kv head)): this warp's
     // pages of it, then the combine of all warps.
@@ -715,7 +795,7 @@ __global__ void __launch_bounds__(kDecodeThreads, G == 1 ? (kFused ? 3 : 4) : 1)
 #pragma unroll
             for (int e = 0; e < EPL; ++e) o[gi][e] = 0.f;
         }
-        segment_epilogue<D, G, T>(p, buf, b, g, np, prefix, r0, r1, chunk, last_flag);
+        segment_epilogue<D, G, T, kCluster>(p, buf, b, g, np, prefix, r0, r1, chunk, last_flag, cpart);
         // next segment: the next kv head of this sequence, or the next non-empty sequence
         u = u_end;
         j = 0;
@@ -728,6 +808,7 @@ __global__ void __launch_bounds__(kDecodeThreads, G == 1 ? (kFused ? 3 : 4) : 1)
         }
     }
     cp_async_wait<0>();
+    if constexpr (kCluster) cluster_merge<D, G, T>(p, cpart, c_b, c_g, c_np >= 2, c_rank, p.cluster);
 }
 
 }  // namespace pkv

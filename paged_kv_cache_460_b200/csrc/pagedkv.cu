@@ -44,6 +44,29 @@ cudaError_t launch_pdl(Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaSt
 
 int status_of(cudaError_t e) { return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA; }
 
+// As launch_pdl, in thread-block clusters of `cluster` CTAs along x.
+template <typename Kernel, typename... Args>
+cudaError_t launch_pdl_cluster(Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream, int cluster,
+                               Args... args)
+{
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = cluster;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 constexpr int kMaxDevices = 64;
 
 // Raise a kernel's dynamic shared-memory limit once per device (and size).
@@ -179,6 +202,49 @@ bool pick_decode(int head_dim, int page_size, int group, int dtype, int storage,
         return i8 ? pick_shape<__nv_bfloat16, true>(head_dim, page_size, group, ops)
                   : pick_shape<__nv_bfloat16, false>(head_dim, page_size, group, ops);
     return false;
+}
+
+// The cluster variant of the CUDA-core kernel (16-bit pages, one query head per kv head):
+// one cluster of C CTAs per (sequence, kv head), used for num_splits = 0 when the batch's
+// (sequence, kv head) pairs number at most half the full wave; C = min(8, wave / pairs,
+// max_pages_per_seq), at least 2.  0 when the variant does not apply.
+int cluster_size(int full_wave, int batch, int kv_heads, int max_pages)
+{
+    const long long pairs = (long long)batch * kv_heads;
+    if (pairs <= 0 || 2 * pairs > full_wave) return 0;
+    int c = (int)(full_wave / pairs);
+    c = c < 8 ? c : 8;
+    c = c < max_pages ? c : max_pages;
+    return c >= 2 ? c : 0;
+}
+
+template <int D, int P, typename T, bool kFused>
+int launch_cluster(const DecodeParams& prm, cudaStream_t st)
+{
+    static int configured[kMaxDevices] = {0};
+    constexpr auto fn = decode_pass1_kernel<D, P, 1, T, kFused, true>;
+    const int smem = DecodeShape<D, P, 1, kFused, true>::smem_bytes(prm.batch);
+    if (smem > kMaxSmemPerCta) return PKV_ERR_UNSUPPORTED;
+    if (ensure_smem(fn, smem, configured) != cudaSuccess) return PKV_ERR_CUDA;
+    const int grid = prm.batch * prm.kv_heads * prm.cluster;
+    return status_of(launch_pdl_cluster(fn, dim3(grid), dim3(kDecodeThreads), smem, st, prm.cluster, prm));
+}
+
+template <typename T, bool kFused>
+int cluster_shape(int head_dim, int page_size, const DecodeParams& prm, cudaStream_t st)
+{
+    if (head_dim == 128 && page_size == 16) return launch_cluster<128, 16, T, kFused>(prm, st);
+    if (head_dim == 128 && page_size == 32) return launch_cluster<128, 32, T, kFused>(prm, st);
+    if (head_dim == 64 && page_size == 16) return launch_cluster<64, 16, T, kFused>(prm, st);
+    if (head_dim == 64 && page_size == 32) return launch_cluster<64, 32, T, kFused>(prm, st);
+    return PKV_ERR_UNSUPPORTED;
+}
+
+template <bool kFused>
+int launch_cluster_variant(const pkv_pool* pool, const DecodeParams& prm, cudaStream_t st)
+{
+    if (pool->dtype == PKV_F16) return cluster_shape<__half, kFused>(pool->head_dim, pool->page_size, prm, st);
+    return cluster_shape<__nv_bfloat16, kFused>(pool->head_dim, pool->page_size, prm, st);
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -382,6 +448,23 @@ extern "C" int pkv_decode_auto_splits(const pkv_pool* pool, int batch, int max_p
     return PKV_OK;
 }
 
+extern "C" int pkv_decode_cluster_size(const pkv_pool* pool, int batch, int max_pages_per_seq, int q_heads,
+                                       int kv_heads, int* cluster_out)
+{
+    if (!pool || !cluster_out || batch < 0 || max_pages_per_seq <= 0 || q_heads <= 0 || kv_heads != pool->kv_heads ||
+        q_heads % kv_heads)
+        return PKV_ERR_INVALID_ARG;
+    DecodeOps ops;
+    if (!pick_decode(pool->head_dim, pool->page_size, q_heads / kv_heads, pool->dtype, pool->storage, ops))
+        return PKV_ERR_UNSUPPORTED;
+    int full = 0;
+    const int st = ops.splits(&full);
+    if (st != PKV_OK) return st;
+    *cluster_out = (pool->storage != kStorageI8 && ops.group == 1)
+                       ? cluster_size(full, batch, kv_heads, max_pages_per_seq) : 0;
+    return PKV_OK;
+}
+
 extern "C" size_t pkv_decode_workspace_size(int batch, int q_heads, int kv_heads, int head_dim, int num_splits)
 {
     if (batch < 0 || q_heads <= 0 || kv_heads <= 0 || q_heads % kv_heads || head_dim <= 0 || num_splits <= 0 ||
@@ -406,15 +489,19 @@ extern "C" int paged_decode_attention(const pkv_pool* pool, int layer, void* out
     DecodeOps ops;
     if (!pick_decode(pool->head_dim, pool->page_size, q_heads / kv_heads, pool->dtype, pool->storage, ops))
         return PKV_ERR_UNSUPPORTED;
+    int cluster = 0;
     if (num_splits == 0) {
         const int st = ops.splits(&num_splits);
         if (st != PKV_OK) return st;
+        if (pool->storage != kStorageI8 && ops.group == 1)
+            cluster = cluster_size(num_splits, batch, kv_heads, max_pages_per_seq);
         num_splits = auto_splits(num_splits, max_decode_units(kv_heads, batch, max_pages_per_seq, pool->page_size,
                                                               ops.unit_tokens));
     }
     const WorkspaceLayout wl = workspace_layout(batch, ops.group, pool->head_dim, num_splits);
     if (workspace_bytes < wl.total) return PKV_ERR_NO_SPACE;
     DecodeParams prm;
+    prm.cluster = cluster;
     prm.k = static_cast<const char*>(pool->k_base) + (size_t)layer * pool->layer_bytes();
     prm.v = static_cast<const char*>(pool->v_base) + (size_t)layer * pool->layer_bytes();
     prm.k_scale = nullptr;
@@ -438,6 +525,7 @@ extern "C" int paged_decode_attention(const pkv_pool* pool, int layer, void* out
     prm.num_pages = pool->num_pages;
     prm.num_splits = num_splits;
     prm.scale_log2 = scale * 1.4426950408889634f;
+    if (cluster) return launch_cluster_variant<false>(pool, prm, reinterpret_cast<cudaStream_t>(stream));
     return ops.launch(prm, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -525,9 +613,11 @@ extern "C" int paged_decode_layer(const pkv_pool* pool, int layer, void* out, co
     DecodeOps ops;
     if (!pick_decode(pool->head_dim, pool->page_size, group, pool->dtype, pool->storage, ops))
         return PKV_ERR_UNSUPPORTED;
+    int cluster = 0;
     if (num_splits == 0) {
         const int st = ops.splits(&num_splits);
         if (st != PKV_OK) return st;
+        if (!i8) cluster = cluster_size(num_splits, batch, kv_heads, max_pages_per_seq);
         num_splits = auto_splits(num_splits, max_decode_units(kv_heads, batch, max_pages_per_seq, pool->page_size,
                                                               ops.unit_tokens));
     }
@@ -559,7 +649,9 @@ extern "C" int paged_decode_layer(const pkv_pool* pool, int layer, void* out, co
     prm.num_pages = pool->num_pages;
     prm.num_splits = num_splits;
     prm.scale_log2 = scale * 1.4426950408889634f;
+    prm.cluster = cluster;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (cluster) return launch_cluster_variant<true>(pool, prm, st);
     if (pool->dtype == PKV_F16) return fused_shape<__half>(pool->head_dim, pool->page_size, group, i8, prm, st);
     return fused_shape<__nv_bfloat16>(pool->head_dim, pool->page_size, group, i8, prm, st);
 }

@@ -259,19 +259,22 @@ def test_rms_norm_matches_oracle(dtype, rows, hidden, fused):
 
 def test_automatic_split_count_follows_the_work_bound():
     """num_splits = 0 takes a full wave of CTAs unless the work bound (kv heads x batch x units
-    of the table's pages) would leave a CTA fewer than 16 units; the automatic call gives the
-    bits of the explicit call with that count."""
+    of the table's pages) would leave a CTA fewer than 16 units; where the cluster variant does
+    not apply, the automatic call gives the bits of the explicit call with that count."""
     full = pkv.pkv_decode_default_splits(32, 32, 128, 16, pkv.PKV_F16)
-    s = synth.random_spec(610, 1, 32, 32, 128, 16, [2048])       # one 2049-token sequence, 32 heads
+    s = synth.random_spec(610, 8, 32, 32, 128, 16, [20] * 8)    # 256 short (sequence, head) pairs
     c = Case(s)
+    assert pkv.pkv_decode_cluster_size(c.pool, s.batch, s.max_pages, s.q_heads) == 0
     auto = pkv.pkv_decode_auto_splits(c.pool, s.batch, s.max_pages, s.q_heads)
-    assert auto == min(full, -(-(32 * 1 * s.max_pages) // 16))
+    assert auto == min(full, -(-(32 * s.batch * s.max_pages) // 16)) and auto < full
     out_auto = c.gpu_layer(0)
     q = c.last_q
     out_expl = torch.empty_like(q)
     pkv.paged_decode_attention(c.pool, 0, out_expl, q, c.bt_t, c.cl_t, c.scale, num_splits=auto)
     assert np.array_equal(to_bits(out_auto), to_bits(out_expl))
     _expect_close(out_auto, c.oracle_layer(0), "f16", "automatic splits")
+    one = Case(synth.random_spec(611, 1, 32, 32, 128, 16, [2048]))   # the single long sequence
+    assert pkv.pkv_decode_auto_splits(one.pool, 1, one.s.max_pages, 32) == min(full, -(-(32 * one.s.max_pages) // 16))
     big = synth.spec("batch10", num_layers=1)
     assert pkv.pkv_decode_auto_splits(pkv.KVPool(*synth.pool_values_torch(big, "cuda")), big.batch, big.max_pages,
                                       big.q_heads) == full

@@ -37,7 +37,8 @@ def short_wait_lib(tmp_path_factory):
         path = str(tmp_path_factory.mktemp("shortwait") / "libpagedkv_shortwait.so")
         pkv_build.build(out=path, defines=SHORT_WAIT_DEFINES)
     h = ctypes.CDLL(path)                       # its own symbols, kernels and error word
-    for name, (res, args) in _lib.SIGNATURES.items():
+    for name in ("kv_get_device_error", "kv_pool_create", "kv_pool_destroy", "paged_prefill_attention"):
+        res, args = _lib.SIGNATURES[name]
         fn = getattr(h, name)
         fn.restype = res
         fn.argtypes = args
