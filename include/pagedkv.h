@@ -93,8 +93,10 @@ const char* pkv_status_string(int status);
  *                   here.
  *   page_size: 16 or 32 tokens; head_dim: 64 or 128; dtype: PKV_F16 or PKV_BF16.
  * The free list starts with every page id 0..num_pages-1, handed out in increasing order.
- * Errors: INVALID_ARG for null/non-positive/misaligned arguments, UNSUPPORTED for other
- * page sizes, head dims or dtypes.
+ * Errors: INVALID_ARG for null/non-positive/misaligned arguments, and for a pool with
+ * num_pages * kv_heads * page_size / 16 above 2^31 - 1 (the kernels index 16-token blocks
+ * of a layer with 32-bit integers; such a layer would hold terabytes), UNSUPPORTED for
+ * other page sizes, head dims or dtypes.
  */
 int kv_pool_create(int num_layers, int num_pages, int page_size, int kv_heads, int head_dim,
                    int dtype, void* k_base, void* v_base, pkv_pool** out);
@@ -112,8 +114,8 @@ int kv_pool_create(int num_layers, int num_pages, int page_size, int kv_heads, i
  *   all four 16-byte aligned and caller-owned, as for kv_pool_create.
  *   dtype: PKV_F16 or PKV_BF16, the type of q, k, v and the output of the calls on this pool.
  * paged_kv_append and rope_append quantise the new rows as they write them;
- * paged_decode_attention reads k = c * s, v = c * s (every q_heads / kv_heads in {1, 2, 4, 8}
- * on the CUDA cores); paged_prefill_attention returns UNSUPPORTED on such a pool.
+ * paged_decode_attention reads k = c * s, v = c * s (every q_heads / kv_heads in {1, 2, 4, 8},
+ * on the tensor cores); paged_prefill_attention returns UNSUPPORTED on such a pool.
  * Errors as for kv_pool_create.
  */
 int kv_pool_create_i8(int num_layers, int num_pages, int page_size, int kv_heads, int head_dim,

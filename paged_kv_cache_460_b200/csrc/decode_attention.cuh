@@ -436,14 +436,16 @@ __global__ void __launch_bounds__(kDecodeThreads, G == 1 ? (kFused ? 3 : 4) : 1)
     }
     const long long n_mine = r1 - r0 > warp ? (r1 - r0 - warp + NW - 1) / NW : 0;   // this warp's pages
 
-    // lane l holds the page id of this warp's page win0 + l (-1: outside the table)
+    // lane l holds the (page, kv head) chunk index page * Hkv + head of this warp's page
+    // win0 + l; -1 for a page outside the table or the pool
     auto load_window = [&](long long win0) {
         const long long k = win0 + lane;
-        int id = 0;
+        int id = -1;
         if (k < n_mine) {
             int bb, gg, jj;
             locate_unit(r0 + warp + k * NW, prefix, p.batch, Hkv, bb, gg, jj);
-            id = jj < p.max_pages ? p.block_tables[(long long)bb * p.max_pages + jj] : -1;
+            const int page = jj < p.max_pages ? p.block_tables[(long long)bb * p.max_pages + jj] : -1;
+            if ((unsigned)page < (unsigned)p.num_pages) id = page * Hkv + gg;
         }
         return id;
     };
@@ -465,10 +467,10 @@ __global__ void __launch_bounds__(kDecodeThreads, G == 1 ? (kFused ? 3 : 4) : 1)
             win0 = k;
             win = load_window(k);
         }
-        const int page = __shfl_sync(0xffffffffu, win, (int)(k - win0));
+        const int ph = __shfl_sync(0xffffffffu, win, (int)(k - win0));
         unsigned char* slot = smem + ring_off + (int)(k % DEPTH) * S::kSlot;
-        if ((unsigned)page < (unsigned)p.num_pages) {
-            const long long off = ((long long)page * Hkv + ig) * (P * D);
+        if (ph >= 0) {
+            const long long off = (long long)ph * (P * D);
             const unsigned char* ks = reinterpret_cast<const unsigned char*>(static_cast<const T*>(p.k) + off);
             const unsigned char* vs = reinterpret_cast<const unsigned char*>(static_cast<const T*>(p.v) + off);
 #pragma unroll

@@ -159,8 +159,9 @@ __global__ void __launch_bounds__(kDecodeThreads, I8Shape<D, G>::kCtasPerSm) dec
     const long long r1 = min(W, r0 + chunk);
     const int n_mine = r1 - r0 > warp ? (int)((r1 - r0 - warp + NW - 1) / NW) : 0;
 
-    // lane l holds the id of page l % PPU of this warp's unit win0 + l / PPU: -1 when the
-    // page table has no such entry, -2 when the unit's tokens end before that page
+    // lane l holds, for page l % PPU of this warp's unit win0 + l / PPU, its (page, kv head)
+    // index page * Hkv + head: -1 when the page table has no such entry or it is outside
+    // the pool, -2 when the unit's tokens end before that page
     auto load_window = [&](int win0) {
         const int k = win0 + lane / PPU;
         int id = -2;
@@ -168,7 +169,10 @@ __global__ void __launch_bounds__(kDecodeThreads, I8Shape<D, G>::kCtasPerSm) dec
             int bb, gg, jj;
             locate_unit(r0 + warp + (long long)k * NW, prefix, p.batch, Hkv, bb, gg, jj);
             const int pg = jj * PPU + lane % PPU;
-            if (pg * P < lens[bb]) id = pg < p.max_pages ? p.block_tables[(long long)bb * p.max_pages + pg] : -1;
+            if (pg * P < lens[bb]) {
+                const int page = pg < p.max_pages ? p.block_tables[(long long)bb * p.max_pages + pg] : -1;
+                id = (unsigned)page < (unsigned)p.num_pages ? page * Hkv + gg : -1;
+            }
         }
         return id;
     };
@@ -191,10 +195,10 @@ __global__ void __launch_bounds__(kDecodeThreads, I8Shape<D, G>::kCtasPerSm) dec
         unsigned char* slot = ring + sl * S::kSlot;
 #pragma unroll
         for (int pp = 0; pp < PPU; ++pp) {
-            const int page = __shfl_sync(0xffffffffu, win, (k - win0) * PPU + pp);
-            if (page == -2) continue;                        // past the sequence's last token
-            if ((unsigned)page < (unsigned)p.num_pages) {
-                const long long row0 = ((long long)page * Hkv + ig) * P;       // first token row
+            const int ph = __shfl_sync(0xffffffffu, win, (k - win0) * PPU + pp);
+            if (ph == -2) continue;                          // past the sequence's last token
+            if (ph >= 0) {
+                const long long row0 = (long long)ph * P;   // first token row
                 const unsigned char* ks = static_cast<const unsigned char*>(p.k) + row0 * D;
                 const unsigned char* vs = static_cast<const unsigned char*>(p.v) + row0 * D;
 #pragma unroll

@@ -129,14 +129,18 @@ __global__ void __launch_bounds__(kDecodeThreads, MmaShape<D, G>::kCtasPerSm) de
     const long long r1 = min(W, r0 + chunk);
     const long long n_mine = r1 - r0 > warp ? (r1 - r0 - warp + NW - 1) / NW : 0;
 
+    // lane l holds the index of the 16-row chunk (page, kv head, half of a 32-token page)
+    // of this warp's unit win0 + l: (page * Hkv + head) * U + row block; -1 for a page
+    // outside the table or the pool
     auto load_window = [&](long long win0) {
         const long long k = win0 + lane;
-        int id = 0;
+        int id = -1;
         if (k < n_mine) {
             int bb, gg, jj;
             locate_unit(r0 + warp + k * NW, prefix, p.batch, Hkv, bb, gg, jj);
             const int pg = jj / U;
-            id = pg < p.max_pages ? p.block_tables[(long long)bb * p.max_pages + pg] : -1;
+            const int page = pg < p.max_pages ? p.block_tables[(long long)bb * p.max_pages + pg] : -1;
+            if ((unsigned)page < (unsigned)p.num_pages) id = (page * Hkv + gg) * U + jj % U;
         }
         return id;
     };
@@ -154,10 +158,10 @@ __global__ void __launch_bounds__(kDecodeThreads, MmaShape<D, G>::kCtasPerSm) de
             win0 = k;
             win = load_window(k);
         }
-        const int page = __shfl_sync(0xffffffffu, win, (int)(k - win0));
+        const int ci = __shfl_sync(0xffffffffu, win, (int)(k - win0));
         unsigned char* slot = smem + ring_off + (int)(k % DEPTH) * S::kSlot;
-        if ((unsigned)page < (unsigned)p.num_pages) {
-            const long long off = (((long long)page * Hkv + ig) * P + (ij % U) * 16) * D;
+        if (ci >= 0) {
+            const long long off = (long long)ci * (16 * D);
             const unsigned char* ks = reinterpret_cast<const unsigned char*>(static_cast<const T*>(p.k) + off);
             const unsigned char* vs = reinterpret_cast<const unsigned char*>(static_cast<const T*>(p.v) + off);
 #pragma unroll

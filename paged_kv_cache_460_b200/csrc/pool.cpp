@@ -40,6 +40,8 @@ int make_pool(int num_layers, int num_pages, int page_size, int kv_heads, int he
     if (page_size != 16 && page_size != 32) return PKV_ERR_UNSUPPORTED;
     if (head_dim != 64 && head_dim != 128) return PKV_ERR_UNSUPPORTED;
     if (dtype != PKV_F16 && dtype != PKV_BF16) return PKV_ERR_UNSUPPORTED;
+    // the kernels index the 16-row blocks of a layer's (page, kv head) chunks with 32-bit ints
+    if ((int64_t)num_pages * kv_heads * (page_size / 16) > INT32_MAX) return PKV_ERR_INVALID_ARG;
     pkv_pool* p = new (std::nothrow) pkv_pool;
     if (!p) return PKV_ERR_NO_SPACE;
     p->num_layers = num_layers;

@@ -73,6 +73,11 @@ def test_pool_create_validates(L):
     assert L.kv_pool_create(1, 8, 16, 2, 96, 0, _fake_ptr(), _fake_ptr(), ctypes.byref(h)) == _lib.PKV_ERR_UNSUPPORTED
     assert L.kv_pool_create(1, 8, 16, 2, 64, 7, _fake_ptr(), _fake_ptr(), ctypes.byref(h)) == _lib.PKV_ERR_UNSUPPORTED
     assert L.kv_pool_create(1, 8, 16, 2, 64, 0, _fake_ptr(), _fake_ptr(), None) == _lib.PKV_ERR_INVALID_ARG
+    # 16-token blocks of a layer past the kernels' 32-bit index: rejected before any allocation
+    assert L.kv_pool_create(1, 1 << 30, 32, 1, 64, 0, _fake_ptr(), _fake_ptr(), ctypes.byref(h)) == \
+        _lib.PKV_ERR_INVALID_ARG
+    assert L.kv_pool_create(1, 1 << 27, 16, 16, 64, 0, _fake_ptr(), _fake_ptr(), ctypes.byref(h)) == \
+        _lib.PKV_ERR_INVALID_ARG
 
 
 def test_free_list_properties(L):
