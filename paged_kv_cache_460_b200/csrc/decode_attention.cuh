@@ -49,6 +49,10 @@ constexpr int kRingBudgetBytes = 68 * 1024;
 // Partials loaded per merge round.  Eight per round measured slower on every workload: the
 // merge is inlined in the segment loop and its registers cost the hot loop spills.
 constexpr int kMaxMergeParts = 4;
+// Independent accumulators over which the tensor-core kernels spread the k-steps of q.K^T
+// (1, 2 and 4 measured within 1.5 % of one another; 2 was the best on the grouped-query and
+// the fused int8 workloads).
+constexpr int kScoreChains = 2;
 
 struct DecodeParams {
     const void* k;              // this layer's K pool  [pages][kv_heads][P][D]

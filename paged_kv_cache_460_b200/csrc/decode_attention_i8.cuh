@@ -407,11 +407,17 @@ __global__ void __launch_bounds__(kDecodeThreads, I8Shape<D, G>::kCtasPerSm) dec
             const float* ksc = reinterpret_cast<const float*>(s + 2 * S::kChunk);
             const float* vsc = reinterpret_cast<const float*>(s + 2 * S::kChunk + S::kScaleBytes);
             // ---- S^T = C_K . Q^T for the two 16-token tiles
-            float sacc[2][4];
+            // (each tile's k-steps spread over kScoreChains independent accumulators)
+            constexpr int SCH = KS < kScoreChains ? KS : kScoreChains;
+            float sacc_c[2][SCH][4];
+#pragma unroll
+            for (int tau = 0; tau < 2; ++tau)
+#pragma unroll
+                for (int c = 0; c < SCH; ++c)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) sacc_c[tau][c][e] = 0.f;
 #pragma unroll
             for (int tau = 0; tau < 2; ++tau) {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) sacc[tau][e] = 0.f;
 #pragma unroll
                 for (int x = 0; x < KS / 2; ++x) {
                     uint32_t r[4];
@@ -421,10 +427,19 @@ __global__ void __launch_bounds__(kDecodeThreads, I8Shape<D, G>::kCtasPerSm) dec
                         uint32_t a[4];
                         i8_lo_hi_biased(r[2 * h], a[0], a[2]);
                         i8_lo_hi_biased(r[2 * h + 1], a[1], a[3]);
-                        Mma::mma(sacc[tau], a, bq[2 * x + h][0], bq[2 * x + h][1]);
+                        Mma::mma(sacc_c[tau][(2 * x + h) % SCH], a, bq[2 * x + h][0], bq[2 * x + h][1]);
                     }
                 }
             }
+            float sacc[2][4];
+#pragma unroll
+            for (int tau = 0; tau < 2; ++tau)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    sacc[tau][e] = sacc_c[tau][0][e];
+#pragma unroll
+                    for (int c = 1; c < SCH; ++c) sacc[tau][e] += sacc_c[tau][c][e];
+                }
             // ---- scores of tokens 16 tau + g4 (+8), heads 2t4, 2t4+1; the unit's 2^E
             float sc[2][4], w[2][2];
             float smax = 0.f;

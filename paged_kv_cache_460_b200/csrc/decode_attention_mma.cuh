@@ -279,14 +279,27 @@ __global__ void __launch_bounds__(kDecodeThreads, MmaShape<D, G>::kCtasPerSm) de
                     reinterpret_cast<uint4*>(s + S::kChunk + nvalid * (2 * D))[x] = make_uint4(0, 0, 0, 0);
                 __syncwarp();
             }
-            // ---- S^T = K . Q^T
-            float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+            // ---- S^T = K . Q^T, the k-steps spread over kScoreChains independent accumulators
+            //      so that consecutive MMAs do not wait on one another
+            constexpr int SCH = KS < kScoreChains ? KS : kScoreChains;
+            float sacc_c[SCH][4];
+#pragma unroll
+            for (int c = 0; c < SCH; ++c)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) sacc_c[c][e] = 0.f;
 #pragma unroll
             for (int kk = 0; kk < KS; ++kk) {
                 uint32_t a[4];
                 const int ch = 2 * kk + k_chunk_hi;
                 ldmatrix_x4(a, s + k_row * (2 * D) + ((ch ^ (k_row & 7)) * 16));
-                MmaOps<T>::mma(sacc, a, bq[kk][0], bq[kk][1]);
+                MmaOps<T>::mma(sacc_c[kk % SCH], a, bq[kk][0], bq[kk][1]);
+            }
+            float sacc[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                sacc[e] = sacc_c[0][e];
+#pragma unroll
+                for (int c = 1; c < SCH; ++c) sacc[e] += sacc_c[c][e];
             }
             // ---- online softmax: sacc = (token g4, heads 2t4, 2t4+1), (token g4 + 8, same heads)
             float sc[4];
