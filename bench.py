@@ -424,7 +424,8 @@ def run_ours(args):
     attn_ms_mean = max_over_ranks(timed(lambda i: attn.replay()), world, dev) / (args.steps * L)
     clk = clocks.stop()
 
-    # ---- e2e through the public API: host buffers in and out, one DecodeStep per step
+    # ---- e2e through the public API: pinned host buffers in and out, one DecodeStep.run per
+    #      step (its graph carries the copies, overlapped with the kernels)
     e2e = None
     if not args.no_e2e:
         st = steps[0]

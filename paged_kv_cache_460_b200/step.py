@@ -6,8 +6,11 @@ RoPE + KV append (one fused kernel) and paged attention (one kernel) from one
 CUDA graph, so a step costs one graph launch instead of two kernel launches per
 layer from Python.  The graph
 reads fixed device buffers; `run` copies a step's inputs from (pinned) host memory
-into them, replays the graph and copies the outputs back.  All arithmetic stays in
-the library's kernels; this module only orders the calls.
+into them, replays the graph and copies the outputs back.  With pinned host buffers
+the copies are part of a second graph and overlap the kernels: the layers' q, k, v go
+in on a copy stream in chunks ahead of the compute, and the outputs go back on another
+stream in chunks as their kernels finish.  All arithmetic stays in the library's kernels; this module only orders the
+calls and copies.
 """
 import math
 
@@ -51,6 +54,7 @@ class DecodeStep:
         self.fused = fused
         self.rope = torch.zeros((batch, d // 2, 2), dtype=torch.float64, device=dev) if fused else None
         self.kernels_per_step = (1 + L) if fused else 2 * L
+        self.host_graphs = {}                 # pinned host buffers (data pointers) -> pipelined graph
 
     def layer(self, i, stream=None):
         """Enqueue layer i of the step on the current stream: RoPE + KV append (one
@@ -99,12 +103,91 @@ class DecodeStep:
         self.block_tables.copy_(torch.as_tensor(block_tables), non_blocking=non_blocking)
         self.context_lens.copy_(torch.as_tensor(context_lens), non_blocking=non_blocking)
 
+    def _pinned(self, *ts):
+        return all(isinstance(t, torch.Tensor) and t.device.type == "cpu" and t.is_pinned() and t.is_contiguous()
+                   for t in ts)
+
+    @staticmethod
+    def _chunks(L, growth=4):
+        """Layer ranges [lo, hi) of growing length: 1, 4, 16, ... layers (a layer's rows copy
+        several times faster than its kernels run, so each chunk lands before its first layer)."""
+        out, lo, n = [], 0, 1
+        while lo < L:
+            out.append((lo, min(L, lo + n)))
+            lo, n = lo + n, growth * n
+        return out
+
+    def capture_host(self, q, k, v, out_host):
+        """Record the step with its host copies (pinned q, k, v, out_host of the device
+        buffers' shapes) into one graph.  A copy stream brings the layers' rows in by chunks of
+        growing length (layer 0, then 1-4, 5-20, ...), each chunk's copy running while the
+        kernels of the chunks before it work, and the compute stream waits for a chunk only at
+        its first layer; the outputs go back on a third stream in chunks that shrink toward the
+        last layer, each once its last kernel is done.  Few waits keep most of the layer
+        kernels' programmatic launches chained.  Run the step once outside any capture first
+        (`eager` or `capture`)."""
+        L = self.pool.num_layers
+        if self.graph is None:
+            self.capture()
+        torch.cuda.synchronize()
+        main, h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+        ins = self._chunks(L)
+        outs = [(L - hi, L - lo) for lo, hi in reversed(self._chunks(L))]
+        got = {lo: torch.cuda.Event() for lo, _ in ins}
+        g = torch.cuda.CUDAGraph()
+        main.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(main):
+            with torch.cuda.graph(g, stream=main):
+                h2d.wait_stream(main)                       # fork the copy streams into the capture
+                d2h.wait_stream(main)
+                with torch.cuda.stream(h2d):
+                    for lo, hi in ins:
+                        self.q[lo:hi].copy_(q[lo:hi], non_blocking=True)
+                        self.k[lo:hi].copy_(k[lo:hi], non_blocking=True)
+                        self.v[lo:hi].copy_(v[lo:hi], non_blocking=True)
+                        got[lo].record(h2d)
+                if self.fused:
+                    rope_table(self.context_lens, self.pool.head_dim, self.theta, table=self.rope)
+                ends = {hi - 1: (lo, hi) for lo, hi in outs}
+                for i in range(L):
+                    if i in got:
+                        main.wait_event(got[i])
+                    self.layer(i)
+                    if i in ends:
+                        lo, hi = ends[i]
+                        done = torch.cuda.Event()
+                        done.record(main)
+                        d2h.wait_event(done)
+                        with torch.cuda.stream(d2h):
+                            out_host[lo:hi].copy_(self.out[lo:hi], non_blocking=True)
+                main.wait_stream(h2d)                       # join
+                main.wait_stream(d2h)
+        torch.cuda.current_stream().wait_stream(main)
+        key = (q.data_ptr(), k.data_ptr(), v.data_ptr(), out_host.data_ptr())
+        self.host_graphs[key] = g
+        return g
+
     def run(self, q, k, v, out_host=None):
-        """Copy the step's q, k, v (host, ideally pinned) in, replay, copy out to out_host."""
+        """Copy the step's q, k, v (host, ideally pinned) in, replay, copy out to out_host.
+        Pinned host buffers of the step's shapes (all four) take the pipelined graph, captured
+        on their first use; other inputs are copied in, then the step graph replays."""
+        if out_host is not None and self._pinned(q, k, v, out_host) and q.shape == self.q.shape and \
+                k.shape == self.k.shape and v.shape == self.v.shape and out_host.shape == self.out.shape and \
+                q.dtype == k.dtype == v.dtype == out_host.dtype == self.q.dtype:
+            key = (q.data_ptr(), k.data_ptr(), v.data_ptr(), out_host.data_ptr())
+            g = self.host_graphs.get(key)
+            if g is None:
+                g = self.capture_host(q, k, v, out_host)
+            g.replay()
+            return out_host
+        if self.graph is None:
+            # capture first: its eager pass runs on the buffers as they are, so this step's
+            # inputs go through the kernels once (the two-launch path turns q in place)
+            self.capture()
         self.q.copy_(q, non_blocking=True)
         self.k.copy_(k, non_blocking=True)
         self.v.copy_(v, non_blocking=True)
-        self.replay()
+        self.graph.replay()
         if out_host is not None:
             out_host.copy_(self.out, non_blocking=True)
         return out_host

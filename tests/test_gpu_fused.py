@@ -106,3 +106,37 @@ def test_fused_layer_rejects_what_it_does_not_serve():
     rope = pkv.rope_table(c.cl_t, s.head_dim, s.theta)
     with pytest.raises(pkv.PagedKVError):
         pkv.paged_decode_layer(c.pool, 0, torch.empty_like(q_t), q_t, k_t, v_t, rope, c.bt_t, c.cl_t, c.scale)
+
+
+@pytest.mark.parametrize("fused,workload,layers", [(True, "batch10", 6), (False, "batch10", 3), (True, "cbatch", 2)])
+def test_step_with_pinned_host_buffers_matches_copy_then_replay(fused, workload, layers):
+    """DecodeStep.run with pinned host buffers captures the host copies into the step's graph
+    (layer l's rows copied in on their own stream, its output copied back as soon as its
+    kernels are done) and must give the bits of the plain path: copy everything in, replay
+    the step graph, copy everything out -- output and pool, on the first run and on replays."""
+    s = synth.spec(workload, num_layers=layers)
+    if s.q_heads != s.kv_heads and fused:
+        fused = False                     # the fused layer takes one query head per kv head
+    kp, vp = synth.pool_values_torch(s, "cuda")
+    pools = [pkv.KVPool(kp, vp), pkv.KVPool(kp.clone(), vp.clone())]
+    qs, ks, vs = synth.step_values_torch(s, 2, "cuda")
+    outs = []
+    for pool, pinned in zip(pools, (False, True)):
+        st = DecodeStep(pool, s.batch, s.q_heads, s.max_pages, theta=s.theta, fused=fused)
+        st.set_metadata(s.block_tables, s.context_lens, non_blocking=False)
+        host = [(x[j].cpu().pin_memory() if pinned else x[j].cpu()) for j in range(2) for x in (qs, ks, vs)]
+        hout = torch.empty(st.out.shape, dtype=st.out.dtype)
+        hout = hout.pin_memory() if pinned else hout
+        res = []
+        for it in range(3):               # set 0, set 1, set 0 again: capture, second graph, replay
+            j = it % 2
+            st.run(host[3 * j], host[3 * j + 1], host[3 * j + 2], hout)
+            torch.cuda.synchronize()
+            res.append(hout.clone())
+        assert len(st.host_graphs) == (2 if pinned else 0)
+        outs.append(res)
+    for a, b in zip(*outs):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    assert torch.equal(pools[0].k_cache.view(torch.int16), pools[1].k_cache.view(torch.int16))
+    assert torch.equal(pools[0].v_cache.view(torch.int16), pools[1].v_cache.view(torch.int16))
+    assert pkv.kv_get_device_error() == 0
