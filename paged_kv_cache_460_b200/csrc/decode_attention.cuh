@@ -546,6 +546,7 @@ __global__ void __launch_bounds__(kDecodeThreads, G == 1 ? (kFused ? 3 : 4) : 1)
             if (fids[i / RV] >= 0)
                 cp_async16(reinterpret_cast<unsigned char*>(rope_c) + i * 16,
                            reinterpret_cast<const unsigned char*>(p.rope + (long long)fids[i / RV] * D) + (i % RV) * 16);
+        cp_async_commit();                   // the oldest group: waited for before the PDL wait
     }
     auto rope_row = [&](int bb) -> const double* {
         if constexpr (kFused) {
@@ -581,6 +582,13 @@ __global__ void __launch_bounds__(kDecodeThreads, G == 1 ? (kFused ? 3 : 4) : 1)
         advance();
         cp_async_commit();
     }
+    if constexpr (kFused) {
+        // every warp reads both angle rows: let them land (the m_pre page groups may stay in
+        // flight) and make them visible to the CTA before the wait, so that no CTA barrier
+        // sits between the wait and the first page
+        cp_async_wait_upto(m_pre);
+        __syncthreads();
+    }
 
     pdl_wait();
     pdl_launch_dependents();
@@ -596,14 +604,23 @@ __global__ void __launch_bounds__(kDecodeThreads, G == 1 ? (kFused ? 3 : 4) : 1)
     float* pbuf = pbuf_all + warp * G * P;
     for (int k = 0; k < m_pre; ++k)
         if (pre_qb[k] >= 0) issue_q(k, pre_qb[k], pre_qg[k]);
-    if constexpr (kFused) {                   // the new k, v rows of the kept sequence ends
+    if constexpr (kFused) {
+        // the new k, v rows of the kept sequence ends, each copied by the warp that owns the
+        // sequence's last page (the one that appends it), so only that warp waits for them
         constexpr int NV = D * 2 / 16;        // 16-byte pieces of one row
-        for (int i = tid; i < 4 * NV; i += kDecodeThreads) {
-            const int a = i / (2 * NV), kv = (i / NV) & 1;
-            if (fids[2 + a] >= 0)
-                cp_async16(reinterpret_cast<unsigned char*>(new_c) + i * 16,
+#pragma unroll
+        for (int a = 0; a < 2; ++a) {
+            const int bg = fids[2 + a];
+            if (bg < 0) continue;
+            const int bb = bg / Hkv, gg = bg - bb * Hkv, nb = prefix[bb + 1] - prefix[bb];
+            const long long u_last = (long long)Hkv * prefix[bb] + (long long)gg * nb + nb - 1;
+            if ((int)((u_last - r0) % NW) != warp) continue;
+            for (int i = lane; i < 2 * NV; i += 32) {
+                const int kv = i / NV;
+                cp_async16(reinterpret_cast<unsigned char*>(new_c) + (a * 2 * NV + i) * 16,
                            reinterpret_cast<const unsigned char*>(static_cast<const T*>(kv ? p.v_new : p.k_new) +
-                                                                  (long long)fids[2 + a] * D) + (i % NV) * 16);
+                                                                  (long long)bg * D) + (i % NV) * 16);
+            }
         }
     }
     if (m_pre == DEPTH) cp_async_commit();
@@ -612,7 +629,6 @@ __global__ void __launch_bounds__(kDecodeThreads, G == 1 ? (kFused ? 3 : 4) : 1)
         cp_async_commit();
     }
     cp_async_wait<0>();
-    if constexpr (kFused) __syncthreads();   // the CTA's kept rows, copied by all threads
 
     // ---- compute side.  q.k: lane (t, h) = (lane / 2, lane % 2) dots rows t (and t + 16
     // at P = 32) over chunks h*CPL .. h*CPL+CPL-1; p.V: lane owns output columns
