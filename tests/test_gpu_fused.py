@@ -108,17 +108,26 @@ def test_fused_layer_rejects_what_it_does_not_serve():
         pkv.paged_decode_layer(c.pool, 0, torch.empty_like(q_t), q_t, k_t, v_t, rope, c.bt_t, c.cl_t, c.scale)
 
 
-@pytest.mark.parametrize("fused,workload,layers", [(True, "batch10", 6), (False, "batch10", 3), (True, "cbatch", 2)])
-def test_step_with_pinned_host_buffers_matches_copy_then_replay(fused, workload, layers):
+@pytest.mark.parametrize("fused,workload,layers,kv", [(True, "batch10", 6, "f16"), (False, "batch10", 3, "f16"),
+                                                  (True, "cbatch", 2, "f16"), (True, "batch10", 6, "int8"),
+                                                  (False, "cbatch", 2, "int8")])
+def test_step_with_pinned_host_buffers_matches_copy_then_replay(fused, workload, layers, kv):
     """DecodeStep.run with pinned host buffers captures the host copies into the step's graph
-    (layer l's rows copied in on their own stream, its output copied back as soon as its
-    kernels are done) and must give the bits of the plain path: copy everything in, replay
-    the step graph, copy everything out -- output and pool, on the first run and on replays."""
+    (the layers' rows copied in by chunks on their own stream, the outputs copied back as their
+    kernels finish) and must give the bits of the plain path: copy everything in, replay the
+    step graph, copy everything out -- output and pool, on the first run and on replays; 16-bit
+    and int8 pages, the fused layer and the two-launch step."""
     s = synth.spec(workload, num_layers=layers)
     if s.q_heads != s.kv_heads and fused:
         fused = False                     # the fused layer takes one query head per kv head
-    kp, vp = synth.pool_values_torch(s, "cuda")
-    pools = [pkv.KVPool(kp, vp), pkv.KVPool(kp.clone(), vp.clone())]
+    if kv == "int8":
+        kc, vc, ksc, vsc = synth.pool_values_i8_torch(s, "cuda")
+        tdt = torch.float16 if s.dtype == "f16" else torch.bfloat16
+        pools = [pkv.KVPool(kc, vc, ksc, vsc, dtype=tdt),
+                 pkv.KVPool(kc.clone(), vc.clone(), ksc.clone(), vsc.clone(), dtype=tdt)]
+    else:
+        kp, vp = synth.pool_values_torch(s, "cuda")
+        pools = [pkv.KVPool(kp, vp), pkv.KVPool(kp.clone(), vp.clone())]
     qs, ks, vs = synth.step_values_torch(s, 2, "cuda")
     outs = []
     for pool, pinned in zip(pools, (False, True)):
@@ -137,6 +146,9 @@ def test_step_with_pinned_host_buffers_matches_copy_then_replay(fused, workload,
         outs.append(res)
     for a, b in zip(*outs):
         assert torch.equal(a.view(torch.int16), b.view(torch.int16))
-    assert torch.equal(pools[0].k_cache.view(torch.int16), pools[1].k_cache.view(torch.int16))
-    assert torch.equal(pools[0].v_cache.view(torch.int16), pools[1].v_cache.view(torch.int16))
+    for x, y in ((pools[0].k_cache, pools[1].k_cache), (pools[0].v_cache, pools[1].v_cache)):
+        assert torch.equal(x.view(torch.uint8), y.view(torch.uint8))
+    if kv == "int8":
+        assert torch.equal(pools[0].k_scales, pools[1].k_scales)
+        assert torch.equal(pools[0].v_scales, pools[1].v_scales)
     assert pkv.kv_get_device_error() == 0
